@@ -1,0 +1,194 @@
+/*
+ * csa.h — C ABI of libcsa.so: the forward hot path of a DeepSeek-V4-style
+ * hybrid compressed attention layer (CSA: compressed sparse attention, HCA:
+ * heavily compressed attention, SWA: sliding window, attention sink) on NVIDIA
+ * B200 (sm_100a).
+ *
+ * Sources (secondary write-ups of the DeepSeek-V4 technical report):
+ *   [CS] "DeepSeek V4 脱离 CUDA 全栈国产化：1.6T MoE 逐层拆解 + 昇腾迁移数据",
+ *        §二 "CSA + HCA 混合注意力" (subsections "KV 压缩", "闪电索引器",
+ *        "共享 KV MQA", "HCA（重压缩注意力）", "其他辅助设计").
+ *   [LD] liduos.com "deepseek-v4-engineering-tradeoffs", "1M Context 的结构与取舍".
+ *   [LQ] "Deepseek-V4 技术报告里最值得复现的三个改动", §3 (config block), §5.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *     allocates no memory.  Scratch comes from a caller-supplied workspace whose
+ *     size is queried first.
+ *   - Tensors are dense row-major with the channel dimension innermost.  Every
+ *     base pointer must be 16-byte aligned; row lengths in bytes must be
+ *     multiples of 16.
+ *   - dtype codes: CSA_F32 (float), CSA_BF16 (__nv_bfloat16), CSA_E4M3 (OCP FP8
+ *     E4M3 "fn" byte).
+ *   - Sequences: n_seq independent sequences; sequence b has T query tokens at
+ *     absolute positions q_pos[b] + t (q_pos is a DEVICE int64 array [n_seq]).
+ *     Per-sequence caches are strided by a row capacity `cap` (rows).
+ *   - Compressed entry i of a sequence (compression ratio m) covers tokens
+ *     [i*m, (i+1)*m) and is visible to the query at position p iff
+ *     (i+1)*m - 1 <= p, i.e. n_vis(p) = min(cap, (p+1)/m).
+ *   - All calls are asynchronous on `stream` and never abort.  Argument errors
+ *     are reported before any launch; csa_last_error() describes the last
+ *     failure.  Kernels that wait on on-chip barriers bound every wait and
+ *     report expiry through the device error word (csa_check_device_error).
+ *   - Results do not depend on batch position or launch geometry: no floating-
+ *     point atomics are used (batch invariance, [CS] §八).
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or flag */
+  CSA_ERR_UNSUPPORTED = 2,   /* valid but unsupported shape/dtype combination */
+  CSA_ERR_WORKSPACE = 3,     /* workspace missing or too small */
+  CSA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  CSA_ERR_TIMEOUT = 5,       /* a bounded on-chip wait expired (device error word) */
+  CSA_ERR_DEVICE = 6         /* a kernel recorded a bad gather index */
+} csa_status_t;
+
+typedef enum { CSA_F32 = 0, CSA_BF16 = 1, CSA_E4M3 = 2 } csa_dtype_t;
+
+/* ABI version of this header (incremented on any signature change). */
+int csa_abi_version(void);
+
+/* Text of a status code, and a description of the most recent failure on the
+ * calling thread (empty string if none).  Both pointers stay valid. */
+const char* csa_status_string(csa_status_t s);
+const char* csa_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the device error words of the
+ * current device.  Returns CSA_ERR_TIMEOUT or CSA_ERR_DEVICE if a kernel
+ * recorded an expired wait or a bad gather index since the last check. */
+csa_status_t csa_check_device_error(cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * csa_compress — softmax-gated KV compressor ([CS] "KV 压缩": an entry is the
+ * per-channel Softmax(Z + B)-weighted sum of the content C over its block; CSA
+ * blocks overlap the previous block, m = 4; HCA ([CS] "HCA") uses
+ * non-overlapping m' = 128 blocks).  Tokens that do not fill a block form no
+ * entry ([LQ] §5).
+ *
+ *   C, Z     [S, D] in_dtype (F32 or BF16): content and gate logits (stream a).
+ *   Cb, Zb   previous-block stream [S, D] or NULL to reuse C, Z.
+ *   B        [2m, D] fp32 if overlap (rows 0..m-1 weight the previous block,
+ *            rows m..2m-1 the current block) else [m, D]; NULL = zero bias.
+ *   overlap  1: entry i pools tokens [(i-1)m, (i+1)m) in ONE joint per-channel
+ *            softmax (entry 0: its own block only); 0: tokens [i*m, (i+1)m).
+ *   norm     1: RMSNorm over D (eps, unit gain) after pooling ([CS] "其他辅助设计").
+ *   rope_dim RoPE on the last rope_dim dims (0 = off), entry i at position
+ *            i*m, pairs (d, d + rope_dim/2), theta_j = rope_base^(-2j/rope_dim).
+ *   out      [S/m, D] out_dtype (F32 or BF16).
+ * Requires D % 8 == 0, 8 <= D <= 2048, 1 <= m <= 1024, S >= 0.
+ * ------------------------------------------------------------------------- */
+csa_status_t csa_compress(const void* C, const void* Z, const void* Cb, const void* Zb,
+                          const float* B, int64_t S, int D, int m, int overlap,
+                          csa_dtype_t in_dtype, int norm, int rope_dim, float rope_base,
+                          float eps, void* out, csa_dtype_t out_dtype, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * csa_rmsnorm_rope — QK normalisation and partial RoPE of raw rows ([CS]
+ * "其他辅助设计": RMSNorm before core attention, RoPE on the last 64 dims).
+ * Used for the queries (rows_per_pos = H heads share a position) and for the
+ * raw window rows (rows_per_pos = 1).
+ *   x   [rows, D] in_dtype; row r has position pos0 + r / rows_per_pos.
+ *   out [rows, D] out_dtype.  norm, rope_dim, rope_base, eps as in csa_compress.
+ * ------------------------------------------------------------------------- */
+csa_status_t csa_rmsnorm_rope(const void* x, csa_dtype_t in_dtype, int64_t rows, int D,
+                              int rows_per_pos, int64_t pos0, int norm, int rope_dim,
+                              float rope_base, float eps, void* out, csa_dtype_t out_dtype,
+                              cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * csa_index_topk — lightning indexer + top-k ([CS] "闪电索引器": index heads,
+ * ReLU of the similarity, weighted over heads; only the top-k entries are kept
+ * for the query, [LD]).  For query token t of sequence b at p = q_pos[b] + t:
+ *     I[s] = ks[s] * sum_h (w[h] * qs[h]) * ReLU(qI[h,:] . kI[s,:]),  s < n_vis(p)
+ * computed with FP8 (e4m3) tensor-core products accumulated in fp32; the row
+ * scales factor out of the ReLU because they are positive.  idx receives the
+ * min(k, n_vis) entries with the largest I, equal scores going to the lower
+ * entry index, in ascending order, padded with -1.
+ *
+ *   qI       [n_seq, T, HI, DI] e4m3     qI_scale [n_seq, T, HI] fp32 or NULL (1)
+ *   w        [n_seq, T, HI] fp32 head weights
+ *   kI       [n_seq, cap, DI] e4m3       kI_scale [n_seq, cap] fp32 or NULL (1)
+ *   q_pos    [n_seq] int64 (device)
+ *   idx      [n_seq, T, k] int32 out
+ *   workspace / ws_bytes: at least csa_index_topk_workspace(n_seq, T, cap, k).
+ * Requires DI in {32, 64, 128}; HI in {1,2,4,...,64} (power of two <= 64 whose
+ * product with the token block is a multiple of 16); 1 <= k <= 2048; cap >= 1.
+ * ------------------------------------------------------------------------- */
+size_t csa_index_topk_workspace(int n_seq, int T, int64_t cap, int k);
+csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale, const float* w,
+                            const uint8_t* kI, const float* kI_scale, const int64_t* q_pos,
+                            int n_seq, int T, int HI, int DI, int64_t cap, int m, int k,
+                            int32_t* idx, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Attention over one shared K = V row set per query token ([CS] "共享 KV MQA":
+ * the selected compressed entries act as both key and value; one KV head
+ * shared by H query heads).  Logits are scale * q_h . row; softmax over the
+ * row set.  Rows come from a KV store that is either
+ *   kv_dtype BF16 / F32 : kv [n_seq, cap, D]
+ *   kv_dtype E4M3       : kv [n_seq, cap, D - rope_dim] e4m3 codes (dequantised
+ *                         as code * kv_scale[row]) + kv_rope [n_seq, cap, rope_dim]
+ *                         bf16 ([CS] "其他辅助设计": RoPE dims BF16, rest FP8).
+ * q [n_seq, T, H, D] (q_dtype BF16 or F32) is already normalised and rotated.
+ * Outputs of the two partial calls: O_part [n_seq, T, H, D] fp32 normalised by
+ * the branch's own softmax sum, lse_part [n_seq, T, H] fp32 natural-log
+ * log-sum-exp of the branch logits (-inf and O = 0 when the set is empty).
+ * Computation: BF16 tensor-core products (F32 inputs are rounded to BF16),
+ * fp32 accumulation and softmax.  Requires D in {128, 512}, H <= 64,
+ * rope_dim in {0, 64} (E4M3 needs 64).
+ * ------------------------------------------------------------------------- */
+
+/* csa_sparse_mqa — CSA main branch: rows kv[b, idx[b,t,j]] for idx >= 0.
+ *   idx [n_seq, T, k] int32, ascending, -1 padded (as produced by csa_index_topk).
+ *   An index >= cap is ignored and recorded as CSA_ERR_DEVICE. */
+csa_status_t csa_sparse_mqa(const void* q, csa_dtype_t q_dtype, const void* kv,
+                            csa_dtype_t kv_dtype, const void* kv_rope, const float* kv_scale,
+                            int64_t cap, const int32_t* idx, int k, int n_seq, int T, int H,
+                            int D, int rope_dim, float scale, float* O_part, float* lse_part,
+                            cudaStream_t stream);
+
+/* hca_dense_attn — HCA main branch ([CS] "HCA": no selection, dense attention
+ * over all heavily compressed entries): rows kv[b, 0 : n_vis(q_pos[b]+t)] with
+ * compression ratio m (entries complete at the query position). */
+csa_status_t hca_dense_attn(const void* q, csa_dtype_t q_dtype, const void* kv,
+                            csa_dtype_t kv_dtype, const void* kv_rope, const float* kv_scale,
+                            int64_t cap, const int64_t* q_pos, int m, int n_seq, int T, int H,
+                            int D, int rope_dim, float scale, float* O_part, float* lse_part,
+                            cudaStream_t stream);
+
+/* swa_sink_combine — sliding window + attention sink + merge ([LD]: a
+ * 128-token uncompressed window joins the attention; the sink lets a head
+ * abstain; [CS] "HCA": an uncompressed 128-window is kept next to the
+ * compressed branch).  For each query token:
+ *   window rows  window_mode 0 (prefill): kv_tok[b, u] for u in [max(0,p-W+1), p]
+ *                window_mode 1 (decode) : kv_tok[b, 0 : min(W, p+1)], a cache
+ *                of the newest tokens in position order, newest included.
+ *   out = (e^{lse_part-M} O_part + sum_w e^{l_w-M} v_w) /
+ *         (e^{lse_part-M} + sum_w e^{l_w-M} + e^{sink_h-M})      (one softmax)
+ *   then, if inv_rope, the last rope_dim dims of out are rotated by -p ([LD]:
+ *   inverse RoPE on the output side).  O_part / lse_part may be NULL (no
+ *   compressed branch).  kv_tok has dtype kv_dtype (BF16 or F32), [n_seq, cap, D].
+ *   out [n_seq, T, H, D] out_dtype (F32 or BF16).
+ * ------------------------------------------------------------------------- */
+csa_status_t swa_sink_combine(const void* q, csa_dtype_t q_dtype, const void* kv_tok,
+                              csa_dtype_t kv_dtype, int64_t cap, const int64_t* q_pos, int W,
+                              int window_mode, const float* sink, const float* O_part,
+                              const float* lse_part, int n_seq, int T, int H, int D,
+                              int rope_dim, float rope_base, int inv_rope, float scale,
+                              void* out, csa_dtype_t out_dtype, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H_ */

@@ -1,0 +1,249 @@
+"""Python binding of libcsa.so (CSA / HCA hybrid compressed attention on B200).
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels
+behind the C ABI declared in include/csa.h.  torch supplies device memory and
+the current stream.  There is no fallback: if libcsa.so is missing or a call
+fails, an exception is raised.
+
+Entry points (same names as the C ABI):
+  csa_compress, csa_rmsnorm_rope, csa_index_topk, csa_sparse_mqa,
+  hca_dense_attn, swa_sink_combine
+and two compositions of them: csa_layer_prefill, hca_layer_prefill.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+F32, BF16, E4M3 = 0, 1, 2
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.uint8: E4M3}
+
+_lib = None
+
+
+class CsaError(RuntimeError):
+    pass
+
+
+def lib():
+    """Loads libcsa.so once and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise CsaError(f"{LIB_PATH} is not built; run `python -m long_context_compressed_02_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "csa_abi_version": ([], I),
+        "csa_status_string": ([I], ctypes.c_char_p),
+        "csa_last_error": ([], ctypes.c_char_p),
+        "csa_check_device_error": ([P], I),
+        "csa_compress": ([P, P, P, P, P, I64, I, I, I, I, I, I, F, F, P, I, P], I),
+        "csa_rmsnorm_rope": ([P, I, I64, I, I, I64, I, I, F, F, P, I, P], I),
+        "csa_index_topk_workspace": ([I, I, I64, I], SZ),
+        "csa_index_topk": ([P, P, P, P, P, P, I, I, I, I, I64, I, I, P, P, SZ, P], I),
+        "csa_sparse_mqa": ([P, I, P, I, P, P, I64, P, I, I, I, I, I, I, F, P, P, P], I),
+        "hca_dense_attn": ([P, I, P, I, P, P, I64, P, I, I, I, I, I, I, F, P, P, P], I),
+        "swa_sink_combine": ([P, I, P, I, I64, P, I, I, P, P, P, I, I, I, I, I, F, I, F, P, I, P], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def _check(status, what):
+    if status != 0:
+        L = lib()
+        raise CsaError(f"{what}: {L.csa_status_string(status).decode()}: {L.csa_last_error().decode()}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, name):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise CsaError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise CsaError(f"{name} must be contiguous")
+
+
+def check_device_error(stream=None):
+    """Synchronises the stream and raises if a kernel recorded an error."""
+    _check(lib().csa_check_device_error(_stream(stream)), "csa_check_device_error")
+
+
+# ---------------------------------------------------------------- steps
+
+def csa_compress(C, Z, B, m, overlap, *, Cb=None, Zb=None, norm=False, rope_dim=0, rope_base=10000.0,
+                 eps=1e-6, out_dtype=None, out=None, stream=None):
+    """Softmax-gated block compressor: [S, D] -> [S // m, D]."""
+    for t, n in ((C, "C"), (Z, "Z"), (B, "B"), (Cb, "Cb"), (Zb, "Zb")):
+        _dev(t, n)
+    S, D = C.shape
+    out_dtype = C.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((S // m, D), dtype=out_dtype, device=C.device)
+    _check(lib().csa_compress(_ptr(C), _ptr(Z), _ptr(Cb), _ptr(Zb), _ptr(B), S, D, m, int(overlap),
+                              _DT[C.dtype], int(norm), rope_dim, rope_base, eps, _ptr(out), _DT[out.dtype],
+                              _stream(stream)), "csa_compress")
+    return out
+
+
+def csa_rmsnorm_rope(x, rows_per_pos=1, pos0=0, *, norm=True, rope_dim=64, rope_base=10000.0, eps=1e-6,
+                     out_dtype=None, out=None, stream=None):
+    """RMSNorm + partial RoPE of rows; x [..., D], rows_per_pos rows share a position."""
+    _dev(x, "x")
+    D = x.shape[-1]
+    rows = x.numel() // D
+    out_dtype = x.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype, device=x.device)
+    _check(lib().csa_rmsnorm_rope(_ptr(x), _DT[x.dtype], rows, D, rows_per_pos, pos0, int(norm), rope_dim,
+                                  rope_base, eps, _ptr(out), _DT[out.dtype], _stream(stream)), "csa_rmsnorm_rope")
+    return out
+
+
+def csa_index_topk_workspace(n_seq, T, cap, k):
+    return int(lib().csa_index_topk_workspace(n_seq, T, cap, k))
+
+
+def csa_index_topk(qI, w, kI, q_pos, m, k, *, qI_scale=None, kI_scale=None, workspace=None, idx=None,
+                   stream=None):
+    """Lightning indexer + top-k.  qI [n_seq, T, HI, DI] uint8 (e4m3 codes),
+    w [n_seq, T, HI] f32, kI [n_seq, cap, DI] uint8, q_pos [n_seq] int64.
+    Returns idx [n_seq, T, k] int32 (ascending, -1 padded)."""
+    for t, n in ((qI, "qI"), (w, "w"), (kI, "kI"), (q_pos, "q_pos"), (qI_scale, "qI_scale"), (kI_scale, "kI_scale")):
+        _dev(t, n)
+    n_seq, T, HI, DI = qI.shape
+    cap = kI.shape[1]
+    need = csa_index_topk_workspace(n_seq, T, cap, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=qI.device)
+    if idx is None:
+        idx = torch.empty((n_seq, T, k), dtype=torch.int32, device=qI.device)
+    _check(lib().csa_index_topk(_ptr(qI), _ptr(qI_scale), _ptr(w), _ptr(kI), _ptr(kI_scale), _ptr(q_pos),
+                                n_seq, T, HI, DI, cap, m, k, _ptr(idx), _ptr(workspace), workspace.numel(),
+                                _stream(stream)), "csa_index_topk")
+    return idx
+
+
+def _kv_args(kv, kv_rope, kv_scale):
+    return _DT[kv.dtype], _ptr(kv), _ptr(kv_rope), _ptr(kv_scale)
+
+
+def csa_sparse_mqa(q, kv, idx, *, kv_rope=None, kv_scale=None, scale=None, rope_dim=None, out=None,
+                   stream=None):
+    """Sparse shared-KV MQA over kv[b, idx[b, t, :]].  q [n_seq, T, H, D];
+    kv [n_seq, cap, D] (bf16/f32) or e4m3 [n_seq, cap, D-64] + kv_rope + kv_scale.
+    Returns (O_part [n_seq, T, H, D] f32, lse_part [n_seq, T, H] f32)."""
+    for t, n in ((q, "q"), (kv, "kv"), (idx, "idx"), (kv_rope, "kv_rope"), (kv_scale, "kv_scale")):
+        _dev(t, n)
+    n_seq, T, H, D = q.shape
+    cap = kv.shape[1]
+    k = idx.shape[-1]
+    rope_dim = (64 if kv.dtype == torch.uint8 else 0) if rope_dim is None else rope_dim
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    O = torch.empty((n_seq, T, H, D), dtype=torch.float32, device=q.device) if out is None else out[0]
+    L = torch.empty((n_seq, T, H), dtype=torch.float32, device=q.device) if out is None else out[1]
+    kvd, kvp, kvr, kvs = _kv_args(kv, kv_rope, kv_scale)
+    _check(lib().csa_sparse_mqa(_ptr(q), _DT[q.dtype], kvp, kvd, kvr, kvs, cap, _ptr(idx), k, n_seq, T, H, D,
+                                rope_dim, scale, _ptr(O), _ptr(L), _stream(stream)), "csa_sparse_mqa")
+    return O, L
+
+
+def hca_dense_attn(q, kv, q_pos, m, *, kv_rope=None, kv_scale=None, scale=None, rope_dim=None, out=None,
+                   stream=None):
+    """Dense causal attention over the complete m-entries kv[b, :n_vis]."""
+    for t, n in ((q, "q"), (kv, "kv"), (q_pos, "q_pos"), (kv_rope, "kv_rope"), (kv_scale, "kv_scale")):
+        _dev(t, n)
+    n_seq, T, H, D = q.shape
+    cap = kv.shape[1]
+    rope_dim = (64 if kv.dtype == torch.uint8 else 0) if rope_dim is None else rope_dim
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    O = torch.empty((n_seq, T, H, D), dtype=torch.float32, device=q.device) if out is None else out[0]
+    L = torch.empty((n_seq, T, H), dtype=torch.float32, device=q.device) if out is None else out[1]
+    kvd, kvp, kvr, kvs = _kv_args(kv, kv_rope, kv_scale)
+    _check(lib().hca_dense_attn(_ptr(q), _DT[q.dtype], kvp, kvd, kvr, kvs, cap, _ptr(q_pos), m, n_seq, T, H, D,
+                                rope_dim, scale, _ptr(O), _ptr(L), _stream(stream)), "hca_dense_attn")
+    return O, L
+
+
+def swa_sink_combine(q, kv_tok, q_pos, W, sink, O_part=None, lse_part=None, *, window_mode=0, inv_rope=False,
+                     rope_dim=64, rope_base=10000.0, scale=None, out_dtype=None, out=None, stream=None):
+    """Window attention + sink + merge with the compressed-branch partial."""
+    for t, n in ((q, "q"), (kv_tok, "kv_tok"), (q_pos, "q_pos"), (sink, "sink"), (O_part, "O_part"),
+                 (lse_part, "lse_part")):
+        _dev(t, n)
+    n_seq, T, H, D = q.shape
+    cap = kv_tok.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((n_seq, T, H, D), dtype=out_dtype, device=q.device)
+    _check(lib().swa_sink_combine(_ptr(q), _DT[q.dtype], _ptr(kv_tok), _DT[kv_tok.dtype], cap, _ptr(q_pos), W,
+                                  window_mode, _ptr(sink), _ptr(O_part), _ptr(lse_part), n_seq, T, H, D,
+                                  rope_dim, rope_base, int(inv_rope), scale,
+                                  _ptr(out), _DT[out.dtype], _stream(stream)), "swa_sink_combine")
+    return out
+
+
+# ---------------------------------------------------------------- layers
+
+def csa_layer_prefill(q, C, Z, B, qI, w, kI, sink, *, k, m=4, W=128, norm_rope=False, inv_rope=False,
+                      rope_dim=64, rope_base=10000.0, kv_dtype=None, workspace=None, return_idx=False):
+    """One CSA layer (batch 1): compress -> index/top-k -> sparse MQA -> window + sink.
+    q [S, H, D], C/Z [S, D], B [2m, D] f32, qI [S, HI, DI] u8, w [S, HI], kI [S//m, DI] u8, sink [H]."""
+    S, H, D = q.shape
+    dev = q.device
+    kv_dtype = q.dtype if kv_dtype is None else kv_dtype
+    pos = torch.zeros(1, dtype=torch.int64, device=dev)
+    if norm_rope:
+        qn = csa_rmsnorm_rope(q, rows_per_pos=H, rope_dim=rope_dim, rope_base=rope_base)
+        kt = csa_rmsnorm_rope(C, rows_per_pos=1, rope_dim=rope_dim, rope_base=rope_base, out_dtype=kv_dtype)
+        kv = csa_compress(C, Z, B, m, True, norm=True, rope_dim=rope_dim, rope_base=rope_base, out_dtype=kv_dtype)
+    else:
+        qn, kt = q, C
+        kv = csa_compress(C, Z, B, m, True, out_dtype=kv_dtype)
+    idx = csa_index_topk(qI[None], w[None], kI[None], pos, m, k, workspace=workspace)
+    Op, Lp = csa_sparse_mqa(qn[None], kv[None], idx)
+    out = swa_sink_combine(qn[None], kt[None], pos, W, sink, Op, Lp, window_mode=0, inv_rope=inv_rope,
+                           rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
+    return (out[0], idx[0]) if return_idx else out[0]
+
+
+def hca_layer_prefill(q, C, Z, B, sink, *, m=128, W=128, norm_rope=False, inv_rope=False, rope_dim=64,
+                      rope_base=10000.0, kv_dtype=None):
+    """One HCA layer (batch 1): compress (m' = 128) -> dense attention -> window + sink."""
+    S, H, D = q.shape
+    dev = q.device
+    kv_dtype = q.dtype if kv_dtype is None else kv_dtype
+    pos = torch.zeros(1, dtype=torch.int64, device=dev)
+    if norm_rope:
+        qn = csa_rmsnorm_rope(q, rows_per_pos=H, rope_dim=rope_dim, rope_base=rope_base)
+        kt = csa_rmsnorm_rope(C, rows_per_pos=1, rope_dim=rope_dim, rope_base=rope_base, out_dtype=kv_dtype)
+        kv = csa_compress(C, Z, B, m, False, norm=True, rope_dim=rope_dim, rope_base=rope_base, out_dtype=kv_dtype)
+    else:
+        qn, kt = q, C
+        kv = csa_compress(C, Z, B, m, False, out_dtype=kv_dtype)
+    Op, Lp = hca_dense_attn(qn[None], kv[None], pos, m)
+    out = swa_sink_combine(qn[None], kt[None], pos, W, sink, Op, Lp, window_mode=0, inv_rope=inv_rope,
+                           rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
+    return out[0]

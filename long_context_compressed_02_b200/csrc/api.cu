@@ -1,0 +1,48 @@
+// Status reporting shared by all entry points of libcsa.so.
+#include <string>
+#include "common.cuh"
+
+namespace csa {
+
+static thread_local std::string g_last_error;
+
+csa_status_t fail(csa_status_t s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+void clear_error() { g_last_error.clear(); }
+
+}  // namespace csa
+
+extern "C" int csa_abi_version(void) { return 1; }
+
+extern "C" const char* csa_status_string(csa_status_t s) {
+  switch (s) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID_ARG: return "CSA_ERR_INVALID_ARG";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
+    case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+    case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT";
+    case CSA_ERR_DEVICE: return "CSA_ERR_DEVICE";
+  }
+  return "CSA_UNKNOWN_STATUS";
+}
+
+extern "C" const char* csa_last_error(void) { return csa::g_last_error.c_str(); }
+
+extern "C" csa_status_t csa_check_device_error(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess)
+    return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: stream sync failed: %s", cudaGetErrorString(e));
+  uint32_t w = csa::read_clear_err_indexer() | csa::read_clear_err_attention();
+  if (w & 1u) return csa::fail(CSA_ERR_TIMEOUT, "a bounded on-chip wait expired (device error word 0x%x)", w);
+  if (w) return csa::fail(CSA_ERR_DEVICE, "a kernel recorded an out-of-range gather index (device error word 0x%x)", w);
+  return CSA_OK;
+}

@@ -1,0 +1,719 @@
+// Shared-K=V multi-query attention over a per-token row set, on tcgen05 tensor
+// cores: the CSA sparse branch, the HCA dense branch and the sliding window
+// with the attention sink.
+//
+// "DeepSeek V4 脱离 CUDA 全栈国产化：1.6T MoE 逐层拆解 + 昇腾迁移数据", §二:
+//   "共享 KV MQA" — the selected compressed entries serve as both key and value
+//                   in multi-query attention;
+//   "HCA（重压缩注意力）" — dense attention over all heavily compressed entries,
+//                   plus an uncompressed 128-token window.
+// liduos.com "1M Context 的结构与取舍": the SWA channel keeps the newest 128
+// raw tokens; the attention sink lets a head abstain; partial RoPE with an
+// inverse RoPE applied on the output side.
+//
+// Design (one query token = 64 query rows: its heads, zero-padded):
+//   S^T[row, head] = KV_chunk[128 rows, D] . Q[64, D]^T     M=128, N=64, K=D
+//   O^T[d, head]  += KV_chunk^T[d, 128 rows] . P^T[rows, 64]  M=128 per 128-d tile
+// Both products are BF16 kind::f16 MMAs with fp32 accumulators in TMEM, so
+// every MMA has M = 128 (the full tensor-core height) while a token's 64 heads
+// sit on N.  K = V: the SAME shared-memory chunk is the K-major A operand of
+// the first product and, read through an MN-major descriptor, the A operand
+// of the second; nothing is transposed or copied.  Softmax runs over TMEM
+// lanes (rows) per column (head): column maxima and sums use warp
+// transpose-reductions plus a 4-warp exchange; the running max is only raised
+// when it grows by more than 2^8, so O^T is rarely rescaled.
+//
+// Roles (288 threads): warps 0-3 softmax + epilogue (one TMEM lane each),
+// warps 4-7 loaders (one chunk row each: gather through cp.async, or
+// load-convert for fp32 / e4m3 stores), warp 8 TMEM allocation + MMA issue.
+// The chunk buffer is loaded slab by slab (64 columns = 128 bytes, 128-byte
+// swizzle) and a slab pair is refilled as soon as the PV MMA of its 128-column
+// tile retires, so loads overlap the tail of the previous chunk's MMAs.
+#include <algorithm>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <math_constants.h>
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace csa {
+
+static __device__ uint32_t g_err_attn;
+
+uint32_t read_clear_err_attention() {
+  uint32_t v = 0, z = 0;
+  cudaMemcpyFromSymbol(&v, g_err_attn, sizeof(v));
+  cudaMemcpyToSymbol(g_err_attn, &z, sizeof(z));
+  return v;
+}
+
+namespace {
+
+constexpr int kThreads = 288;
+constexpr int kNQ = 64;            // query rows (heads) per tile = MMA N
+constexpr int kRows = 128;         // KV rows per chunk = MMA M
+constexpr float kTau = 8.0f;       // lazy-rescale threshold (log2 units)
+constexpr float kLn2 = 0.6931471805599453f;
+
+enum KvKind { KV_BF16 = 0, KV_F32 = 1, KV_FP8 = 2 };
+enum EpiMode { EPI_PARTIAL = 0, EPI_COMBINE = 1 };
+enum RowKind { ROWS_GATHER = 0, ROWS_DENSE = 1, ROWS_WINDOW = 2, ROWS_CACHE = 3 };
+
+struct AttnParams {
+  const void* q;            // [n_seq, T, H, D] bf16 or f32
+  int q_f32;
+  const void* kv;           // bf16/f32 [n_seq, cap, D] or e4m3 [n_seq, cap, D - rope_dim]
+  const __nv_bfloat16* kv_rope;   // e4m3 store: [n_seq, cap, rope_dim]
+  const float* kv_scale;          // e4m3 store: [n_seq, cap]
+  int64_t cap;
+  const int32_t* idx;       // gather: [n_seq, T, k]
+  int k;
+  const int64_t* q_pos;     // [n_seq]
+  int row_kind, m, W;
+  int n_seq, T, H;
+  float scale_log2;
+  float* O_part;            // partial outputs
+  float* lse_part;
+  const float* O_in;        // combine inputs (may be null)
+  const float* lse_in;
+  const float* sink;        // [H] or null
+  void* out;
+  int out_bf16, inv_rope, rope_dim;
+  float rope_base;
+};
+
+struct RowSet {
+  int64_t lo;               // range modes: first KV row
+  int n;                    // rows in the set
+  const int32_t* idx;       // gather mode: row list
+};
+
+__device__ __forceinline__ RowSet row_set(const AttnParams& p, int b, int t) {
+  RowSet r{0, 0, nullptr};
+  const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
+  if (p.row_kind == ROWS_GATHER) {
+    const int32_t* row = p.idx + ((int64_t)b * p.T + t) * p.k;
+    int lo = 0, hi = p.k;                      // first -1 of an ascending, -1 padded list
+    while (lo < hi) { int mid = (lo + hi) >> 1; if (row[mid] >= 0) lo = mid + 1; else hi = mid; }
+    r.idx = row; r.n = lo;
+  } else if (p.row_kind == ROWS_DENSE) {
+    r.lo = 0; r.n = (int)min(p.cap, (pos + 1) / p.m);
+  } else if (p.row_kind == ROWS_WINDOW) {
+    int64_t lo = max((int64_t)0, pos - p.W + 1), hi = min(p.cap, pos + 1);
+    r.lo = lo; r.n = (int)max((int64_t)0, hi - lo);
+  } else {
+    r.lo = 0; r.n = (int)min(min((int64_t)p.W, p.cap), pos + 1);
+  }
+  return r;
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  uint64_t start = 0;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0) {
+      if (*abort_flag) return false;
+      const uint64_t now = global_ns();
+      if (start == 0) start = now;
+      else if (now - start > kWaitNs) break;
+    }
+  }
+  *abort_flag = 1;
+  atomicOr(&g_err_attn, DEV_ERR_TIMEOUT_MBAR);
+  return false;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 8 consecutive values -> one 16-byte chunk of bf16
+__device__ __forceinline__ uint4 to_bf16x8(const float* v) {
+  return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+}
+
+__device__ __forceinline__ void st_shared16(uint8_t* dst, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" :: "r"(smem_u32(dst)), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// e4m3 x 16 -> 16 floats (hardware conversion through f16x2)
+__device__ __forceinline__ void e4m3x16_to_float(uint4 raw, float scale, float* out) {
+  const uint16_t* pr = reinterpret_cast<const uint16_t*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)pr[i], __NV_E4M3);
+    __half2 hh = *reinterpret_cast<__half2*>(&h2);
+    float2 f = __half22float2(hh);
+    out[2 * i] = f.x * scale;
+    out[2 * i + 1] = f.y * scale;
+  }
+}
+
+// Loads the 64-column slab `s` of KV row `row` (or zeros) into row `r` of a
+// 128-byte-swizzled slab buffer.  BF16 rows use cp.async (caller commits).
+template <int D, int KV>
+__device__ __forceinline__ void load_kv_slab(const AttnParams& p, int b, int64_t row, bool valid, int s,
+                                             uint8_t* slab_base, int r) {
+  if constexpr (KV == KV_BF16) {
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kv) +
+                         ((((int64_t)b * p.cap + (valid ? row : 0)) * D + 64 * s) * 2);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) cp_async16(slab_base + swz128(r, q), src + 16 * q, valid ? 16u : 0u);
+  } else if constexpr (KV == KV_F32) {
+    const float* src = reinterpret_cast<const float*>(p.kv) + ((int64_t)b * p.cap + (valid ? row : 0)) * D + 64 * s;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float v[8];
+      if (valid) {
+        float4 a = __ldg(reinterpret_cast<const float4*>(src + 8 * q));
+        float4 c = __ldg(reinterpret_cast<const float4*>(src + 8 * q) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      }
+      st_shared16(slab_base + swz128(r, q), to_bf16x8(v));
+    }
+  } else {
+    const int nope = D - p.rope_dim;           // rope_dim == 64: last slab is the bf16 RoPE part
+    if (64 * s < nope) {
+      float v[64];
+      if (valid) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kv) + ((int64_t)b * p.cap + row) * nope + 64 * s;
+        const float sc = p.kv_scale[(int64_t)b * p.cap + row];
+        uint4 raw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) raw[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) e4m3x16_to_float(raw[i], sc, v + 16 * i);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) st_shared16(slab_base + swz128(r, q), to_bf16x8(v + 8 * q));
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(p.kv_rope + ((int64_t)b * p.cap + (valid ? row : 0)) * p.rope_dim);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) st_shared16(slab_base + swz128(r, q), valid ? __ldg(src + q) : make_uint4(0, 0, 0, 0));
+    }
+  }
+}
+
+template <int D, int KV, int EPI>
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
+  constexpr int NS = D / 64;                 // 128-byte slabs per row
+  constexpr int NT = D / 128;                // O^T tiles
+  constexpr uint32_t kQSlab = kNQ * 128;     // 8 KB
+  constexpr uint32_t kKSlab = kRows * 128;   // 16 KB
+  constexpr uint32_t kTmemCols = (64 + 64 * NT) <= 128 ? 128 : ((64 + 64 * NT) <= 256 ? 256 : 512);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + NS * kQSlab;
+  uint8_t* sP = sKV + NS * kKSlab;
+  float* s_red = reinterpret_cast<float*>(sP + kRows * 128);   // [2][4][64] column partials
+  float* s_bc = s_red + 2 * 4 * 64;                              // [4 warps][3][64] broadcasts
+  float2* s_cs = reinterpret_cast<float2*>(s_bc + 4 * 3 * 64);  // [2][32] inverse-RoPE cos/sin
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_cs + 64);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_free = bars + 1;
+  uint64_t* s_done = bars + 2;
+  uint64_t* p_full = bars + 3;
+  uint64_t* epi_done = bars + 4;
+  uint64_t* kv_full = bars + 5;              // [NS]
+  uint64_t* pv_done = kv_full + NS;          // [NT]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(pv_done + NT);
+  int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(q_full, 128); mbar_init(q_free, 1); mbar_init(s_done, 1);
+    mbar_init(p_full, 128); mbar_init(epi_done, 128);
+    for (int s = 0; s < NS; ++s) mbar_init(&kv_full[s], 128);
+    for (int t = 0; t < NT; ++t) mbar_init(&pv_done[t], 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) tmem_alloc(s_tmem, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  volatile int* abort_flag = s_abort;
+  const int64_t n_items = (int64_t)p.n_seq * p.T;
+
+  if (warp >= 4 && warp < 8) {
+    // ============================ loaders
+    const int lt = tid - 128;
+    uint32_t g = 0, qcount = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int b = (int)(item / p.T), t = (int)(item % p.T);
+      const RowSet rs = row_set(p, b, t);
+      if (rs.n == 0) continue;
+      // ---- Q tile: 64 rows x NS slabs of 128 B
+      if (!wait_bar(q_free, (qcount & 1) ^ 1, abort_flag)) { ok = false; break; }
+      ++qcount;
+      for (int u = lt; u < kNQ * NS; u += 128) {
+        const int r = u % kNQ, s = u / kNQ;
+        uint8_t* dst = sQ + s * kQSlab;
+        const bool v = r < p.H;
+        const int64_t qrow = ((int64_t)b * p.T + t) * p.H + (v ? r : 0);
+        if (p.q_f32) {
+          const float* src = reinterpret_cast<const float*>(p.q) + qrow * D + 64 * s;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float x[8];
+            if (v) {
+              float4 a = __ldg(reinterpret_cast<const float4*>(src + 8 * q));
+              float4 c = __ldg(reinterpret_cast<const float4*>(src + 8 * q) + 1);
+              x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) x[i] = 0.f;
+            }
+            st_shared16(dst + swz128(r, q), to_bf16x8(x));
+          }
+        } else {
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(p.q) + (qrow * D + 64 * s) * 2;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) cp_async16(dst + swz128(r, q), src + 16 * q, v ? 16u : 0u);
+        }
+      }
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      fence_proxy_async_smem();
+      mbar_arrive(q_full);
+      // ---- KV chunks
+      const int n_chunks = (rs.n + kRows - 1) / kRows;
+      for (int c = 0; c < n_chunks && ok; ++c, ++g) {
+        const int r = c * kRows + lt;
+        bool valid = r < rs.n;
+        int64_t row = 0;
+        if (valid) {
+          if (rs.idx) {
+            row = rs.idx[r];
+            if (row < 0 || row >= p.cap) { atomicOr(&g_err_attn, DEV_ERR_BAD_INDEX); valid = false; row = 0; }
+          } else {
+            row = rs.lo + r;
+          }
+        }
+        for (int tt = 0; tt < NT; ++tt) {
+          if (!wait_bar(&pv_done[tt], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
+          load_kv_slab<D, KV>(p, b, row, valid, 2 * tt, sKV + (2 * tt) * kKSlab, lt);
+          if constexpr (KV == KV_BF16) asm volatile("cp.async.commit_group;" ::: "memory");
+          load_kv_slab<D, KV>(p, b, row, valid, 2 * tt + 1, sKV + (2 * tt + 1) * kKSlab, lt);
+          if constexpr (KV == KV_BF16) {
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            if (tt > 0) {
+              asm volatile("cp.async.wait_group 2;" ::: "memory");
+              fence_proxy_async_smem();
+              mbar_arrive(&kv_full[2 * tt - 2]);
+              mbar_arrive(&kv_full[2 * tt - 1]);
+            }
+          } else {
+            fence_proxy_async_smem();
+            mbar_arrive(&kv_full[2 * tt]);
+            mbar_arrive(&kv_full[2 * tt + 1]);
+          }
+        }
+        if constexpr (KV == KV_BF16) {
+          if (ok) {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            fence_proxy_async_smem();
+            mbar_arrive(&kv_full[2 * NT - 2]);
+            mbar_arrive(&kv_full[2 * NT - 1]);
+          }
+        }
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 8) {
+    // ============================ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = make_idesc(128, kNQ, 1, 1, 0, 0);
+      const uint32_t idesc_o = make_idesc(128, kNQ, 1, 1, 1, 1);
+      const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV), aP = smem_u32(sP);
+      uint32_t g = 0, qcount = 0, icount = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        const int b = (int)(item / p.T), t = (int)(item % p.T);
+        const RowSet rs = row_set(p, b, t);
+        if (rs.n == 0) continue;
+        if (!wait_bar(q_full, qcount & 1, abort_flag)) { ok = false; break; }
+        ++qcount;
+        const int n_chunks = (rs.n + kRows - 1) / kRows;
+        for (int c = 0; c < n_chunks && ok; ++c, ++g) {
+          for (int s = 0; s < NS; ++s) {
+            if (!wait_bar(&kv_full[s], g & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              uint64_t ad = smem_desc(aKV + s * kKSlab + kk * 32, 16, 1024, SWZ_128B);
+              uint64_t bd = smem_desc(aQ + s * kQSlab + kk * 32, 16, 1024, SWZ_128B);
+              mma_bf16(tmem, ad, bd, idesc_s, (s | kk) != 0);
+            }
+          }
+          if (!ok) break;
+          mma_commit(s_done);
+          if (c == n_chunks - 1) mma_commit(q_free);
+          if (!wait_bar(p_full, g & 1, abort_flag)) { ok = false; break; }
+          if (c == 0 && !wait_bar(epi_done, (icount & 1) ^ 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          for (int tt = 0; tt < NT; ++tt) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              uint64_t ad = smem_desc(aKV + (2 * tt) * kKSlab + kk * 2048, kKSlab, 1024, SWZ_128B);
+              uint64_t bd = smem_desc(aP + kk * 2048, 16, 1024, SWZ_128B);
+              mma_bf16(tmem + 64 + 64 * tt, ad, bd, idesc_o, (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&pv_done[tt]);
+          }
+        }
+        ++icount;
+      }
+    }
+  } else {
+    // ============================ softmax + epilogue (warps 0-3)
+    const int e = tid;                        // TMEM lane = chunk row = O^T d-row
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    float* bc_m = s_bc + warp * 192;          // per-warp broadcast: [0,64) max, [64,128) alpha / coef_w, [128,192) coef_p
+    uint32_t g = 0, icount = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int b = (int)(item / p.T), t = (int)(item % p.T);
+      const RowSet rs = row_set(p, b, t);
+      const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
+      float2* cs = s_cs + (icount & 1) * 32;
+      if (EPI == EPI_COMBINE && p.inv_rope && tid < 32) {
+        const int j = tid;
+        double inv_freq = exp(-2.0 * (double)j / (double)p.rope_dim * log((double)p.rope_base));
+        double ang = fmod((double)pos * inv_freq, 6.283185307179586476925286766559);
+        double sd, cd;
+        sincos(ang, &sd, &cd);
+        cs[j] = make_float2((float)cd, (float)sd);
+      }
+      float m_own[2] = {-CUDART_INF_F, -CUDART_INF_F};   // running max of columns lane, 32 + lane
+      float l_own[2] = {0.f, 0.f};
+      const int n_chunks = (rs.n + kRows - 1) / kRows;
+      for (int c = 0; c < n_chunks && ok; ++c, ++g) {
+        if (!wait_bar(s_done, g & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        float x[64];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld16(tmem + lane_base + 16 * q, x + 16 * q);
+        tmem_wait_ld();
+        const bool valid = c * kRows + e < rs.n;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) x[j] = valid ? x[j] * p.scale_log2 : -CUDART_INF_F;
+        // column maxima over this warp's 32 rows: lane ends with columns lane, 32 + lane
+        float cm[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = x[32 * h + i];
+#pragma unroll
+          for (int off = 16, n = 32; off >= 1; off >>= 1, n >>= 1) {
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int i = 0; i < n / 2; ++i) {
+              float keep = up ? v[i + n / 2] : v[i];
+              float send = up ? v[i] : v[i + n / 2];
+              v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
+            }
+          }
+          cm[h] = v[0];
+        }
+        float* red = s_red + (g & 1) * 256;
+        red[warp * 64 + lane] = cm[0];
+        red[warp * 64 + 32 + lane] = cm[1];
+        named_bar_sync(1, 128);
+        bool need_rescale = false;
+        float alpha[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int col = 32 * h + lane;
+          float mx = fmaxf(fmaxf(red[col], red[64 + col]), fmaxf(red[128 + col], red[192 + col]));
+          float mn = (mx > m_own[h] + kTau) ? mx : m_own[h];
+          alpha[h] = exp2f(m_own[h] - mn);             // 0 on the first chunk
+          if (mn != m_own[h] && c > 0) need_rescale = true;
+          m_own[h] = mn;
+          bc_m[col] = mn;
+          bc_m[64 + col] = alpha[h];
+        }
+        need_rescale = __any_sync(0xffffffffu, need_rescale);
+        __syncwarp();
+        float p_[64];
+#pragma unroll
+        for (int j = 0; j < 64; j += 4) {
+          float4 mm = *reinterpret_cast<const float4*>(bc_m + j);
+          p_[j] = exp2f(x[j] - mm.x); p_[j + 1] = exp2f(x[j + 1] - mm.y);
+          p_[j + 2] = exp2f(x[j + 2] - mm.z); p_[j + 3] = exp2f(x[j + 3] - mm.w);
+        }
+        // P^T row e -> shared memory (MN-major B operand of the PV MMA)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) st_shared16(sP + swz128(e, q), to_bf16x8(p_ + 8 * q));
+        // column sums of this chunk (per-lane ownership, like the maxima)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = p_[32 * h + i];
+#pragma unroll
+          for (int off = 16, n = 32; off >= 1; off >>= 1, n >>= 1) {
+            const bool up = (lane & off) != 0;
+#pragma unroll
+            for (int i = 0; i < n / 2; ++i) {
+              float keep = up ? v[i + n / 2] : v[i];
+              float send = up ? v[i] : v[i + n / 2];
+              v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            }
+          }
+          l_own[h] = l_own[h] * alpha[h] + v[0];
+        }
+        if (need_rescale) {
+          // O^T columns scale by alpha (this thread is TMEM lane e of every tile)
+          for (int tt = 0; tt < NT; ++tt) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float o[16];
+              const uint32_t ta = tmem + lane_base + 64 + 64 * tt + 16 * q;
+              tmem_ld16(ta, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) o[i] *= bc_m[64 + 16 * q + i];
+              tmem_st16(ta, o);
+            }
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      // ---------------- epilogue
+      // column sums over the 4 warps
+      float* red = s_red + (g & 1) * 256;
+      red[warp * 64 + lane] = l_own[0];
+      red[warp * 64 + 32 + lane] = l_own[1];
+      named_bar_sync(1, 128);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int col = 32 * h + lane;
+        const float lt = red[col] + red[64 + col] + red[128 + col] + red[192 + col];
+        const float lse_w = (lt > 0.f) ? (m_own[h] + log2f(lt)) * kLn2 : -CUDART_INF_F;
+        float cw, cp = 0.f;
+        if (EPI == EPI_PARTIAL) {
+          cw = lt > 0.f ? 1.f / lt : 0.f;
+          if (warp == 0 && col < p.H) p.lse_part[((int64_t)b * p.T + t) * p.H + col] = lse_w;
+        } else {
+          const int64_t o = ((int64_t)b * p.T + t) * p.H + (col < p.H ? col : 0);
+          const float lse_p = (p.O_in && col < p.H) ? p.lse_in[o] : -CUDART_INF_F;
+          const float sk = (p.sink && col < p.H) ? p.sink[col] : -CUDART_INF_F;
+          float M = fmaxf(fmaxf(lse_w, lse_p), sk);
+          if (M == -CUDART_INF_F) M = 0.f;
+          const float ew = __expf(lse_w - M), ep = __expf(lse_p - M), es = __expf(sk - M);
+          const float den = ew + ep + es;
+          cw = lt > 0.f ? ew / (den * lt) : 0.f;
+          cp = den > 0.f ? ep / den : 0.f;
+        }
+        bc_m[64 + col] = cw;
+        bc_m[128 + col] = cp;
+      }
+      __syncwarp();
+      if (rs.n > 0) {
+        for (int tt = 0; tt < NT; ++tt)
+          if (!wait_bar(&pv_done[tt], (g - 1) & 1, abort_flag)) { ok = false; break; }
+        if (!ok) break;
+        tc_fence_after();
+      }
+      const int64_t obase = ((int64_t)b * p.T + t) * p.H;
+      for (int tt = 0; tt < NT; ++tt) {
+        float o[64];
+        if (rs.n > 0) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_ld16(tmem + lane_base + 64 + 64 * tt + 16 * q, o + 16 * q);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) o[i] = 0.f;
+        }
+        const int d = tt * 128 + e;
+        if (EPI == EPI_PARTIAL) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < p.H) p.O_part[(obase + c) * D + d] = o[c] * bc_m[64 + c];
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            float v = o[c] * bc_m[64 + c];
+            if (p.O_in && c < p.H) v = fmaf(bc_m[128 + c], p.O_in[(obase + c) * D + d], v);
+            o[c] = v;
+          }
+          const int r0 = D - p.rope_dim;
+          if (p.inv_rope && tt == NT - 1) {
+            // pairs (d, d + 32) of the last 64 dims sit in warps 2 and 3: swap through sP
+            float* ex = reinterpret_cast<float*>(sP);
+            named_bar_sync(2, 128);
+            if (d >= r0) {
+#pragma unroll
+              for (int c = 0; c < 64; ++c) ex[c * 64 + (d - r0)] = o[c];
+            }
+            named_bar_sync(2, 128);
+            if (d >= r0) {
+              const int jj = d - r0, half = p.rope_dim / 2;
+              const int j = jj % half;
+              const float2 csj = cs[j];
+#pragma unroll
+              for (int c = 0; c < 64; ++c) {
+                // inverse rotation by -pos: (a, b) -> (a cos + b sin, -a sin + b cos)
+                if (jj < half) o[c] = o[c] * csj.x + ex[c * 64 + jj + half] * csj.y;
+                else           o[c] = o[c] * csj.x - ex[c * 64 + jj - half] * csj.y;
+              }
+            }
+          }
+          if (p.out_bf16) {
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c < p.H) out[(obase + c) * D + d] = __float2bfloat16_rn(o[c]);
+          } else {
+            float* out = reinterpret_cast<float*>(p.out);
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c < p.H) out[(obase + c) * D + d] = o[c];
+          }
+        }
+      }
+      if (rs.n > 0) {
+        tc_fence_before();
+        mbar_arrive(epi_done);
+        ++icount;
+      } else {
+        // keep the cos/sin double buffer in step only for items that used it
+        ++icount;
+      }
+      named_bar_sync(1, 128);   // s_red / bc reuse across items
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, int KV, int EPI>
+csa_status_t launch_attn(const AttnParams& p, cudaStream_t st) {
+  constexpr int NS = D / 64, NT = D / 128;
+  const size_t smem = 1024 + NS * (kNQ * 128) + NS * (kRows * 128) + kRows * 128 +
+                      (2 * 4 * 64 + 4 * 3 * 64) * 4 + 64 * 8 + (5 + NS + NT) * 8 + 16;
+  auto kern = attn_kernel<D, KV, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attention: cannot reserve %zu bytes of shared memory: %s", smem, cudaGetErrorString(e));
+  const int64_t items = (int64_t)p.n_seq * p.T;
+  if (items == 0) return CSA_OK;
+  const int grid = (int)std::min<int64_t>(items, num_sms());
+  kern<<<grid, kThreads, smem, st>>>(p);
+  return check_launch("attention");
+}
+
+template <int EPI>
+csa_status_t dispatch(const AttnParams& p, int D, csa_dtype_t kv_dtype, cudaStream_t st) {
+  if (D == 512) {
+    if (kv_dtype == CSA_BF16) return launch_attn<512, KV_BF16, EPI>(p, st);
+    if (kv_dtype == CSA_F32) return launch_attn<512, KV_F32, EPI>(p, st);
+    return launch_attn<512, KV_FP8, EPI>(p, st);
+  }
+  if (kv_dtype == CSA_BF16) return launch_attn<128, KV_BF16, EPI>(p, st);
+  if (kv_dtype == CSA_F32) return launch_attn<128, KV_F32, EPI>(p, st);
+  return launch_attn<128, KV_FP8, EPI>(p, st);
+}
+
+csa_status_t check_common(const char* fn, const void* q, csa_dtype_t q_dtype, const void* kv, csa_dtype_t kv_dtype,
+                          const void* kv_rope, const float* kv_scale, int64_t cap, int n_seq, int T, int H, int D,
+                          int rope_dim) {
+  CSA_REQUIRE(n_seq >= 0 && T >= 0 && cap >= 1, "%s: bad n_seq/T/cap", fn);
+  CSA_REQUIRE(H >= 1 && H <= 64, "%s: H must be in [1, 64]", fn);
+  CSA_REQUIRE(D == 128 || D == 512, "%s: D must be 128 or 512", fn);
+  CSA_REQUIRE(rope_dim == 0 || rope_dim == 64, "%s: rope_dim must be 0 or 64", fn);
+  CSA_REQUIRE(q_dtype == CSA_BF16 || q_dtype == CSA_F32, "%s: q_dtype must be BF16 or F32", fn);
+  CSA_REQUIRE(kv_dtype == CSA_BF16 || kv_dtype == CSA_F32 || kv_dtype == CSA_E4M3, "%s: bad kv_dtype", fn);
+  CSA_REQUIRE(q && kv && aligned16(q) && aligned16(kv), "%s: q/kv must be non-null and 16-byte aligned", fn);
+  if (kv_dtype == CSA_E4M3) {
+    CSA_REQUIRE(rope_dim == 64 && kv_rope && kv_scale && aligned16(kv_rope) && aligned16(kv_scale),
+                "%s: an e4m3 KV store needs rope_dim 64, kv_rope and kv_scale", fn);
+  }
+  return CSA_OK;
+}
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" csa_status_t csa_sparse_mqa(const void* q, csa_dtype_t q_dtype, const void* kv,
+                                       csa_dtype_t kv_dtype, const void* kv_rope, const float* kv_scale,
+                                       int64_t cap, const int32_t* idx, int k, int n_seq, int T, int H,
+                                       int D, int rope_dim, float scale, float* O_part, float* lse_part,
+                                       cudaStream_t stream) {
+  clear_error();
+  csa_status_t s = check_common("csa_sparse_mqa", q, q_dtype, kv, kv_dtype, kv_rope, kv_scale, cap, n_seq, T, H, D, rope_dim);
+  if (s != CSA_OK) return s;
+  CSA_REQUIRE(k >= 1 && idx && aligned16(idx), "csa_sparse_mqa: idx must be non-null, aligned, k >= 1");
+  CSA_REQUIRE(O_part && lse_part && aligned16(O_part), "csa_sparse_mqa: O_part / lse_part must be non-null");
+  AttnParams p{};
+  p.q = q; p.q_f32 = q_dtype == CSA_F32; p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale;
+  p.cap = cap; p.idx = idx; p.k = k; p.q_pos = nullptr; p.row_kind = ROWS_GATHER; p.m = 1; p.W = 0;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.O_part = O_part; p.lse_part = lse_part; p.rope_dim = rope_dim;
+  return dispatch<EPI_PARTIAL>(p, D, kv_dtype, stream);
+}
+
+extern "C" csa_status_t hca_dense_attn(const void* q, csa_dtype_t q_dtype, const void* kv,
+                                       csa_dtype_t kv_dtype, const void* kv_rope, const float* kv_scale,
+                                       int64_t cap, const int64_t* q_pos, int m, int n_seq, int T, int H,
+                                       int D, int rope_dim, float scale, float* O_part, float* lse_part,
+                                       cudaStream_t stream) {
+  clear_error();
+  csa_status_t s = check_common("hca_dense_attn", q, q_dtype, kv, kv_dtype, kv_rope, kv_scale, cap, n_seq, T, H, D, rope_dim);
+  if (s != CSA_OK) return s;
+  CSA_REQUIRE(m >= 1 && q_pos && aligned16(q_pos), "hca_dense_attn: m >= 1 and q_pos required");
+  CSA_REQUIRE(O_part && lse_part && aligned16(O_part), "hca_dense_attn: O_part / lse_part must be non-null");
+  AttnParams p{};
+  p.q = q; p.q_f32 = q_dtype == CSA_F32; p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale;
+  p.cap = cap; p.q_pos = q_pos; p.row_kind = ROWS_DENSE; p.m = m; p.W = 0;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.O_part = O_part; p.lse_part = lse_part; p.rope_dim = rope_dim;
+  return dispatch<EPI_PARTIAL>(p, D, kv_dtype, stream);
+}
+
+extern "C" csa_status_t swa_sink_combine(const void* q, csa_dtype_t q_dtype, const void* kv_tok,
+                                         csa_dtype_t kv_dtype, int64_t cap, const int64_t* q_pos, int W,
+                                         int window_mode, const float* sink, const float* O_part,
+                                         const float* lse_part, int n_seq, int T, int H, int D,
+                                         int rope_dim, float rope_base, int inv_rope, float scale,
+                                         void* out, csa_dtype_t out_dtype, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(kv_dtype == CSA_BF16 || kv_dtype == CSA_F32, "swa_sink_combine: kv_dtype must be BF16 or F32");
+  csa_status_t s = check_common("swa_sink_combine", q, q_dtype, kv_tok, kv_dtype, nullptr, nullptr, cap, n_seq, T, H, D, rope_dim);
+  if (s != CSA_OK) return s;
+  CSA_REQUIRE(W >= 1 && q_pos && aligned16(q_pos), "swa_sink_combine: W >= 1 and q_pos required");
+  CSA_REQUIRE(window_mode == 0 || window_mode == 1, "swa_sink_combine: window_mode must be 0 or 1");
+  CSA_REQUIRE(!inv_rope || rope_dim == 64, "swa_sink_combine: inv_rope needs rope_dim 64");
+  CSA_REQUIRE((O_part == nullptr) == (lse_part == nullptr), "swa_sink_combine: give both O_part and lse_part or neither");
+  CSA_REQUIRE(!O_part || aligned16(O_part), "swa_sink_combine: O_part must be 16-byte aligned");
+  CSA_REQUIRE(out && aligned16(out) && (out_dtype == CSA_F32 || out_dtype == CSA_BF16), "swa_sink_combine: bad out");
+  AttnParams p{};
+  p.q = q; p.q_f32 = q_dtype == CSA_F32; p.kv = kv_tok; p.cap = cap; p.q_pos = q_pos;
+  p.row_kind = window_mode == 0 ? ROWS_WINDOW : ROWS_CACHE; p.m = 1; p.W = W;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.O_in = O_part; p.lse_in = lse_part; p.sink = sink; p.out = out; p.out_bf16 = out_dtype == CSA_BF16;
+  p.inv_rope = inv_rope; p.rope_dim = rope_dim; p.rope_base = rope_base;
+  return dispatch<EPI_COMBINE>(p, D, kv_dtype, stream);
+}

@@ -1,0 +1,40 @@
+// Host-side helpers shared by the C-ABI translation units: last-error text,
+// argument checks, and the per-unit device error words.
+#pragma once
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cuda_runtime.h>
+#include "../../include/csa.h"
+
+namespace csa {
+
+csa_status_t fail(csa_status_t s, const char* fmt, ...);
+void clear_error();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline csa_status_t check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  return CSA_OK;
+}
+
+inline int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Each translation unit that launches kernels owns a device error word and
+// exposes a reader that returns and clears it (synchronous).
+uint32_t read_clear_err_indexer();
+uint32_t read_clear_err_attention();
+
+}  // namespace csa
+
+#define CSA_REQUIRE(cond, ...)                                 \
+  do {                                                         \
+    if (!(cond)) return ::csa::fail(CSA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)

@@ -1,0 +1,335 @@
+// KV compressor (CSA m = 4 with overlap, HCA m' = 128 without) and the QK
+// RMSNorm + partial-RoPE prologue.
+//
+// "DeepSeek V4 脱离 CUDA 全栈国产化：1.6T MoE 逐层拆解 + 昇腾迁移数据", §二:
+//   "KV 压缩"  — an entry is the per-channel Softmax(Z + B)-weighted sum of C
+//               over its block, blocks overlapping the previous one (m = 4);
+//   "HCA"      — m' = 128 non-overlapping blocks;
+//   "其他辅助设计" — RMSNorm on Q and K before attention; RoPE on the last 64 dims.
+// "Deepseek-V4 技术报告里最值得复现的三个改动", §5: tail tokens that do not fill
+// a block are dropped.
+//
+// Both kernels are HBM-streaming: every thread owns 8 consecutive channels and
+// moves them with 16-byte (bf16) or 2 x 16-byte (fp32) vector loads, so a group
+// of D/8 threads reads one row with fully coalesced transactions.  No tensor
+// cores: there is no contraction here.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+#include "common.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <typename T> struct Vec8;
+template <> struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float* v) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float* v) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+};
+template <> struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* v) {
+    uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&a);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { float2 f = __bfloat1622float2(h[i]); v[2 * i] = f.x; v[2 * i + 1] = f.y; }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float* v) {
+    uint4 a;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&a);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = a;
+  }
+};
+
+// cos/sin of pos * base^(-2j/rope_dim): the angle is formed and reduced in
+// double so that positions up to 2^20 and beyond keep fp32-accurate rotations.
+__device__ __forceinline__ void rope_cs(int64_t pos, int j, int rope_dim, float rope_base, float* c, float* s) {
+  double inv_freq = exp(-2.0 * (double)j / (double)rope_dim * log((double)rope_base));
+  double ang = fmod((double)pos * inv_freq, 6.283185307179586476925286766559);
+  double sd, cd;
+  sincos(ang, &sd, &cd);
+  *c = (float)cd;
+  *s = (float)sd;
+}
+
+// One CTA: `epc` entries, each owned by `gpe` groups of tpg = D/8 threads.
+// The groups of an entry split its window rows round-robin, keep an online
+// per-channel softmax state (running max, sum, weighted sum of C) and merge
+// through shared memory; the entry's first group then applies RMSNorm and RoPE.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads)
+compress_kernel(const Tin* __restrict__ C, const Tin* __restrict__ Z, const Tin* __restrict__ Cb,
+                const Tin* __restrict__ Zb, const float* __restrict__ B, int64_t n_e, int D, int m,
+                int overlap, int norm, int rope_dim, float rope_base, float eps, Tout* __restrict__ out,
+                int tpg, int gpe, int epc) {
+  extern __shared__ float sm[];            // 3 * kThreads * 8 floats + kThreads
+  float* s_mx = sm;
+  float* s_sum = sm + kThreads * 8;
+  float* s_acc = sm + 2 * kThreads * 8;
+  float* s_red = sm + 3 * kThreads * 8;
+
+  const int tid = threadIdx.x;
+  const int ngroups = kThreads / tpg;
+  const int g = tid / tpg, c8 = tid % tpg;
+  const int el = g / gpe, sub = g % gpe;
+  const bool active_group = g < epc * gpe;
+  const int64_t i = (int64_t)blockIdx.x * epc + el;
+  const bool valid = active_group && i < n_e;
+  const int ch0 = c8 * 8;
+
+  float mx[8], sum[8], acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) { mx[c] = -CUDART_INF_F; sum[c] = 0.f; acc[c] = 0.f; }
+
+  if (valid) {
+    const int64_t cur0 = i * m;
+    const int64_t lo = (overlap && i > 0) ? cur0 - m : cur0;
+    const int64_t hi = cur0 + m;
+    for (int64_t j = lo + sub; j < hi; j += gpe) {
+      const bool prev = j < cur0;
+      const Tin* cp = (prev ? Cb : C) + j * D + ch0;
+      const Tin* zp = (prev ? Zb : Z) + j * D + ch0;
+      const int brow = overlap ? (prev ? (int)(j - lo) : m + (int)(j - cur0)) : (int)(j - cur0);
+      float cv[8], zv[8], bv[8];
+      Vec8<Tin>::load(cp, cv);
+      Vec8<Tin>::load(zp, zv);
+      if (B) Vec8<float>::load(B + (int64_t)brow * D + ch0, bv);
+      else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) bv[c] = 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float l = (zv[c] + bv[c]) * kLog2e;
+        if (l > mx[c]) {
+          float a = exp2f(mx[c] - l);
+          sum[c] *= a; acc[c] *= a; mx[c] = l;
+        }
+        float p = exp2f(l - mx[c]);
+        sum[c] += p;
+        acc[c] = fmaf(p, cv[c], acc[c]);
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    s_mx[tid * 8 + c] = mx[c]; s_sum[tid * 8 + c] = sum[c]; s_acc[tid * 8 + c] = acc[c];
+  }
+  __syncthreads();
+
+  float x[8];
+  const bool owner = valid && sub == 0;
+  float ss = 0.f;
+  if (owner) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float M = mx[c], Ssum = sum[c], A = acc[c];
+      for (int q = 1; q < gpe; ++q) {
+        int t2 = (g + q) * tpg + c8;
+        float m2 = s_mx[t2 * 8 + c], s2 = s_sum[t2 * 8 + c], a2 = s_acc[t2 * 8 + c];
+        if (m2 == -CUDART_INF_F) continue;
+        float Mn = fmaxf(M, m2);
+        float f1 = exp2f(M - Mn), f2 = exp2f(m2 - Mn);
+        Ssum = Ssum * f1 + s2 * f2;
+        A = A * f1 + a2 * f2;
+        M = Mn;
+      }
+      x[c] = A / Ssum;
+      ss = fmaf(x[c], x[c], ss);
+    }
+  }
+  s_red[tid] = ss;
+  __syncthreads();
+  if (owner && norm) {
+    float tot = 0.f;
+    const int base = g * tpg;
+    for (int q = 0; q < tpg; ++q) tot += s_red[base + q];
+    float inv = rsqrtf(tot / (float)D + eps);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[c] *= inv;
+  }
+  // RoPE: partners live in other threads; exchange through shared memory
+  // (s_acc is free now: every thread has read what it needs).
+  __syncthreads();
+  float* s_x = s_acc;
+  if (owner) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) s_x[el * D + ch0 + c] = x[c];
+  }
+  __syncthreads();
+  if (owner && rope_dim > 0) {
+    const int half = rope_dim / 2, r0 = D - rope_dim;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      int d = ch0 + c;
+      if (d < r0) continue;
+      int j = (d - r0) % half;
+      float cs, sn;
+      rope_cs(i * m, j, rope_dim, rope_base, &cs, &sn);
+      if (d < r0 + half) x[c] = s_x[el * D + d] * cs - s_x[el * D + d + half] * sn;
+      else               x[c] = s_x[el * D + d - half] * sn + s_x[el * D + d] * cs;
+    }
+  }
+  if (owner) Vec8<Tout>::store(out + i * D + ch0, x);
+}
+
+// Rows of `rows_per_pos` share one position; a CTA handles `ppb` positions.
+// Each warp normalises whole rows: lane owns D/32 consecutive channels.
+template <typename Tin, typename Tout, int CPL>
+__global__ void __launch_bounds__(kThreads)
+rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int D, int rows_per_pos, int64_t pos0,
+                    int ppb, int norm, int rope_dim, float rope_base, float eps, Tout* __restrict__ out) {
+  __shared__ float2 s_cs[8][64];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t p_first = (int64_t)blockIdx.x * ppb;
+  const int half = rope_dim / 2;
+  for (int e = tid; e < ppb * half; e += kThreads) {
+    int pl = e / half, j = e % half;
+    float c, s;
+    rope_cs(pos0 + p_first + pl, j, rope_dim, rope_base, &c, &s);
+    s_cs[pl][j] = make_float2(c, s);
+  }
+  __syncthreads();
+  const int64_t r_begin = p_first * rows_per_pos;
+  const int64_t r_end = min(rows, (p_first + ppb) * rows_per_pos);
+  for (int64_t r = r_begin + warp; r < r_end; r += kThreads / 32) {
+    float v[CPL];
+    const Tin* src = x + r * D + lane * CPL;
+#pragma unroll
+    for (int c = 0; c < CPL; c += 8) Vec8<Tin>::load(src + c, v + c);
+    if (norm) {
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) ss = fmaf(v[c], v[c], ss);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      float inv = rsqrtf(ss / (float)D + eps);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) v[c] *= inv;
+    }
+    if (rope_dim > 0) {
+      const int pl = (int)(r / rows_per_pos - p_first);
+      const int r0 = D - rope_dim;
+      const int partner = half / CPL;   // lane distance between (d, d + half)
+      float w[CPL];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        float up = __shfl_down_sync(0xffffffffu, v[c], partner);
+        float dn = __shfl_up_sync(0xffffffffu, v[c], partner);
+        int d = lane * CPL + c;
+        if (d < r0) { w[c] = v[c]; continue; }
+        int j = (d - r0) % half;
+        float2 cs = s_cs[pl][j];
+        w[c] = (d < r0 + half) ? v[c] * cs.x - up * cs.y : dn * cs.y + v[c] * cs.x;
+      }
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) v[c] = w[c];
+    }
+#pragma unroll
+    for (int c = 0; c < CPL; c += 8) Vec8<Tout>::store(out + r * D + lane * CPL + c, v + c);
+  }
+}
+
+template <typename Tin, typename Tout>
+csa_status_t launch_compress(const void* C, const void* Z, const void* Cb, const void* Zb, const float* B,
+                             int64_t n_e, int D, int m, int overlap, int norm, int rope_dim,
+                             float rope_base, float eps, void* out, cudaStream_t st) {
+  const int tpg = D / 8;
+  const int ngroups = kThreads / tpg;
+  // Long blocks (HCA) are split across several groups; short ones get one.
+  const int window = overlap ? 2 * m : m;
+  int gpe = 1;
+  while (gpe * 2 <= ngroups && window / (gpe * 2) >= 8) gpe *= 2;
+  const int epc = ngroups / gpe;
+  const int64_t grid = (n_e + epc - 1) / epc;
+  const size_t smem = (3 * kThreads * 8 + kThreads) * sizeof(float);
+  if (grid == 0) return CSA_OK;
+  if (grid > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "csa_compress: too many entries");
+  auto kern = compress_kernel<Tin, Tout>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  kern<<<(unsigned)grid, kThreads, smem, st>>>(
+      (const Tin*)C, (const Tin*)Z, (const Tin*)(Cb ? Cb : C), (const Tin*)(Zb ? Zb : Z), B, n_e, D, m,
+      overlap, norm, rope_dim, rope_base, eps, (Tout*)out, tpg, gpe, epc);
+  return check_launch("csa_compress");
+}
+
+template <typename Tin, typename Tout, int CPL>
+csa_status_t launch_norm(const void* x, int64_t rows, int D, int rpp, int64_t pos0, int norm, int rope_dim,
+                         float rope_base, float eps, void* out, cudaStream_t st) {
+  int ppb = rpp >= 8 ? 1 : 8 / rpp;
+  int64_t npos = (rows + rpp - 1) / rpp;
+  int64_t grid = (npos + ppb - 1) / ppb;
+  if (grid == 0) return CSA_OK;
+  if (grid > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "csa_rmsnorm_rope: too many rows");
+  rmsnorm_rope_kernel<Tin, Tout, CPL><<<(unsigned)grid, kThreads, 0, st>>>(
+      (const Tin*)x, rows, D, rpp, pos0, ppb, norm, rope_dim, rope_base, eps, (Tout*)out);
+  return check_launch("csa_rmsnorm_rope");
+}
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" csa_status_t csa_compress(const void* C, const void* Z, const void* Cb, const void* Zb,
+                                     const float* B, int64_t S, int D, int m, int overlap,
+                                     csa_dtype_t in_dtype, int norm, int rope_dim, float rope_base,
+                                     float eps, void* out, csa_dtype_t out_dtype, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(S >= 0, "csa_compress: S < 0");
+  CSA_REQUIRE(D % 8 == 0 && D >= 8 && D <= 2048, "csa_compress: D must be a multiple of 8 in [8, 2048]");
+  CSA_REQUIRE(m >= 1 && m <= 1024, "csa_compress: m must be in [1, 1024]");
+  CSA_REQUIRE(overlap == 0 || overlap == 1, "csa_compress: overlap must be 0 or 1");
+  CSA_REQUIRE(rope_dim >= 0 && rope_dim % 2 == 0 && rope_dim <= D && (rope_dim == 0 || (rope_dim / 2) % 8 == 0),
+              "csa_compress: rope_dim must be 0 or an even size <= D with rope_dim/2 a multiple of 8");
+  CSA_REQUIRE(in_dtype == CSA_F32 || in_dtype == CSA_BF16, "csa_compress: in_dtype must be F32 or BF16");
+  CSA_REQUIRE(out_dtype == CSA_F32 || out_dtype == CSA_BF16, "csa_compress: out_dtype must be F32 or BF16");
+  const int64_t n_e = S / m;
+  if (n_e == 0) return CSA_OK;
+  CSA_REQUIRE(C && Z && out, "csa_compress: C, Z and out must be non-null");
+  CSA_REQUIRE(aligned16(C) && aligned16(Z) && aligned16(out) && (!Cb || aligned16(Cb)) &&
+              (!Zb || aligned16(Zb)) && (!B || aligned16(B)), "csa_compress: pointers must be 16-byte aligned");
+  if (in_dtype == CSA_F32 && out_dtype == CSA_F32)
+    return launch_compress<float, float>(C, Z, Cb, Zb, B, n_e, D, m, overlap, norm, rope_dim, rope_base, eps, out, stream);
+  if (in_dtype == CSA_F32 && out_dtype == CSA_BF16)
+    return launch_compress<float, __nv_bfloat16>(C, Z, Cb, Zb, B, n_e, D, m, overlap, norm, rope_dim, rope_base, eps, out, stream);
+  if (in_dtype == CSA_BF16 && out_dtype == CSA_F32)
+    return launch_compress<__nv_bfloat16, float>(C, Z, Cb, Zb, B, n_e, D, m, overlap, norm, rope_dim, rope_base, eps, out, stream);
+  return launch_compress<__nv_bfloat16, __nv_bfloat16>(C, Z, Cb, Zb, B, n_e, D, m, overlap, norm, rope_dim, rope_base, eps, out, stream);
+}
+
+extern "C" csa_status_t csa_rmsnorm_rope(const void* x, csa_dtype_t in_dtype, int64_t rows, int D,
+                                         int rows_per_pos, int64_t pos0, int norm, int rope_dim,
+                                         float rope_base, float eps, void* out, csa_dtype_t out_dtype,
+                                         cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(rows >= 0 && rows_per_pos >= 1 && pos0 >= 0, "csa_rmsnorm_rope: bad rows/rows_per_pos/pos0");
+  CSA_REQUIRE(D == 128 || D == 256 || D == 512, "csa_rmsnorm_rope: D must be 128, 256 or 512");
+  CSA_REQUIRE(rope_dim == 0 || rope_dim == 64, "csa_rmsnorm_rope: rope_dim must be 0 or 64");
+  CSA_REQUIRE(in_dtype == CSA_F32 || in_dtype == CSA_BF16, "csa_rmsnorm_rope: in_dtype must be F32 or BF16");
+  CSA_REQUIRE(out_dtype == CSA_F32 || out_dtype == CSA_BF16, "csa_rmsnorm_rope: out_dtype must be F32 or BF16");
+  if (rows == 0) return CSA_OK;
+  CSA_REQUIRE(x && out && aligned16(x) && aligned16(out), "csa_rmsnorm_rope: x/out must be non-null and 16-byte aligned");
+#define CSA_NORM_CASE(TI, TO)                                                                    \
+  if (D == 256) return launch_norm<TI, TO, 8>(x, rows, D, rows_per_pos, pos0, norm, rope_dim,   \
+                                              rope_base, eps, out, stream);                      \
+  if (D == 512) return launch_norm<TI, TO, 16>(x, rows, D, rows_per_pos, pos0, norm, rope_dim,  \
+                                               rope_base, eps, out, stream);
+  CSA_REQUIRE(D != 128, "csa_rmsnorm_rope: D = 128 is not supported (use D >= 256)");
+  if (in_dtype == CSA_F32 && out_dtype == CSA_F32) { CSA_NORM_CASE(float, float) }
+  if (in_dtype == CSA_F32 && out_dtype == CSA_BF16) { CSA_NORM_CASE(float, __nv_bfloat16) }
+  if (in_dtype == CSA_BF16 && out_dtype == CSA_F32) { CSA_NORM_CASE(__nv_bfloat16, float) }
+  if (in_dtype == CSA_BF16 && out_dtype == CSA_BF16) { CSA_NORM_CASE(__nv_bfloat16, __nv_bfloat16) }
+#undef CSA_NORM_CASE
+  return fail(CSA_ERR_UNSUPPORTED, "csa_rmsnorm_rope: unsupported combination");
+}

@@ -1,0 +1,529 @@
+// Lightning indexer and top-k selection.
+//
+// "DeepSeek V4 脱离 CUDA 全栈国产化：1.6T MoE 逐层拆解 + 昇腾迁移数据", §二 CSA
+// "闪电索引器": several index heads score every compressed entry through a
+// ReLU of the query/key similarity, weighted over heads, then the top-k
+// entries are kept (512 for Flash, 1024 for Pro); the QK path runs at the
+// lowest precision.  liduos.com "1M Context 的结构与取舍": only the top-k
+// entries are read by the query.
+//
+// Kernel 1 (indexer_scores_kernel) is an FP8 e4m3 tensor-core contraction:
+//   D[key, (token, head)] = kI[key, :] . qI[token, head, :]
+// with M = 128 keys per tile (A operand, streamed by TMA through a ring of
+// shared-memory stages), N = TQ tokens x HI heads (B operand, loaded once per
+// CTA), K = DI, fp32 accumulation in TMEM (two accumulators so the epilogue
+// of tile j overlaps the MMA of tile j+1).  The epilogue applies ReLU, the
+// head weights w * qs, the key scale ks and the visibility mask, and writes
+// one fp32 score per (token, key).
+//
+// Kernels 2/3 select the top-k per query row by a 4-pass 8-bit radix select
+// on order-preserving uint32 keys, then compact in index order, so the result
+// is ascending, deterministic, and ties go to the lower entry index.  Rows
+// longer than one shared-memory chunk are split into chunks (local top-k
+// each) and the candidates merged; the global top-k restricted to a chunk is
+// always within that chunk's local top-k, so the merge is exact.
+#include <algorithm>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace csa {
+
+static __device__ uint32_t g_err_idx;
+
+uint32_t read_clear_err_indexer() {
+  uint32_t v = 0, z = 0;
+  cudaMemcpyFromSymbol(&v, g_err_idx, sizeof(v));
+  cudaMemcpyToSymbol(g_err_idx, &z, sizeof(z));
+  return v;
+}
+
+namespace {
+
+// ------------------------------------------------------------------ TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows, row_bytes] with boxes of [box_rows, row_bytes],
+// swizzled to match the tcgen05 K-major layout of the same width.
+bool make_byte_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes, uint32_t box_rows) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  CUtensorMapSwizzle swz = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                         : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  cuuint64_t gdim[2] = {row_bytes, rows};
+  cuuint64_t gstride[1] = {row_bytes};
+  cuuint32_t box[2] = {row_bytes, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ scores
+constexpr int kIdxThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kStages = 8;
+
+struct IdxParams {
+  const float* qs;        // [n_seq, T, HI] or null
+  const float* w;         // [n_seq, T, HI]
+  const float* ks;        // [n_seq, cap] or null
+  const int64_t* q_pos;   // [n_seq]
+  float* scores;          // [n_seq, T, cap]
+  int64_t cap;
+  int T, HI, DI, m, TQ, N, tiles_per_chunk;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  uint64_t start = 0;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0) {
+      if (*abort_flag) return false;
+      const uint64_t now = global_ns();
+      if (start == 0) start = now;
+      else if (now - start > kWaitNs) break;
+    }
+  }
+  *abort_flag = 1;
+  atomicOr(&g_err_idx, DEV_ERR_TIMEOUT_MBAR);
+  return false;
+}
+
+__global__ void __launch_bounds__(kIdxThreads, 1)
+indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                      IdxParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int b = blockIdx.z, qb = blockIdx.y, chunk = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t0 = qb * p.TQ;
+  const int t_last = min(p.T, t0 + p.TQ) - 1;
+  const int64_t pos0 = p.q_pos[b];
+  const int64_t nv_max = min(p.cap, (pos0 + t_last + 1) / p.m);
+  const int n_tiles_all = (int)((nv_max + 127) / 128);
+  const int tile0 = chunk * p.tiles_per_chunk;
+  const int n_tiles = min(n_tiles_all - tile0, p.tiles_per_chunk);
+  if (n_tiles <= 0) return;
+
+  const uint32_t a_bytes = 128u * p.DI;
+  const uint32_t b_bytes = (uint32_t)p.N * p.DI;
+  uint8_t* sB = smem;
+  uint8_t* sA = smem + ((b_bytes + 1023u) & ~1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sA + kStages * a_bytes);
+  uint64_t* full = bars;                 // [kStages]
+  uint64_t* empty = bars + kStages;      // [kStages]
+  uint64_t* tfull = bars + 2 * kStages;  // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* qbar = tempty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(qbar + 1);
+  int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
+  float* s_w = reinterpret_cast<float*>(s_abort + 1);   // [N] = w * qs per column
+
+  const uint32_t tmem_cols = p.N <= 16 ? 32u : (p.N <= 32 ? 64u : (p.N <= 64 ? 128u : (p.N <= 128 ? 256u : 512u)));
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 128); }
+    mbar_init(qbar, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  for (int c = tid; c < p.N; c += kIdxThreads) {
+    const int tq = c / p.HI, h = c % p.HI;
+    const int t = t0 + tq;
+    float v = 0.f;
+    if (t < p.T) {
+      const int64_t o = ((int64_t)b * p.T + t) * p.HI + h;
+      v = p.w[o] * (p.qs ? p.qs[o] : 1.f);
+    }
+    s_w[c] = v;
+  }
+  if (warp == 1) tmem_alloc(s_tmem, tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  volatile int* abort_flag = s_abort;
+
+  const uint32_t swz = p.DI == 128 ? SWZ_128B : (p.DI == 64 ? SWZ_64B : SWZ_32B);
+  const uint32_t sbo = 8u * p.DI;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_q);
+    mbar_expect_tx(qbar, b_bytes);
+    tma_load_2d(sB, &tmap_q, 0, (int32_t)(((int64_t)b * p.T + t0) * p.HI), qbar);
+    for (int it = 0; it < n_tiles; ++it) {
+      const int s = it % kStages;
+      const uint32_t ph = (it / kStages) & 1;
+      if (!wait_bar(&empty[s], ph ^ 1, abort_flag)) break;
+      mbar_expect_tx(&full[s], a_bytes);
+      tma_load_2d(sA + s * a_bytes, &tmap_k, 0, (int32_t)((int64_t)b * p.cap + (int64_t)(tile0 + it) * 128), &full[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint32_t idesc = make_idesc(128, p.N, 0, 0, 0, 0);
+    const uint32_t sB_addr = smem_u32(sB), sA_addr = smem_u32(sA);
+    if (wait_bar(qbar, 0, abort_flag)) {
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!wait_bar(&full[s], ph, abort_flag)) break;
+        if (!wait_bar(&tempty[acc], aph ^ 1, abort_flag)) break;
+        tc_fence_after();
+        for (int kk = 0; kk < p.DI / 32; ++kk) {
+          uint64_t ad = smem_desc(sA_addr + s * a_bytes + kk * 32, 16, sbo, swz);
+          uint64_t bd = smem_desc(sB_addr + kk * 32, 16, sbo, swz);
+          mma_f8(tmem + acc * p.N, ad, bd, idesc, kk > 0);
+        }
+        mma_commit(&empty[s]);
+        mma_commit(&tfull[acc]);
+      }
+    }
+  } else if (warp >= 2) {
+    // ---------------- epilogue: 128 threads, one key (TMEM lane) each
+    const int sp = warp & 3;                       // TMEM sub-partition of this warp
+    const int key_in_tile = sp * 32 + lane;
+    for (int it = 0; it < n_tiles; ++it) {
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      if (!wait_bar(&tfull[acc], aph, abort_flag)) break;
+      tc_fence_after();
+      const int64_t key = (int64_t)(tile0 + it) * 128 + key_in_tile;
+      const float ksc = (key < p.cap) ? (p.ks ? p.ks[(int64_t)b * p.cap + key] : 1.f) : 0.f;
+      float run = 0.f;
+      for (int cc = 0; cc < p.N; cc += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N + cc, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = cc + i;
+          run = fmaf(s_w[col], fmaxf(v[i], 0.f), run);
+          if (((col + 1) & (p.HI - 1)) == 0) {
+            const int t = t0 + col / p.HI;
+            if (t < p.T) {
+              const int64_t nv = min(p.cap, (pos0 + t + 1) / p.m);
+              if (key < nv) p.scores[((int64_t)b * p.T + t) * p.cap + key] = run * ksc;
+            }
+            run = 0.f;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------------ top-k
+constexpr int kTopkThreads = 512;
+constexpr int kChunk = 16384;          // keys per shared-memory chunk (64 KB)
+constexpr int kMergeCap = 16384;       // candidates per row in the merge stage
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f + 0.0f);   // -0 -> +0 so that equal values tie
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+struct SelectSmem {
+  uint32_t hist[256];
+  uint64_t warp_tot[kTopkThreads / 32];
+  uint32_t digit, above;
+};
+
+// Block-wide inclusive scan of a packed (gt << 32 | eq) count.
+__device__ __forceinline__ uint64_t block_scan_incl(uint64_t v, SelectSmem& ss) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint64_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) ss.warp_tot[warp] = v;
+  __syncthreads();
+  uint64_t off = 0;
+  for (int w = 0; w < warp; ++w) off += ss.warp_tot[w];
+  __syncthreads();
+  return v + off;
+}
+
+// Selects the top-k of keys[0..n) (ties to the lower position) and writes
+// out[pos] = ids[e] (or id_base + e when ids == null) in ascending position
+// order; also returns the count written (min(k, n)).  All threads participate.
+__device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id_base, int n, int k,
+                            int32_t* out_idx, uint32_t* out_key, SelectSmem& ss) {
+  const int tid = threadIdx.x;
+  uint32_t T = 0;
+  int need_eq = 0;
+  const bool all = n <= k;
+  if (!all) {
+    uint32_t prefix = 0, mask = 0;
+    int remaining = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kTopkThreads) ss.hist[i] = 0;
+      __syncthreads();
+      for (int e = tid; e < n; e += kTopkThreads) {
+        const uint32_t key = keys[e];
+        if ((key & mask) == prefix) atomicAdd(&ss.hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (tid < 32) {
+        uint32_t c[8], s = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { c[i] = ss.hist[tid * 8 + i]; s += c[i]; }
+        // exclusive suffix sum over higher lanes
+        uint32_t suf = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          uint32_t nn = __shfl_down_sync(0xffffffffu, suf, o);
+          if (tid + o < 32) suf += nn;
+        }
+        uint32_t excl = suf - s;
+        if (excl < (uint32_t)remaining && (uint32_t)remaining <= excl + s) {
+          uint32_t cum = excl;
+#pragma unroll
+          for (int i = 7; i >= 0; --i) {
+            if (cum + c[i] >= (uint32_t)remaining) { ss.digit = tid * 8 + i; ss.above = cum; break; }
+            cum += c[i];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= ss.digit << shift;
+      mask |= 255u << shift;
+      remaining -= (int)ss.above;
+      __syncthreads();
+    }
+    T = prefix;
+    need_eq = remaining;
+  }
+  // stable compaction in position order
+  const int per = (n + kTopkThreads - 1) / kTopkThreads;
+  const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
+  uint32_t gt = 0, eq = 0;
+  if (!all) {
+    for (int e = e0; e < e1; ++e) { uint32_t key = keys[e]; gt += key > T; eq += key == T; }
+  } else {
+    gt = (uint32_t)(e1 - e0);
+  }
+  uint64_t incl = block_scan_incl(((uint64_t)gt << 32) | eq, ss);
+  uint64_t excl = incl - (((uint64_t)gt << 32) | eq);
+  uint32_t gt_b = (uint32_t)(excl >> 32), eq_b = (uint32_t)excl;
+  for (int e = e0; e < e1; ++e) {
+    const uint32_t key = keys[e];
+    bool sel;
+    int pos;
+    if (all) { sel = true; pos = (int)gt_b; ++gt_b; }
+    else if (key > T) { sel = true; pos = (int)(gt_b + min(eq_b, (uint32_t)need_eq)); ++gt_b; }
+    else if (key == T) { sel = eq_b < (uint32_t)need_eq; pos = (int)(gt_b + eq_b); ++eq_b; }
+    else { sel = false; pos = 0; }
+    if (sel) {
+      out_idx[pos] = ids ? ids[e] : (int32_t)(id_base + e);
+      if (out_key) out_key[pos] = key;
+    }
+  }
+  return min(n, k);
+}
+
+struct TopkParams {
+  const float* scores;     // [rows, cap]
+  const int64_t* q_pos;    // [n_seq]
+  int64_t cap;
+  int T, m, k, n_chunks;
+  int32_t* idx;            // final [rows, k]
+  uint32_t* cand_key;      // [rows, n_chunks, k]
+  int32_t* cand_idx;       // [rows, n_chunks, k]
+  int32_t* cand_cnt;       // [rows, n_chunks]
+};
+
+// Stage 1 (or the only stage when n_chunks == 1): one CTA per (chunk, row).
+__global__ void __launch_bounds__(kTopkThreads)
+topk_chunk_kernel(TopkParams p) {
+  extern __shared__ uint32_t s_keys[];   // kChunk
+  __shared__ SelectSmem ss;
+  const int64_t row = blockIdx.x;
+  const int chunk = blockIdx.y;
+  const int b = (int)(row / p.T), t = (int)(row % p.T);
+  const int64_t nv = min(p.cap, (p.q_pos[b] + t + 1) / p.m);
+  const int64_t lo = (int64_t)chunk * kChunk;
+  const int n = (int)max((int64_t)0, min((int64_t)kChunk, nv - lo));
+  const float* src = p.scores + row * p.cap + lo;
+  for (int e = threadIdx.x; e < n; e += kTopkThreads) s_keys[e] = order_key(src[e]);
+  __syncthreads();
+  if (p.n_chunks == 1) {
+    int32_t* out = p.idx + row * p.k;
+    int cnt = block_select(s_keys, nullptr, lo, n, p.k, out, nullptr, ss);
+    for (int i = cnt + threadIdx.x; i < p.k; i += kTopkThreads) out[i] = -1;
+  } else {
+    const int64_t o = (row * p.n_chunks + chunk) * p.k;
+    int cnt = block_select(s_keys, nullptr, lo, n, p.k, p.cand_idx + o, p.cand_key + o, ss);
+    if (threadIdx.x == 0) p.cand_cnt[row * p.n_chunks + chunk] = cnt;
+  }
+}
+
+// Stage 2: merge the chunk candidates of one row (chunk order keeps the
+// candidates in ascending entry order).
+__global__ void __launch_bounds__(kTopkThreads)
+topk_merge_kernel(TopkParams p) {
+  extern __shared__ uint32_t s_mem[];
+  uint32_t* s_keys = s_mem;                                   // kMergeCap
+  int32_t* s_ids = reinterpret_cast<int32_t*>(s_mem + kMergeCap);
+  __shared__ SelectSmem ss;
+  __shared__ int s_off[65];
+  const int64_t row = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int c = 0; c < p.n_chunks; ++c) { s_off[c] = acc; acc += p.cand_cnt[row * p.n_chunks + c]; }
+    s_off[p.n_chunks] = acc;
+  }
+  __syncthreads();
+  const int n = s_off[p.n_chunks];
+  for (int c = 0; c < p.n_chunks; ++c) {
+    const int cnt = s_off[c + 1] - s_off[c];
+    const int64_t o = (row * p.n_chunks + c) * p.k;
+    for (int i = threadIdx.x; i < cnt; i += kTopkThreads) {
+      s_keys[s_off[c] + i] = p.cand_key[o + i];
+      s_ids[s_off[c] + i] = p.cand_idx[o + i];
+    }
+  }
+  __syncthreads();
+  int32_t* out = p.idx + row * p.k;
+  int cnt = block_select(s_keys, s_ids, 0, n, p.k, out, nullptr, ss);
+  for (int i = cnt + threadIdx.x; i < p.k; i += kTopkThreads) out[i] = -1;
+}
+
+struct WsLayout {
+  size_t scores, cand_key, cand_idx, cand_cnt, total;
+  int n_chunks;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WsLayout ws_layout(int n_seq, int T, int64_t cap, int k) {
+  WsLayout L{};
+  const size_t rows = (size_t)n_seq * (size_t)T;
+  L.n_chunks = (int)((cap + kChunk - 1) / kChunk);
+  size_t off = 0;
+  L.scores = off; off = align_up(off + rows * (size_t)cap * 4, 256);
+  if (L.n_chunks > 1) {
+    L.cand_key = off; off = align_up(off + rows * L.n_chunks * (size_t)k * 4, 256);
+    L.cand_idx = off; off = align_up(off + rows * L.n_chunks * (size_t)k * 4, 256);
+    L.cand_cnt = off; off = align_up(off + rows * L.n_chunks * 4, 256);
+  }
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" size_t csa_index_topk_workspace(int n_seq, int T, int64_t cap, int k) {
+  if (n_seq <= 0 || T <= 0 || cap <= 0 || k <= 0) return 0;
+  return ws_layout(n_seq, T, cap, k).total;
+}
+
+extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale, const float* w,
+                                       const uint8_t* kI, const float* kI_scale, const int64_t* q_pos,
+                                       int n_seq, int T, int HI, int DI, int64_t cap, int m, int k,
+                                       int32_t* idx, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(n_seq >= 1 && T >= 1 && cap >= 1 && m >= 1, "csa_index_topk: n_seq, T, cap, m must be >= 1");
+  CSA_REQUIRE(DI == 32 || DI == 64 || DI == 128, "csa_index_topk: DI must be 32, 64 or 128");
+  CSA_REQUIRE(HI >= 1 && HI <= 64 && (HI & (HI - 1)) == 0, "csa_index_topk: HI must be a power of two <= 64");
+  CSA_REQUIRE(k >= 1 && k <= 2048, "csa_index_topk: k must be in [1, 2048]");
+  CSA_REQUIRE(qI && w && kI && q_pos && idx, "csa_index_topk: null pointer");
+  CSA_REQUIRE(aligned16(qI) && aligned16(kI) && aligned16(w) && aligned16(idx) && aligned16(q_pos) &&
+              (!qI_scale || aligned16(qI_scale)) && (!kI_scale || aligned16(kI_scale)),
+              "csa_index_topk: pointers must be 16-byte aligned");
+  CSA_REQUIRE((int64_t)n_seq * cap < (int64_t)1 << 31 && (int64_t)n_seq * T * HI < (int64_t)1 << 31,
+              "csa_index_topk: tensor too large for 32-bit TMA coordinates");
+  const WsLayout L = ws_layout(n_seq, T, cap, k);
+  if (!workspace || ws_bytes < L.total)
+    return fail(CSA_ERR_WORKSPACE, "csa_index_topk: workspace of %zu bytes needed, %zu given", L.total, ws_bytes);
+  CSA_REQUIRE(aligned16(workspace), "csa_index_topk: workspace must be 16-byte aligned");
+  if (L.n_chunks > 1 && (int64_t)L.n_chunks * k > kMergeCap)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: ceil(cap/%d) * k = %lld exceeds %d merge candidates",
+                kChunk, (long long)L.n_chunks * k, kMergeCap);
+  CSA_REQUIRE(L.n_chunks <= 64, "csa_index_topk: cap too large");
+
+  // token block: N = TQ * HI columns, a multiple of 16 and at most 256
+  int TQ = 256 / HI;
+  while (TQ > 1 && (TQ / 2) * HI >= 16 && TQ / 2 >= T) TQ /= 2;
+  const int N = TQ * HI;
+  if (N % 16 != 0) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: HI=%d gives no valid MMA width", HI);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  IdxParams ip{};
+  ip.qs = qI_scale; ip.w = w; ip.ks = kI_scale; ip.q_pos = q_pos;
+  ip.scores = reinterpret_cast<float*>(ws + L.scores);
+  ip.cap = cap; ip.T = T; ip.HI = HI; ip.DI = DI; ip.m = m; ip.TQ = TQ; ip.N = N;
+
+  const int n_qblocks = (T + TQ - 1) / TQ;
+  const int64_t tiles = (cap + 127) / 128;
+  int64_t n_kchunks = 1;
+  const int64_t ctas = (int64_t)n_seq * n_qblocks;
+  const int sms = num_sms();
+  if (ctas < sms) n_kchunks = std::max<int64_t>(1, std::min<int64_t>(tiles, sms / ctas));
+  ip.tiles_per_chunk = (int)((tiles + n_kchunks - 1) / n_kchunks);
+  n_kchunks = (tiles + ip.tiles_per_chunk - 1) / ip.tiles_per_chunk;
+  CSA_REQUIRE(n_qblocks <= 65535 && n_seq <= 65535, "csa_index_topk: grid too large");
+
+  CUtensorMap mk, mq;
+  if (!make_byte_map(&mk, kI, (uint64_t)n_seq * cap, DI, 128) ||
+      !make_byte_map(&mq, qI, (uint64_t)n_seq * T * HI, DI, N))
+    return fail(CSA_ERR_CUDA, "csa_index_topk: cuTensorMapEncodeTiled failed");
+
+  const size_t smem = 1024 + ((N * DI + 1023) / 1024) * 1024 + (size_t)kStages * 128 * DI +
+                      (2 * kStages + 5) * 8 + 16 + N * 4;
+  cudaFuncSetAttribute(indexer_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid((unsigned)n_kchunks, (unsigned)n_qblocks, (unsigned)n_seq);
+  indexer_scores_kernel<<<grid, kIdxThreads, smem, stream>>>(mk, mq, ip);
+  csa_status_t st = check_launch("csa_index_topk(scores)");
+  if (st != CSA_OK) return st;
+
+  TopkParams tp{};
+  tp.scores = ip.scores; tp.q_pos = q_pos; tp.cap = cap; tp.T = T; tp.m = m; tp.k = k;
+  tp.n_chunks = L.n_chunks; tp.idx = idx;
+  tp.cand_key = reinterpret_cast<uint32_t*>(ws + L.cand_key);
+  tp.cand_idx = reinterpret_cast<int32_t*>(ws + L.cand_idx);
+  tp.cand_cnt = reinterpret_cast<int32_t*>(ws + L.cand_cnt);
+  const int64_t rows = (int64_t)n_seq * T;
+  CSA_REQUIRE(rows <= 0x7fffffff, "csa_index_topk: too many rows");
+  const size_t smem1 = kChunk * sizeof(uint32_t);
+  cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  dim3 g1((unsigned)rows, (unsigned)L.n_chunks);
+  topk_chunk_kernel<<<g1, kTopkThreads, smem1, stream>>>(tp);
+  st = check_launch("csa_index_topk(select)");
+  if (st != CSA_OK) return st;
+  if (L.n_chunks > 1) {
+    const size_t smem2 = kMergeCap * 8;
+    cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
+    topk_merge_kernel<<<(unsigned)rows, kTopkThreads, smem2, stream>>>(tp);
+    st = check_launch("csa_index_topk(merge)");
+  }
+  return st;
+}

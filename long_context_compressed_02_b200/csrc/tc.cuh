@@ -46,13 +46,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
                : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-// Bounded wait: each try_wait may suspend for a hardware time slice, so the
-// limit below is generous (seconds).  On expiry the error word is set and the
-// caller proceeds; results are then garbage but the context stays usable.
-constexpr uint32_t kSpinLimit = 1u << 26;
+// Bounded waits: a wait gives up after kWaitNs of wall time (read from the
+// %globaltimer nanosecond clock every 256 polls), records the expiry in the
+// error word and returns false; callers then leave their loops, so a logic
+// error can never hold the GPU.
+constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  uint64_t start = 0;
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0) {
+      const uint64_t now = global_ns();
+      if (start == 0) start = now;
+      else if (now - start > kWaitNs) break;
+    }
   }
   if (err) atomicOr(err, DEV_ERR_TIMEOUT_MBAR);
   return false;

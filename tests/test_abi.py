@@ -1,0 +1,92 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point declared in include/csa.h, and rejects bad arguments on the host before
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(csa_\w+|hca_\w+|swa_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from long_context_compressed_02_b200 import build, lib
+    build.build()
+    return lib()
+
+
+def test_header_declares_the_five_layer_entry_points():
+    d = _declared()
+    for n in ("csa_compress", "csa_index_topk", "csa_sparse_mqa", "hca_dense_attn", "swa_sink_combine"):
+        assert n in d
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.csa_abi_version() == 1
+    assert L.csa_status_string(0) == b"CSA_OK"
+    assert L.csa_status_string(3) == b"CSA_ERR_WORKSPACE"
+
+
+def test_workspace_size_is_host_arithmetic(L):
+    # prefill: one chunk, only the score matrix; decode: chunked candidates too
+    assert L.csa_index_topk_workspace(1, 16384, 4096, 512) == 16384 * 4096 * 4
+    dec = L.csa_index_topk_workspace(16, 1, 262144, 512)
+    assert dec >= 16 * 262144 * 4 + 2 * 16 * 16 * 512 * 4
+    assert L.csa_index_topk_workspace(0, 1, 1, 1) == 0
+
+
+def test_host_argument_validation(L):
+    null = None
+    # D not a multiple of 8
+    st = L.csa_compress(ctypes.c_void_p(16), ctypes.c_void_p(16), null, null, null, 64, 7, 4, 1, 0, 0, 0,
+                        10000.0, 1e-6, ctypes.c_void_p(16), 0, null)
+    assert st == 1 and b"multiple of 8" in L.csa_last_error()
+    # misaligned pointer
+    st = L.csa_compress(ctypes.c_void_p(17), ctypes.c_void_p(16), null, null, null, 64, 8, 4, 1, 0, 0, 0,
+                        10000.0, 1e-6, ctypes.c_void_p(16), 0, null)
+    assert st == 1 and b"aligned" in L.csa_last_error()
+    # indexer: DI unsupported
+    st = L.csa_index_topk(ctypes.c_void_p(16), null, ctypes.c_void_p(16), ctypes.c_void_p(16), null,
+                          ctypes.c_void_p(16), 1, 1, 4, 48, 8, 4, 4, ctypes.c_void_p(16), ctypes.c_void_p(16), 1 << 20,
+                          null)
+    assert st == 1 and b"DI" in L.csa_last_error()
+    # indexer: workspace too small
+    st = L.csa_index_topk(ctypes.c_void_p(16), null, ctypes.c_void_p(16), ctypes.c_void_p(16), null,
+                          ctypes.c_void_p(16), 1, 8, 4, 32, 64, 4, 4, ctypes.c_void_p(16), ctypes.c_void_p(16), 8,
+                          null)
+    assert st == 3
+    # attention: unsupported head dim
+    st = L.csa_sparse_mqa(ctypes.c_void_p(16), 1, ctypes.c_void_p(16), 1, null, null, 16, ctypes.c_void_p(16), 4,
+                          1, 1, 8, 96, 0, 0.1, ctypes.c_void_p(16), ctypes.c_void_p(16), null)
+    assert st == 1 and b"D must be" in L.csa_last_error()
+    # e4m3 store without its RoPE part
+    st = L.hca_dense_attn(ctypes.c_void_p(16), 1, ctypes.c_void_p(16), 2, null, null, 16, ctypes.c_void_p(16), 128,
+                          1, 1, 8, 512, 64, 0.1, ctypes.c_void_p(16), ctypes.c_void_p(16), null)
+    assert st == 1 and b"e4m3" in L.csa_last_error()
+    # combine: inverse RoPE without RoPE dims
+    st = L.swa_sink_combine(ctypes.c_void_p(16), 1, ctypes.c_void_p(16), 1, 16, ctypes.c_void_p(16), 128, 0, null,
+                            null, null, 1, 1, 8, 512, 0, 10000.0, 1, 0.1, ctypes.c_void_p(16), 1, null)
+    assert st == 1 and b"inv_rope" in L.csa_last_error()
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    import long_context_compressed_02_b200 as csa
+    with pytest.raises(csa.CsaError):
+        csa.csa_compress(torch.zeros(8, 8), torch.zeros(8, 8), torch.zeros(8, 8), 4, True)

@@ -1,0 +1,145 @@
+"""GPU parity: tcgen05 shared-KV attention (sparse, dense, window + sink) vs
+the float64 oracle on the same (bf16 / e4m3-valued) inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gpu_util import assert_close, cuda, host, lib_loaded
+from long_context_compressed_02_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    lib_loaded()
+
+
+def _bf16(rng, shape, scale=1.0):
+    return synth.to_bf16_values(rng.standard_normal(shape) * scale)
+
+
+def _rand_idx(rng, T, k, ne, sizes):
+    idx = np.full((T, k), -1, np.int32)
+    for t in range(T):
+        n = sizes[t % len(sizes)]
+        n = min(n, ne, k)
+        idx[t, :n] = np.sort(rng.choice(ne, n, replace=False))
+    return idx
+
+
+@pytest.mark.parametrize("H,D,dt", [(64, 512, "bf16"), (8, 128, "f32"), (64, 128, "bf16")])
+def test_sparse_partial(H, D, dt):
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(1)
+    T, ne, k = 70, 1000, 512
+    q = O.rmsnorm(rng.standard_normal((T, H, D)))
+    kv = O.rmsnorm(rng.standard_normal((ne, D)))
+    if dt == "bf16":
+        q, kv = synth.to_bf16_values(q), synth.to_bf16_values(kv)
+        tq = cuda(q, torch.bfloat16); tkv = cuda(kv, torch.bfloat16)
+    else:
+        q, kv = q.astype(np.float32), kv.astype(np.float32)
+        tq = cuda(q); tkv = cuda(kv)
+    idx = _rand_idx(rng, T, k, ne, [512, 0, 1, 127, 128, 129, 300, 511, 256])
+    Og, Lg = csa.csa_sparse_mqa(tq[None], tkv[None], cuda(idx)[None])
+    csa.check_device_error()
+    Or, Lr = O.sparse_attention_partial(q, kv, idx)
+    has = (idx >= 0).any(axis=1)
+    assert_close(host(Og)[0][has], Or[has], what="O_part")
+    assert np.all(host(Og)[0][~has] == 0) and np.all(np.isneginf(host(Lg)[0][~has]))
+    assert_close(host(Lg)[0][has], Lr[has], max_abs=1e-2, rel_l2=1e-3, what="lse")
+
+
+def test_sparse_partial_e4m3_store():
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(2)
+    gen = torch.Generator(device="cuda").manual_seed(2)
+    ne, D, H, T, k = 3000, 512, 64, 4, 512
+    cache = synth.decode_csa_cache(ne, D, 128, 64, gen, "cuda")
+    q = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((T, H, D))) * 0.5)
+    idx = _rand_idx(rng, T, k, ne, [512, 200, 1, 129])
+    Og, Lg = csa.csa_sparse_mqa(cuda(q, torch.bfloat16)[None], cache["kv_nope"][None], cuda(idx)[None],
+                                kv_rope=cache["kv_rope"][None], kv_scale=cache["kv_scale"][None])
+    csa.check_device_error()
+    kv = np.concatenate([O.e4m3_decode(cache["kv_nope"].cpu().numpy()) * cache["kv_scale"].cpu().numpy()[:, None],
+                         cache["kv_rope"].float().cpu().numpy()], axis=1)
+    Or, Lr = O.sparse_attention_partial(q, kv, idx, scale=1 / math.sqrt(D))
+    assert_close(host(Og)[0], Or, what="e4m3 O_part")
+    assert_close(host(Lg)[0], Lr, max_abs=2e-2, rel_l2=1e-3, what="e4m3 lse")
+
+
+def test_dense_partial_multi_chunk():
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(3)
+    T, cap, H, D, m = 40, 700, 64, 512, 128
+    q = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((T, H, D))))
+    kv = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((cap, D))))
+    pos0 = 128 * 520 - 20                         # n_vis crosses 520 -> 521 inside the block
+    Og, Lg = csa.hca_dense_attn(cuda(q, torch.bfloat16)[None], cuda(kv, torch.bfloat16)[None],
+                                cuda(np.array([pos0], np.int64)), m)
+    csa.check_device_error()
+    Or, Lr = O.dense_attention_partial(q, kv, O.n_visible(pos0 + np.arange(T), m))
+    assert_close(host(Og)[0], Or, what="dense O_part")
+    assert_close(host(Lg)[0], Lr, max_abs=1e-2, rel_l2=1e-3, what="dense lse")
+
+
+@pytest.mark.parametrize("with_partial,inv_rope", [(True, True), (False, False), (True, False)])
+def test_window_sink_combine_prefill(with_partial, inv_rope):
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(4)
+    S, H, D, W = 300, 64, 512, 128
+    q = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((S, H, D))))
+    kt = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((S, D))))
+    sink = rng.standard_normal(H).astype(np.float32)
+    Op = (0.3 * rng.standard_normal((S, H, D))).astype(np.float32)
+    Lp = rng.standard_normal((S, H)).astype(np.float32)
+    Lp[5] = -np.inf; Op[5] = 0                       # an empty compressed branch
+    pos = np.array([0], np.int64)
+    out = csa.swa_sink_combine(cuda(q, torch.bfloat16)[None], cuda(kt, torch.bfloat16)[None], cuda(pos), W,
+                               cuda(sink), cuda(Op)[None] if with_partial else None,
+                               cuda(Lp)[None] if with_partial else None, inv_rope=inv_rope,
+                               rope_dim=64, out_dtype=torch.float32)
+    csa.check_device_error()
+    if not with_partial:
+        Op2 = np.zeros_like(Op); Lp2 = np.full_like(Lp, -np.inf)
+    else:
+        Op2, Lp2 = Op, Lp
+    ref = O.window_sink_combine(q, kt, np.arange(S), W, sink, Op2, Lp2, inv_rope=inv_rope)
+    assert_close(host(out)[0], ref, what="combine")
+
+
+def test_window_cache_decode_batch():
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(5)
+    n_seq, H, D, W = 5, 64, 512, 128
+    q = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((n_seq, 1, H, D))))
+    swa = synth.to_bf16_values(rng.standard_normal((n_seq, W, D)))
+    sink = rng.standard_normal(H).astype(np.float32)
+    pos = np.array([1 << 20, 3, 127, 128, 5000], np.int64)
+    out = csa.swa_sink_combine(cuda(q, torch.bfloat16), cuda(swa, torch.bfloat16), cuda(pos), W, cuda(sink),
+                               window_mode=1, inv_rope=True, out_dtype=torch.float32)
+    csa.check_device_error()
+    for b in range(n_seq):
+        nrow = min(W, pos[b] + 1)
+        ref = O.window_sink_combine(q[b], None, [pos[b]], W, sink, np.zeros((1, H, D)), np.full((1, H), -np.inf),
+                                    inv_rope=True, window_rows=[swa[b][:nrow]])
+        assert_close(host(out)[b], ref, what=f"decode window b={b}")
+
+
+def test_batch_invariance_bit_exact():
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(6)
+    n_seq, T, ne, H, D, k = 16, 3, 900, 64, 512, 512
+    q = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((n_seq, T, H, D))))
+    kv = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((n_seq, ne, D))))
+    idx = np.stack([_rand_idx(rng, T, k, ne, [512, 300, 77]) for _ in range(n_seq)])
+    tq, tkv, ti = cuda(q, torch.bfloat16), cuda(kv, torch.bfloat16), cuda(idx)
+    Ob, Lb = csa.csa_sparse_mqa(tq, tkv, ti)
+    for b in (0, 7, 15):
+        Oa, La = csa.csa_sparse_mqa(tq[b:b + 1].contiguous(), tkv[b:b + 1].contiguous(), ti[b:b + 1].contiguous())
+        assert torch.equal(Oa[0], Ob[b]) and torch.equal(La[0], Lb[b])
+    csa.check_device_error()

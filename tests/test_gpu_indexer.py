@@ -1,0 +1,116 @@
+"""GPU parity: FP8 lightning indexer + top-k vs the float64 oracle.
+
+On grid inputs (values multiples of 1/8, head weights of 1/16) every score is
+exact in fp32, so the selected index sets must be bit-identical.  On the
+continuous distribution the sets may differ only by entries whose oracle
+score lies within the fp32 rounding bound of the k-th score."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gpu_util import cuda, lib_loaded
+from long_context_compressed_02_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    lib_loaded()
+
+
+def _run(qI_codes, w, kI_codes, q_pos, m, k, qs=None, ks=None):
+    import long_context_compressed_02_b200 as csa
+    idx = csa.csa_index_topk(cuda(qI_codes), cuda(w), cuda(kI_codes), cuda(np.asarray(q_pos, np.int64)), m, k,
+                             qI_scale=None if qs is None else cuda(qs), kI_scale=None if ks is None else cuda(ks))
+    csa.check_device_error()
+    return idx.cpu().numpy()
+
+
+def _oracle(qI_codes, w, kI_codes, q_pos, m, k, qs=None, ks=None):
+    n_seq, T = qI_codes.shape[:2]
+    out = np.zeros((n_seq, T, k), np.int32)
+    for b in range(n_seq):
+        qI = O.e4m3_decode(qI_codes[b])
+        if qs is not None:
+            qI = qI * qs[b][..., None]
+        kI = O.e4m3_decode(kI_codes[b])
+        if ks is not None:
+            kI = kI * ks[b][:, None]
+        nv = np.minimum(kI.shape[0], O.n_visible(q_pos[b] + np.arange(T), m))
+        s = O.indexer_scores(qI, w[b], kI, nv)
+        out[b] = O.topk_select(s, nv, k)
+    return out
+
+
+def test_tiny_csa_bit_exact():
+    inp, cfg = synth.prefill_inputs("tiny_csa")
+    args = (inp["qI_codes"][None], inp["w"][None], inp["kI_codes"][None], [0], 4, 64)
+    got = _run(*args)
+    ref = _oracle(*args)
+    assert np.array_equal(got, ref)
+    # rows before the first complete entry select nothing
+    assert np.all(got[0, :3] == -1) and got[0, 3, 0] == 0 and np.all(got[0, 3, 1:] == -1)
+
+
+@pytest.mark.parametrize("S,k", [(2048, 64), (4100, 512), (777, 1000)])
+def test_flash_shaped_grid_bit_exact(S, k):
+    inp, cfg = synth.prefill_inputs("csa_prefill", S=S, grid=True)
+    args = (inp["qI_codes"][None], inp["w"][None], inp["kI_codes"][None], [0], 4, k)
+    got = _run(*args)
+    ref = _oracle(*args)
+    assert np.array_equal(got, ref)
+
+
+def test_decode_chunked_rows_with_scales_bit_exact():
+    rng = np.random.default_rng(5)
+    n_seq, cap, HI, DI, m, k = 3, 40000, 64, 128, 4, 512
+    kI = synth.grid_codes(rng, (n_seq, cap, DI))
+    qI = synth.grid_codes(rng, (n_seq, 1, HI, DI))
+    w = (np.floor(rng.random((n_seq, 1, HI)) * 16) / 16).astype(np.float32)
+    ks = np.ones((n_seq, cap), np.float32)
+    qs = np.ones((n_seq, 1, HI), np.float32)
+    ks[:, ::7] = 0.5                     # power-of-two scales keep every score exact
+    qs[:, :, ::3] = 2.0
+    q_pos = [4 * cap - 1, 70001, 5]
+    got = _run(qI, w, kI, q_pos, m, k, qs, ks)
+    ref = _oracle(qI, w, kI, q_pos, m, k, qs, ks)
+    assert np.array_equal(got, ref)
+    assert np.all(got[2, 0, 1:] == -1) and got[2, 0, 0] == 0
+
+
+def test_ties_go_to_lower_index():
+    # all keys identical: every score ties, the first k visible entries win
+    rng = np.random.default_rng(6)
+    T, ne, HI, DI = 40, 300, 8, 32
+    k1 = synth.grid_codes(rng, (1, DI))
+    kI = np.repeat(k1, ne, axis=0)[None]
+    qI = synth.grid_codes(rng, (1, T, HI, DI))
+    w = np.ones((1, T, HI), np.float32)
+    got = _run(qI, w, kI, [4 * 200], 4, 50)
+    assert np.array_equal(got[0], np.repeat(np.arange(50, dtype=np.int32)[None], T, 0))
+
+
+def test_continuous_inputs_within_rounding_bound():
+    inp, cfg = synth.prefill_inputs("csa_prefill", S=3000, grid=False)
+    k = 256
+    args = (inp["qI_codes"][None], inp["w"][None], inp["kI_codes"][None], [0], 4, k)
+    got = _run(*args)[0]
+    qI = O.e4m3_decode(inp["qI_codes"]); kI = O.e4m3_decode(inp["kI_codes"])
+    nv = O.n_visible(np.arange(3000), 4)
+    s = O.indexer_scores(qI, inp["w"], kI, nv)
+    ref = O.topk_select(s, nv, k)
+    mism = 0
+    for t in range(3000):
+        a = set(got[t][got[t] >= 0].tolist()); b = set(ref[t][ref[t] >= 0].tolist())
+        assert len(a) == len(b) == min(k, nv[t])
+        if a == b:
+            continue
+        mism += 1
+        kth = np.sort(s[t, :nv[t]])[::-1][min(k, nv[t]) - 1]
+        # fp32 bound: relative 2^-20 of the sum of |terms| is far above the real rounding error
+        bound = 1e-5 * (np.abs(inp["w"][t])[:, None] * np.abs(qI[t] @ kI[:nv[t]].T)).sum(axis=0).max()
+        for e in a ^ b:
+            assert abs(s[t, e] - kth) <= bound, (t, e, s[t, e], kth, bound)
+    assert mism < 30
