@@ -1,0 +1,322 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA layer forward on B200 (Flash-shaped prefill:
+S 16384, 64 heads x 512, m 4 with overlap -> 4096 entries, e4m3 indexer
+64 x 128, top-k 512, window 128, sink).
+
+One step = the whole hot path of the layer, in the library's kernels:
+  Q RMSNorm+RoPE, window-row RMSNorm+RoPE, compressor (+ K norm/RoPE),
+  lightning indexer + top-k, sparse shared-KV MQA, window + sink combine.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs an independent
+replica of the workload (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import signal
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA decode tokens/s @1M ctx and prefill TFLOP/s, % of HBM/TC roofline"
+WORKLOAD = "csa_prefill"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _flops(S, H, D, m, k, W, HI, DI):
+    t = np.arange(S, dtype=np.int64)
+    nv = (t + 1) // m
+    sparse = 4 * D * H * int(np.minimum(k, nv).sum())
+    window = 4 * D * H * int(np.minimum(W, t + 1).sum())
+    indexer = 2 * HI * DI * int(nv.sum())
+    return sparse, window, indexer
+
+
+class Clocks:
+    """Samples nvidia-smi during the timed region."""
+
+    def __init__(self, index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.send_signal(signal.SIGTERM)
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        with open(self.f.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_oracle_sample(inp_host, cfg, rows):
+    """Times the float64 oracle on the given query rows of the workload."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    O.csa_layer(inp_host["q"][rows], inp_host["C"], inp_host["Z"], inp_host["B"],
+                O.e4m3_decode(inp_host["qI_codes"][rows]), inp_host["w"][rows],
+                O.e4m3_decode(inp_host["kI_codes"]), inp_host["sink"], k=cfg["k"], m=cfg["m"], W=cfg["W"],
+                norm_rope=True, inv_rope=True, rows=rows, row_inputs=True)
+    dt = time.perf_counter() - t0
+    t = np.asarray(rows, np.int64)
+    nv = (t + 1) // cfg["m"]
+    fl = (4 * cfg["D"] * cfg["H"] * (np.minimum(cfg["k"], nv) + np.minimum(cfg["W"], t + 1)).sum()
+          + 2 * cfg["HI"] * cfg["DI"] * nv.sum())
+    return float(fl), dt, cores
+
+
+def host_inputs(dev_inp):
+    """float32 / uint8 numpy copies of the workload tensors."""
+    import torch
+    return {k: (v.cpu().numpy() if v.dtype == torch.uint8 else v.float().cpu().numpy()) for k, v in dev_inp.items()}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the float64 CPU oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import torch
+    from long_context_compressed_02_b200 import synth
+    inp, cfg = synth.prefill_inputs_device(WORKLOAD, "cpu", seed=0)
+    host = host_inputs(inp)
+    rng = np.random.default_rng(0)
+    times, flops = [], []
+    cores = 1
+    for step in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(cfg["S"], 8, replace=False))
+        fl, dt, cores = cpu_oracle_sample(host, cfg, rows)
+        if step >= args.warmup:
+            times.append(dt)
+            flops.append(fl)
+    value = sum(flops) / sum(times) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "S": cfg["S"], "H": cfg["H"], "D": cfg["D"], "m": cfg["m"],
+                       "top_k": cfg["k"], "window": cfg["W"], "sample": "8 random query rows per step"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": "8 random query rows of the S=16384 layer per step (oracle recomputes the "
+                                       "compressor and window rows each call)"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--S", type=int, default=None, help="shorter sequence (profiling cases only)")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    import long_context_compressed_02_b200 as csa
+    from long_context_compressed_02_b200 import build, synth
+    build.build()
+    csa.lib()
+
+    inp, cfg = synth.prefill_inputs_device(WORKLOAD, dev, seed=rank, S=args.S)
+    S, H, D, m, k, W, HI, DI = (cfg[x] for x in ("S", "H", "D", "m", "k", "W", "HI", "DI"))
+    ne = S // m
+    bf = torch.bfloat16
+    pos = torch.zeros(1, dtype=torch.int64, device=dev)
+    # persistent buffers (the library allocates nothing)
+    qn = torch.empty(S, H, D, dtype=bf, device=dev)
+    kt = torch.empty(S, D, dtype=bf, device=dev)
+    kv = torch.empty(ne, D, dtype=bf, device=dev)
+    idx = torch.empty(1, S, k, dtype=torch.int32, device=dev)
+    ws = torch.empty(csa.csa_index_topk_workspace(1, S, ne, k), dtype=torch.uint8, device=dev)
+    Op = torch.empty(1, S, H, D, dtype=torch.float32, device=dev)
+    Lp = torch.empty(1, S, H, dtype=torch.float32, device=dev)
+    out = torch.empty(1, S, H, D, dtype=bf, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ["q_norm_rope", "kv_tok_norm_rope", "compress", "index_topk", "sparse_mqa", "swa_sink_combine"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        csa.csa_rmsnorm_rope(inp["q"], rows_per_pos=H, out=qn)
+        mark(1)
+        csa.csa_rmsnorm_rope(inp["C"], rows_per_pos=1, out=kt)
+        mark(2)
+        csa.csa_compress(inp["C"], inp["Z"], inp["B"], m, True, norm=True, rope_dim=64, out=kv)
+        mark(3)
+        csa.csa_index_topk(inp["qI_codes"][None], inp["w"][None], inp["kI_codes"][None], pos, m, k,
+                           workspace=ws, idx=idx)
+        mark(4)
+        csa.csa_sparse_mqa(qn[None], kv[None], idx, out=(Op, Lp))
+        mark(5)
+        csa.swa_sink_combine(qn[None], kt[None], pos, W, inp["sink"], Op, Lp, inv_rope=True, rope_dim=64,
+                             out=out)
+        mark(6)
+
+    launches_per_step = 7      # 2 norm/rope, compress, scores, top-k, sparse MQA, combine
+    for _ in range(max(3, args.warmup)):
+        step()
+    csa.check_device_error()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clocks = Clocks(torch.cuda.current_device()) if rank == 0 else None
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    csa.check_device_error()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    per = {n: float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]))
+           for j, n in enumerate(names)}
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    fl_sparse, fl_window, fl_index = _flops(S, H, D, m, k, W, HI, DI)
+    fl_total = fl_sparse + fl_window + fl_index
+    value = world * fl_total / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if rank == 0 and not args.no_e2e:
+        keys = ["q", "C", "Z", "B", "qI_codes", "w", "kI_codes", "sink"]
+        pinned = {kk: torch.empty(inp[kk].shape, dtype=inp[kk].dtype, pin_memory=True) for kk in keys}
+        for kk in keys:
+            pinned[kk].copy_(inp[kk])
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(pinned[kk].numel() * pinned[kk].element_size() for kk in keys)
+        d2h = out_host.numel() * out_host.element_size()
+        n_e2e = max(2, min(args.steps, 5))
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            for kk in keys:
+                inp[kk].copy_(pinned[kk], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / n_e2e
+        e2e = {"value": fl_total / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # ---- roofline of the dominant call
+    hbm, bf16_burst, bf16_sus, src = _peaks()
+    algo = {"sparse_mqa": (fl_sparse, "tensor", bf16_sus), "swa_sink_combine": (fl_window, "tensor", bf16_sus),
+            "index_topk": (fl_index, "tensor", 2 * bf16_sus)}
+    dom = max(per, key=per.get)
+    if dom in algo:
+        fl, bound, peak = algo[dom]
+        ach = fl / (per[dom] * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": None,
+                "peak_source": f"{src} bf16 sustained" + (" x2 (fp8 nominal ratio)" if dom == "index_topk" else "")}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s", "frac": None,
+                "traffic": None}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = host_inputs(inp)
+        rows = np.linspace(0, S - 1, 32).astype(np.int64)
+        fl, dt, cores = cpu_oracle_sample(host, cfg, rows)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": "32 evenly spaced query rows of the same S=16384 layer (float64 numpy oracle, "
+                         f"{dt:.1f} s including its full-sequence compressor and window-row passes)"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD if args.S is None else f"{WORKLOAD}_S{S}", "S": S, "H": H, "D": D, "m": m, "entries": ne, "top_k": k,
+                           "window": W, "indexer": f"e4m3 {HI}x{DI}", "batch_per_gpu": 1,
+                           "parallelism": f"replicas x{world}",
+                           "l2": "inputs larger than L2 (q alone is 1 GiB)",
+                           "flops_per_step": {"sparse_mqa": fl_sparse, "swa_window": fl_window,
+                                              "indexer_fp8": fl_index}},
+                "prefill_tokens_per_s": world * S / (ms * 1e-3),
+                "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -144,3 +144,37 @@ def decode_query(H: int, D: int, HI: int, DI: int, W: int, gen: torch.Generator,
     swa = torch.randn(W, D, generator=gen, device=device).to(torch.bfloat16)
     sink = torch.randn(H, generator=gen, device=device)
     return dict(q=q, qI=qI, qI_scale=qs, w=w, swa=swa, sink=sink)
+
+
+def prefill_inputs_device(name: str, device, seed: int = 0, S: int | None = None, grid: bool = False):
+    """The same recipe as prefill_inputs, drawn on `device` with torch's seeded
+    generator (for benchmark-sized inputs).  Returns torch tensors: q [S,H,D],
+    C, Z [S,D] in the workload dtype, B [2m or m, D] f32, sink [H] f32 and, for
+    CSA, qI_codes [S,HI,DI] u8, kI_codes [n_e,DI] u8, w [S,HI] f32."""
+    cfg = dict(WORKLOADS[name])
+    S = cfg["S"] if S is None else S
+    g = torch.Generator(device=device).manual_seed(seed)
+    H, D, m = cfg["H"], cfg["D"], cfg["m"]
+    dt = torch.bfloat16 if cfg["dtype"] == "bf16" else torch.float32
+    csa = "HI" in cfg
+    out = {
+        "C": torch.randn(S, D, generator=g, device=device).to(dt),
+        "Z": torch.randn(S, D, generator=g, device=device).to(dt),
+        "B": (0.1 * torch.randn(2 * m if csa else m, D, generator=g, device=device)).to(dt).float(),
+        "q": torch.randn(S, H, D, generator=g, device=device).to(dt),
+        "sink": (torch.zeros(H, device=device) if cfg["sink"] == "zero"
+                 else torch.randn(H, generator=g, device=device)),
+    }
+    if csa:
+        HI, DI, ne = cfg["HI"], cfg["DI"], S // m
+        qI = torch.randn(S, HI, DI, generator=g, device=device)
+        kI = torch.randn(ne, DI, generator=g, device=device)
+        if grid:
+            qI, kI = torch.round(qI * 8) / 8, torch.round(kI * 8) / 8
+            w = torch.floor(torch.rand(S, HI, generator=g, device=device) * 16) / 16
+        else:
+            w = torch.rand(S, HI, generator=g, device=device)
+        out["qI_codes"] = qI.to(torch.float8_e4m3fn).view(torch.uint8)
+        out["kI_codes"] = kI.to(torch.float8_e4m3fn).view(torch.uint8)
+        out["w"] = w.contiguous()
+    return out, dict(cfg, S=S)

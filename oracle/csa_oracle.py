@@ -358,20 +358,22 @@ def _entries(C, Z, B, m, overlap, norm_rope, rope_dim, rope_base, store_round):
 
 def csa_layer(q, C, Z, B, qI, w, kI, sink, *, k: int, m: int = 4, W: int = 128,
               norm_rope: bool = False, inv_rope: bool = False, rope_dim: int = 64,
-              rope_base: float = 10000.0, store_round=None, rows=None):
+              rope_base: float = 10000.0, store_round=None, rows=None, row_inputs: bool = False):
     """CSA layer forward for query rows `rows` (default all): compress (a1),
     indexer + top-k (a3, a4), sparse MQA (a5), window + sink (a7).
     store_round rounds tensors the method stores (entries, normalised q, window
-    rows) to their storage type, e.g. bf16_round.  Returns (O, idx)."""
+    rows) to their storage type, e.g. bf16_round.  row_inputs: q, qI and w hold
+    only the selected rows (in the order of `rows`).  Returns (O, idx)."""
     S = np.asarray(C).shape[0]
     rows = np.arange(S) if rows is None else np.asarray(rows)
-    qr = np.asarray(q, np.float64)[rows]
+    sel = slice(None) if row_inputs else rows
+    qr = np.asarray(q)[sel].astype(np.float64)
     qn, kt = _prep(qr, C, rows, norm_rope, rope_dim, rope_base)
     if store_round:
         qn, kt = store_round(qn), store_round(kt)
     kv = _entries(C, Z, B, m, True, norm_rope, rope_dim, rope_base, store_round)
     nv = n_visible(rows, m)
-    idx = topk_select(indexer_scores(np.asarray(qI, np.float64)[rows], np.asarray(w)[rows], kI, nv), nv, k)
+    idx = topk_select(indexer_scores(np.asarray(qI)[sel].astype(np.float64), np.asarray(w)[sel], kI, nv), nv, k)
     Op, lp = sparse_attention_partial(qn, kv, idx)
     O = window_sink_combine(qn, kt, rows, W, sink, Op, lp, inv_rope=inv_rope,
                             rope_dim=rope_dim, rope_base=rope_base)
