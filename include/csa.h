@@ -132,6 +132,30 @@ csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale, const floa
                             int32_t* idx, void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * csa_index_topk_noalloc — csa_index_topk without a workspace argument.
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory, e.g. a plug-in inside an engine that has
+ * already reserved the GPU's memory for its own pools, or a latency-critical
+ * path that must not call cudaMalloc because it may synchronise the device.
+ * Its scratch is one file-scope device array of 32 MiB in libcsa.so, which
+ * every GPU that loads the library holds until the process exits.  Arguments
+ * and results are those of csa_index_topk; a call whose scratch would exceed
+ * 32 MiB (csa_index_topk_workspace(n_seq, T, cap, k), dominated by
+ * n_seq * T * cap * 4 bytes of scores) returns CSA_ERR_UNSUPPORTED.
+ * The first call on each device looks up the array's device address (a CUDA
+ * runtime query), so make that first call before any stream capture.  Every
+ * call on a device shares the same array and it keeps the previous call's
+ * contents (each kernel overwrites every scratch byte before reading it, so
+ * nothing needs clearing); calls that may overlap on the GPU (different
+ * streams, or host threads racing) must be serialised by the caller.  No
+ * memory is allocated or freed.
+ * ------------------------------------------------------------------------- */
+csa_status_t csa_index_topk_noalloc(const uint8_t* qI, const float* qI_scale, const float* w,
+                                    const uint8_t* kI, const float* kI_scale, const int64_t* q_pos,
+                                    int n_seq, int T, int HI, int DI, int64_t cap, int m, int k,
+                                    int32_t* idx, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Attention over one shared K = V row set per query token ([CS] "共享 KV MQA":
  * the selected compressed entries act as both key and value; one KV head
  * shared by H query heads).  Logits are scale * q_h . row; softmax over the

@@ -527,3 +527,58 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
   }
   return st;
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of csa_index_topk.  Its scratch (the score matrix
+// and the top-k candidates) lives in a fixed file-scope device array instead
+// of a caller workspace, for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace csa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB, held by every GPU that loads the library
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+}  // namespace csa
+
+extern "C" csa_status_t csa_index_topk_noalloc(const uint8_t* qI, const float* qI_scale, const float* w,
+                                               const uint8_t* kI, const float* kI_scale, const int64_t* q_pos,
+                                               int n_seq, int T, int HI, int DI, int64_t cap, int m, int k,
+                                               int32_t* idx, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(n_seq >= 1 && T >= 1 && cap >= 1 && k >= 1,
+              "csa_index_topk_noalloc: n_seq, T, cap and k must be >= 1");
+  const size_t need = csa_index_topk_workspace(n_seq, T, cap, k);
+  if (need > kNoAllocScratchBytes)
+    return fail(CSA_ERR_UNSUPPORTED,
+                "csa_index_topk_noalloc: this call needs %zu bytes of scratch but the built-in array holds %zu "
+                "(n_seq * T * cap * 4 bytes of scores must fit); use csa_index_topk with a workspace",
+                need, kNoAllocScratchBytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_index_topk_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk_noalloc: device %d out of range", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      // Host code only sees a stand-in for the array: its device address is
+      // looked up once per device, with that device current.
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess)
+        return fail(CSA_ERR_CUDA, "csa_index_topk_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return csa_index_topk(qI, qI_scale, w, kI, kI_scale, q_pos, n_seq, T, HI, DI, cap, m, k, idx, scratch,
+                        kNoAllocScratchBytes, stream);
+}
