@@ -212,6 +212,25 @@ csa_status_t swa_sink_combine(const void* q, csa_dtype_t q_dtype, const void* kv
                               int rope_dim, float rope_base, int inv_rope, float scale,
                               void* out, csa_dtype_t out_dtype, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * csa_fused_attention — the attention side of a CSA or HCA layer in one
+ * kernel: the compressed-branch rows (CSA: kv[b, idx[b,t,:]] as in
+ * csa_sparse_mqa; HCA, idx == NULL: kv[b, 0 : n_vis] with ratio m as in
+ * hca_dense_attn), the raw window rows (as in swa_sink_combine, from kv_tok
+ * with tok_cap rows per sequence) and the sink share ONE softmax ([CS]
+ * "共享 KV MQA" and "HCA"; [LD] SWA channel and attention sink), followed by
+ * the optional inverse RoPE of the output.  Same result as csa_sparse_mqa /
+ * hca_dense_attn followed by swa_sink_combine, without the fp32 partials.
+ *   kv_tok dtype must be BF16 (F32 when kv is F32).  out [n_seq, T, H, D].
+ * ------------------------------------------------------------------------- */
+csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, const void* kv, csa_dtype_t kv_dtype,
+                                 const void* kv_rope, const float* kv_scale, int64_t cap,
+                                 const int32_t* idx, int k, int m, const void* kv_tok,
+                                 csa_dtype_t tok_dtype, int64_t tok_cap, int W, int window_mode,
+                                 const int64_t* q_pos, const float* sink, int n_seq, int T, int H,
+                                 int D, int rope_dim, float rope_base, int inv_rope, float scale,
+                                 void* out, csa_dtype_t out_dtype, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -7,7 +7,7 @@ fails, an exception is raised.
 
 Entry points (same names as the C ABI):
   csa_compress, csa_rmsnorm_rope, csa_index_topk, csa_sparse_mqa,
-  hca_dense_attn, swa_sink_combine
+  hca_dense_attn, swa_sink_combine, csa_fused_attention
 and two compositions of them: csa_layer_prefill, hca_layer_prefill.
 """
 from __future__ import annotations
@@ -52,6 +52,9 @@ def lib():
         "csa_sparse_mqa": ([P, I, P, I, P, P, I64, P, I, I, I, I, I, I, F, P, P, P], I),
         "hca_dense_attn": ([P, I, P, I, P, P, I64, P, I, I, I, I, I, I, F, P, P, P], I),
         "swa_sink_combine": ([P, I, P, I, I64, P, I, I, P, P, P, I, I, I, I, I, F, I, F, P, I, P], I),
+        "csa_fused_attention": ([P, I, P, I, P, P, I64, P, I, I, P, I, I64, I, I, P, P, I, I, I, I, I, F, I, F,
+                                 P, I, P], I),
+        "csa_index_topk_noalloc": ([P, P, P, P, P, P, I, I, I, I, I64, I, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -205,10 +208,36 @@ def swa_sink_combine(q, kv_tok, q_pos, W, sink, O_part=None, lse_part=None, *, w
     return out
 
 
+def csa_fused_attention(q, kv, kv_tok, q_pos, W, sink, *, idx=None, m=1, kv_rope=None, kv_scale=None,
+                        window_mode=0, inv_rope=False, rope_dim=None, rope_base=10000.0, scale=None,
+                        out_dtype=None, out=None, stream=None):
+    """Compressed rows (idx given: gathered top-k entries; else the dense prefix
+    of complete m-entries) + raw window rows + sink in one softmax, then the
+    optional inverse RoPE.  q [n_seq, T, H, D]; kv [n_seq, cap, D] (or e4m3 +
+    kv_rope + kv_scale); kv_tok [n_seq, tok_cap, D]."""
+    for t, n in ((q, "q"), (kv, "kv"), (kv_tok, "kv_tok"), (q_pos, "q_pos"), (sink, "sink"), (idx, "idx"),
+                 (kv_rope, "kv_rope"), (kv_scale, "kv_scale")):
+        _dev(t, n)
+    n_seq, T, H, D = q.shape
+    rope_dim = (64 if (kv.dtype == torch.uint8 or inv_rope) else 0) if rope_dim is None else rope_dim
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((n_seq, T, H, D), dtype=out_dtype, device=q.device)
+    k = 0 if idx is None else idx.shape[-1]
+    kvd, kvp, kvr, kvs = _kv_args(kv, kv_rope, kv_scale)
+    _check(lib().csa_fused_attention(_ptr(q), _DT[q.dtype], kvp, kvd, kvr, kvs, kv.shape[1], _ptr(idx), k, m,
+                                     _ptr(kv_tok), _DT[kv_tok.dtype], kv_tok.shape[1], W, window_mode, _ptr(q_pos),
+                                     _ptr(sink), n_seq, T, H, D, rope_dim, rope_base, int(inv_rope), scale,
+                                     _ptr(out), _DT[out.dtype], _stream(stream)), "csa_fused_attention")
+    return out
+
+
 # ---------------------------------------------------------------- layers
 
 def csa_layer_prefill(q, C, Z, B, qI, w, kI, sink, *, k, m=4, W=128, norm_rope=False, inv_rope=False,
-                      rope_dim=64, rope_base=10000.0, kv_dtype=None, workspace=None, return_idx=False):
+                      rope_dim=64, rope_base=10000.0, kv_dtype=None, workspace=None, return_idx=False,
+                      fused=True):
     """One CSA layer (batch 1): compress -> index/top-k -> sparse MQA -> window + sink.
     q [S, H, D], C/Z [S, D], B [2m, D] f32, qI [S, HI, DI] u8, w [S, HI], kI [S//m, DI] u8, sink [H]."""
     S, H, D = q.shape
@@ -223,14 +252,18 @@ def csa_layer_prefill(q, C, Z, B, qI, w, kI, sink, *, k, m=4, W=128, norm_rope=F
         qn, kt = q, C
         kv = csa_compress(C, Z, B, m, True, out_dtype=kv_dtype)
     idx = csa_index_topk(qI[None], w[None], kI[None], pos, m, k, workspace=workspace)
-    Op, Lp = csa_sparse_mqa(qn[None], kv[None], idx)
-    out = swa_sink_combine(qn[None], kt[None], pos, W, sink, Op, Lp, window_mode=0, inv_rope=inv_rope,
-                           rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
+    if fused:
+        out = csa_fused_attention(qn[None], kv[None], kt[None], pos, W, sink, idx=idx, inv_rope=inv_rope,
+                                  rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
+    else:
+        Op, Lp = csa_sparse_mqa(qn[None], kv[None], idx)
+        out = swa_sink_combine(qn[None], kt[None], pos, W, sink, Op, Lp, window_mode=0, inv_rope=inv_rope,
+                               rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
     return (out[0], idx[0]) if return_idx else out[0]
 
 
 def hca_layer_prefill(q, C, Z, B, sink, *, m=128, W=128, norm_rope=False, inv_rope=False, rope_dim=64,
-                      rope_base=10000.0, kv_dtype=None):
+                      rope_base=10000.0, kv_dtype=None, fused=True):
     """One HCA layer (batch 1): compress (m' = 128) -> dense attention -> window + sink."""
     S, H, D = q.shape
     dev = q.device
@@ -243,7 +276,11 @@ def hca_layer_prefill(q, C, Z, B, sink, *, m=128, W=128, norm_rope=False, inv_ro
     else:
         qn, kt = q, C
         kv = csa_compress(C, Z, B, m, False, out_dtype=kv_dtype)
-    Op, Lp = hca_dense_attn(qn[None], kv[None], pos, m)
-    out = swa_sink_combine(qn[None], kt[None], pos, W, sink, Op, Lp, window_mode=0, inv_rope=inv_rope,
-                           rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
+    if fused:
+        out = csa_fused_attention(qn[None], kv[None], kt[None], pos, W, sink, m=m, inv_rope=inv_rope,
+                                  rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
+    else:
+        Op, Lp = hca_dense_attn(qn[None], kv[None], pos, m)
+        out = swa_sink_combine(qn[None], kt[None], pos, W, sink, Op, Lp, window_mode=0, inv_rope=inv_rope,
+                               rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
     return out[0]

@@ -57,19 +57,28 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 enum KvKind { KV_BF16 = 0, KV_F32 = 1, KV_FP8 = 2 };
 enum EpiMode { EPI_PARTIAL = 0, EPI_COMBINE = 1 };
-enum RowKind { ROWS_GATHER = 0, ROWS_DENSE = 1, ROWS_WINDOW = 2, ROWS_CACHE = 3 };
+// Row set of a query token: source 1 (compressed entries: a gathered top-k
+// list or the dense prefix of complete entries) followed by source 2 (raw
+// window rows).  Either may be absent.  All rows share one softmax.
+enum Src1Kind { SRC1_NONE = 0, SRC1_GATHER = 1, SRC1_DENSE = 2 };
+enum Src2Kind { SRC2_NONE = 0, SRC2_WINDOW = 1, SRC2_CACHE = 2 };
 
 struct AttnParams {
   const void* q;            // [n_seq, T, H, D] bf16 or f32
   int q_f32;
+  // source 1: compressed entries
   const void* kv;           // bf16/f32 [n_seq, cap, D] or e4m3 [n_seq, cap, D - rope_dim]
   const __nv_bfloat16* kv_rope;   // e4m3 store: [n_seq, cap, rope_dim]
   const float* kv_scale;          // e4m3 store: [n_seq, cap]
   int64_t cap;
+  int src1, m;
   const int32_t* idx;       // gather: [n_seq, T, k]
   int k;
-  const int64_t* q_pos;     // [n_seq]
-  int row_kind, m, W;
+  // source 2: raw window rows
+  const void* kv2;          // [n_seq, cap2, D], bf16 (f32 when source 1 is f32)
+  int64_t cap2;
+  int src2, W;
+  const int64_t* q_pos;     // [n_seq] (null: 0)
   int n_seq, T, H;
   float scale_log2;
   float* O_part;            // partial outputs
@@ -83,27 +92,48 @@ struct AttnParams {
 };
 
 struct RowSet {
-  int64_t lo;               // range modes: first KV row
-  int n;                    // rows in the set
-  const int32_t* idx;       // gather mode: row list
+  int n1, n2, n;            // rows from source 1, source 2, total
+  int64_t lo2;              // first window row
+  const int32_t* idx;       // gather list (source 1)
 };
 
-__device__ __forceinline__ RowSet row_set(const AttnParams& p, int b, int t) {
-  RowSet r{0, 0, nullptr};
-  const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
-  if (p.row_kind == ROWS_GATHER) {
-    const int32_t* row = p.idx + ((int64_t)b * p.T + t) * p.k;
-    int lo = 0, hi = p.k;                      // first -1 of an ascending, -1 padded list
-    while (lo < hi) { int mid = (lo + hi) >> 1; if (row[mid] >= 0) lo = mid + 1; else hi = mid; }
-    r.idx = row; r.n = lo;
-  } else if (p.row_kind == ROWS_DENSE) {
-    r.lo = 0; r.n = (int)min(p.cap, (pos + 1) / p.m);
-  } else if (p.row_kind == ROWS_WINDOW) {
-    int64_t lo = max((int64_t)0, pos - p.W + 1), hi = min(p.cap, pos + 1);
-    r.lo = lo; r.n = (int)max((int64_t)0, hi - lo);
-  } else {
-    r.lo = 0; r.n = (int)min(min((int64_t)p.W, p.cap), pos + 1);
+// Length of an ascending, -1 padded index list, found by one warp with two
+// dependent loads (segment ends, then the segment holding the first -1).
+__device__ __forceinline__ int count_valid_warp(const int32_t* row, int k, int lane) {
+  const int seg = (k + 31) >> 5;
+  const bool in = lane * seg < k;
+  const int v = in ? row[min(k, (lane + 1) * seg) - 1] : -1;
+  const unsigned neg = __ballot_sync(0xffffffffu, !in || v < 0);
+  const int f = __ffs(neg) - 1;
+  if (f < 0 || f * seg >= k) return k;
+  const int s0 = f * seg, s1 = min(k, s0 + seg);
+  for (int base = s0; base < s1; base += 32) {
+    const int i = base + lane;
+    const unsigned m2 = __ballot_sync(0xffffffffu, i < s1 && row[i] < 0);
+    if (m2) return base + __ffs(m2) - 1;
   }
+  return s1;
+}
+
+// Whole-warp call: every lane gets the same row set.
+__device__ __forceinline__ RowSet row_set_warp(const AttnParams& p, int b, int t, int lane) {
+  RowSet r{0, 0, 0, 0, nullptr};
+  const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
+  if (p.src1 == SRC1_GATHER) {
+    r.idx = p.idx + ((int64_t)b * p.T + t) * p.k;
+    r.n1 = count_valid_warp(r.idx, p.k, lane);
+  } else if (p.src1 == SRC1_DENSE) {
+    r.n1 = (int)min(p.cap, (pos + 1) / p.m);
+  }
+  if (p.src2 == SRC2_WINDOW) {
+    const int64_t lo = max((int64_t)0, pos - p.W + 1), hi = min(p.cap2, pos + 1);
+    r.lo2 = lo;
+    r.n2 = (int)max((int64_t)0, hi - lo);
+  } else if (p.src2 == SRC2_CACHE) {
+    r.lo2 = 0;
+    r.n2 = (int)min(min((int64_t)p.W, p.cap2), pos + 1);
+  }
+  r.n = r.n1 + r.n2;
   return r;
 }
 
@@ -201,6 +231,42 @@ __device__ __forceinline__ void load_kv_slab(const AttnParams& p, int b, int64_t
   }
 }
 
+// Source-2 (window) rows: bf16 or f32 [n_seq, cap2, D].  ASYNC selects
+// cp.async (bf16 only, caller commits) or a synchronous load + store.
+template <int D, int KV2, bool ASYNC>
+__device__ __forceinline__ void load_tok_slab(const AttnParams& p, int b, int64_t row, bool valid, int s,
+                                              uint8_t* slab_base, int r) {
+  if constexpr (KV2 == KV_BF16) {
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kv2) +
+                         ((((int64_t)b * p.cap2 + (valid ? row : 0)) * D + 64 * s) * 2);
+    if constexpr (ASYNC) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) cp_async16(slab_base + swz128(r, q), src + 16 * q, valid ? 16u : 0u);
+    } else {
+      uint4 v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = valid ? __ldg(reinterpret_cast<const uint4*>(src) + q) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) st_shared16(slab_base + swz128(r, q), v[q]);
+    }
+  } else {
+    const float* src = reinterpret_cast<const float*>(p.kv2) + ((int64_t)b * p.cap2 + (valid ? row : 0)) * D + 64 * s;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float v[8];
+      if (valid) {
+        float4 a = __ldg(reinterpret_cast<const float4*>(src + 8 * q));
+        float4 c = __ldg(reinterpret_cast<const float4*>(src + 8 * q) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      }
+      st_shared16(slab_base + swz128(r, q), to_bf16x8(v));
+    }
+  }
+}
+
 template <int D, int KV, int EPI>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
   constexpr int NS = D / 64;                 // 128-byte slabs per row
@@ -208,6 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   constexpr uint32_t kQSlab = kNQ * 128;     // 8 KB
   constexpr uint32_t kKSlab = kRows * 128;   // 16 KB
   constexpr uint32_t kTmemCols = (64 + 64 * NT) <= 128 ? 128 : ((64 + 64 * NT) <= 256 ? 256 : 512);
+  constexpr int KV2 = (KV == KV_F32) ? KV_F32 : KV_BF16;   // window rows: bf16 unless the store is fp32
+  constexpr bool kAsync = (KV == KV_BF16);                  // cp.async for every row of a bf16 store
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -252,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     bool ok = true;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const int b = (int)(item / p.T), t = (int)(item % p.T);
-      const RowSet rs = row_set(p, b, t);
+      const RowSet rs = row_set_warp(p, b, t, lane);
       if (rs.n == 0) continue;
       // ---- Q tile: 64 rows x NS slabs of 128 B
       if (!wait_bar(q_free, (qcount & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -291,22 +359,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       for (int c = 0; c < n_chunks && ok; ++c, ++g) {
         const int r = c * kRows + lt;
         bool valid = r < rs.n;
+        const bool win = r >= rs.n1;                 // source-2 (window) row
         int64_t row = 0;
         if (valid) {
-          if (rs.idx) {
+          if (win) {
+            row = rs.lo2 + (r - rs.n1);
+          } else if (rs.idx) {
             row = rs.idx[r];
             if (row < 0 || row >= p.cap) { atomicOr(&g_err_attn, DEV_ERR_BAD_INDEX); valid = false; row = 0; }
           } else {
-            row = rs.lo + r;
+            row = r;
           }
         }
         for (int tt = 0; tt < NT; ++tt) {
           if (!wait_bar(&pv_done[tt], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
-          load_kv_slab<D, KV>(p, b, row, valid, 2 * tt, sKV + (2 * tt) * kKSlab, lt);
-          if constexpr (KV == KV_BF16) asm volatile("cp.async.commit_group;" ::: "memory");
-          load_kv_slab<D, KV>(p, b, row, valid, 2 * tt + 1, sKV + (2 * tt + 1) * kKSlab, lt);
-          if constexpr (KV == KV_BF16) {
-            asm volatile("cp.async.commit_group;" ::: "memory");
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int sl = 2 * tt + h;
+            if (win) load_tok_slab<D, KV2, kAsync>(p, b, row, valid, sl, sKV + sl * kKSlab, lt);
+            else     load_kv_slab<D, KV>(p, b, row, valid, sl, sKV + sl * kKSlab, lt);
+            if constexpr (kAsync) asm volatile("cp.async.commit_group;" ::: "memory");
+          }
+          if constexpr (kAsync) {
             if (tt > 0) {
               asm volatile("cp.async.wait_group 2;" ::: "memory");
               fence_proxy_async_smem();
@@ -319,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             mbar_arrive(&kv_full[2 * tt + 1]);
           }
         }
-        if constexpr (KV == KV_BF16) {
+        if constexpr (kAsync) {
           if (ok) {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
             fence_proxy_async_smem();
@@ -331,18 +405,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 8) {
-    // ============================ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_s = make_idesc(128, kNQ, 1, 1, 0, 0);
-      const uint32_t idesc_o = make_idesc(128, kNQ, 1, 1, 1, 1);
-      const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV), aP = smem_u32(sP);
-      uint32_t g = 0, qcount = 0, icount = 0;
-      bool ok = true;
-      for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-        const int b = (int)(item / p.T), t = (int)(item % p.T);
-        const RowSet rs = row_set(p, b, t);
-        if (rs.n == 0) continue;
-        if (!wait_bar(q_full, qcount & 1, abort_flag)) { ok = false; break; }
+    // ============================ MMA issuer (lane 0; the warp computes row sets)
+    const uint32_t idesc_s = make_idesc(128, kNQ, 1, 1, 0, 0);
+    const uint32_t idesc_o = make_idesc(128, kNQ, 1, 1, 1, 1);
+    const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV), aP = smem_u32(sP);
+    uint32_t g = 0, qcount = 0, icount = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int b = (int)(item / p.T), t = (int)(item % p.T);
+      const RowSet rs = row_set_warp(p, b, t, lane);
+      if (rs.n == 0) continue;
+      if (lane == 0) {
+        if (!wait_bar(q_full, qcount & 1, abort_flag)) ok = false;
         ++qcount;
         const int n_chunks = (rs.n + kRows - 1) / kRows;
         for (int c = 0; c < n_chunks && ok; ++c, ++g) {
@@ -374,6 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
         ++icount;
       }
+      __syncwarp();
+      ok = __shfl_sync(0xffffffffu, ok, 0);
     }
   } else {
     // ============================ softmax + epilogue (warps 0-3)
@@ -384,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     bool ok = true;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const int b = (int)(item / p.T), t = (int)(item % p.T);
-      const RowSet rs = row_set(p, b, t);
+      const RowSet rs = row_set_warp(p, b, t, lane);
       const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
       float2* cs = s_cs + (icount & 1) * 32;
       if (EPI == EPI_COMBINE && p.inv_rope && tid < 32) {
@@ -533,59 +609,70 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
       const int64_t obase = ((int64_t)b * p.T + t) * p.H;
       for (int tt = 0; tt < NT; ++tt) {
-        float o[64];
-        if (rs.n > 0) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_ld16(tmem + lane_base + 64 + 64 * tt + 16 * q, o + 16 * q);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) o[i] = 0.f;
-        }
         const int d = tt * 128 + e;
-        if (EPI == EPI_PARTIAL) {
+        const bool rope_tile = EPI == EPI_COMBINE && p.inv_rope && tt == NT - 1;
+        // 32 query rows at a time keeps the live set small
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          float o[32];
+          if (rs.n > 0) {
+            tmem_ld16(tmem + lane_base + 64 + 64 * tt + 32 * hh, o);
+            tmem_ld16(tmem + lane_base + 64 + 64 * tt + 32 * hh + 16, o + 16);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < p.H) p.O_part[(obase + c) * D + d] = o[c] * bc_m[64 + c];
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            float v = o[c] * bc_m[64 + c];
-            if (p.O_in && c < p.H) v = fmaf(bc_m[128 + c], p.O_in[(obase + c) * D + d], v);
-            o[c] = v;
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
           }
-          const int r0 = D - p.rope_dim;
-          if (p.inv_rope && tt == NT - 1) {
-            // pairs (d, d + 32) of the last 64 dims sit in warps 2 and 3: swap through sP
-            float* ex = reinterpret_cast<float*>(sP);
-            named_bar_sync(2, 128);
-            if (d >= r0) {
+          if (EPI == EPI_PARTIAL) {
 #pragma unroll
-              for (int c = 0; c < 64; ++c) ex[c * 64 + (d - r0)] = o[c];
+            for (int i = 0; i < 32; ++i) {
+              const int c = 32 * hh + i;
+              if (c < p.H) p.O_part[(obase + c) * D + d] = o[i] * bc_m[64 + c];
             }
-            named_bar_sync(2, 128);
-            if (d >= r0) {
-              const int jj = d - r0, half = p.rope_dim / 2;
-              const int j = jj % half;
-              const float2 csj = cs[j];
+          } else {
 #pragma unroll
-              for (int c = 0; c < 64; ++c) {
-                // inverse rotation by -pos: (a, b) -> (a cos + b sin, -a sin + b cos)
-                if (jj < half) o[c] = o[c] * csj.x + ex[c * 64 + jj + half] * csj.y;
-                else           o[c] = o[c] * csj.x - ex[c * 64 + jj - half] * csj.y;
+            for (int i = 0; i < 32; ++i) {
+              const int c = 32 * hh + i;
+              float v = o[i] * bc_m[64 + c];
+              if (p.O_in && c < p.H) v = fmaf(bc_m[128 + c], p.O_in[(obase + c) * D + d], v);
+              o[i] = v;
+            }
+            const int r0 = D - p.rope_dim;
+            if (rope_tile) {
+              // pairs (d, d + 32) of the last 64 dims sit in warps 2 and 3: swap through sP
+              float* ex = reinterpret_cast<float*>(sP);
+              named_bar_sync(2, 128);
+              if (d >= r0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ex[i * 64 + (d - r0)] = o[i];
+              }
+              named_bar_sync(2, 128);
+              if (d >= r0) {
+                const int jj = d - r0, half = p.rope_dim / 2;
+                const float2 csj = cs[jj % half];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  // inverse rotation by -pos: (a, b) -> (a cos + b sin, -a sin + b cos)
+                  if (jj < half) o[i] = o[i] * csj.x + ex[i * 64 + jj + half] * csj.y;
+                  else           o[i] = o[i] * csj.x - ex[i * 64 + jj - half] * csj.y;
+                }
               }
             }
-          }
-          if (p.out_bf16) {
-            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+            if (p.out_bf16) {
+              __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (c < p.H) out[(obase + c) * D + d] = __float2bfloat16_rn(o[c]);
-          } else {
-            float* out = reinterpret_cast<float*>(p.out);
+              for (int i = 0; i < 32; ++i) {
+                const int c = 32 * hh + i;
+                if (c < p.H) out[(obase + c) * D + d] = __float2bfloat16_rn(o[i]);
+              }
+            } else {
+              float* out = reinterpret_cast<float*>(p.out);
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (c < p.H) out[(obase + c) * D + d] = o[c];
+              for (int i = 0; i < 32; ++i) {
+                const int c = 32 * hh + i;
+                if (c < p.H) out[(obase + c) * D + d] = o[i];
+              }
+            }
           }
         }
       }
@@ -669,7 +756,7 @@ extern "C" csa_status_t csa_sparse_mqa(const void* q, csa_dtype_t q_dtype, const
   CSA_REQUIRE(O_part && lse_part && aligned16(O_part), "csa_sparse_mqa: O_part / lse_part must be non-null");
   AttnParams p{};
   p.q = q; p.q_f32 = q_dtype == CSA_F32; p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale;
-  p.cap = cap; p.idx = idx; p.k = k; p.q_pos = nullptr; p.row_kind = ROWS_GATHER; p.m = 1; p.W = 0;
+  p.cap = cap; p.src1 = SRC1_GATHER; p.idx = idx; p.k = k; p.m = 1; p.src2 = SRC2_NONE;
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = O_part; p.lse_part = lse_part; p.rope_dim = rope_dim;
   return dispatch<EPI_PARTIAL>(p, D, kv_dtype, stream);
@@ -687,7 +774,7 @@ extern "C" csa_status_t hca_dense_attn(const void* q, csa_dtype_t q_dtype, const
   CSA_REQUIRE(O_part && lse_part && aligned16(O_part), "hca_dense_attn: O_part / lse_part must be non-null");
   AttnParams p{};
   p.q = q; p.q_f32 = q_dtype == CSA_F32; p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale;
-  p.cap = cap; p.q_pos = q_pos; p.row_kind = ROWS_DENSE; p.m = m; p.W = 0;
+  p.cap = cap; p.q_pos = q_pos; p.src1 = SRC1_DENSE; p.m = m; p.src2 = SRC2_NONE;
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = O_part; p.lse_part = lse_part; p.rope_dim = rope_dim;
   return dispatch<EPI_PARTIAL>(p, D, kv_dtype, stream);
@@ -710,10 +797,40 @@ extern "C" csa_status_t swa_sink_combine(const void* q, csa_dtype_t q_dtype, con
   CSA_REQUIRE(!O_part || aligned16(O_part), "swa_sink_combine: O_part must be 16-byte aligned");
   CSA_REQUIRE(out && aligned16(out) && (out_dtype == CSA_F32 || out_dtype == CSA_BF16), "swa_sink_combine: bad out");
   AttnParams p{};
-  p.q = q; p.q_f32 = q_dtype == CSA_F32; p.kv = kv_tok; p.cap = cap; p.q_pos = q_pos;
-  p.row_kind = window_mode == 0 ? ROWS_WINDOW : ROWS_CACHE; p.m = 1; p.W = W;
+  p.q = q; p.q_f32 = q_dtype == CSA_F32; p.q_pos = q_pos;
+  p.kv = kv_tok; p.cap = cap; p.src1 = SRC1_NONE; p.m = 1;
+  p.kv2 = kv_tok; p.cap2 = cap; p.src2 = window_mode == 0 ? SRC2_WINDOW : SRC2_CACHE; p.W = W;
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_in = O_part; p.lse_in = lse_part; p.sink = sink; p.out = out; p.out_bf16 = out_dtype == CSA_BF16;
+  p.inv_rope = inv_rope; p.rope_dim = rope_dim; p.rope_base = rope_base;
+  return dispatch<EPI_COMBINE>(p, D, kv_dtype, stream);
+}
+
+extern "C" csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, const void* kv, csa_dtype_t kv_dtype,
+                                            const void* kv_rope, const float* kv_scale, int64_t cap,
+                                            const int32_t* idx, int k, int m, const void* kv_tok,
+                                            csa_dtype_t tok_dtype, int64_t tok_cap, int W, int window_mode,
+                                            const int64_t* q_pos, const float* sink, int n_seq, int T, int H,
+                                            int D, int rope_dim, float rope_base, int inv_rope, float scale,
+                                            void* out, csa_dtype_t out_dtype, cudaStream_t stream) {
+  clear_error();
+  csa_status_t s = check_common("csa_fused_attention", q, q_dtype, kv, kv_dtype, kv_rope, kv_scale, cap, n_seq, T, H, D, rope_dim);
+  if (s != CSA_OK) return s;
+  CSA_REQUIRE(q_pos && aligned16(q_pos), "csa_fused_attention: q_pos required");
+  CSA_REQUIRE(idx ? (k >= 1 && aligned16(idx)) : m >= 1, "csa_fused_attention: need idx with k >= 1, or m >= 1 for dense rows");
+  CSA_REQUIRE(kv_tok && aligned16(kv_tok) && tok_cap >= 1 && W >= 1, "csa_fused_attention: kv_tok, tok_cap >= 1 and W >= 1 required");
+  CSA_REQUIRE(tok_dtype == (kv_dtype == CSA_F32 ? CSA_F32 : CSA_BF16),
+              "csa_fused_attention: window rows must be f32 with an f32 store and bf16 otherwise");
+  CSA_REQUIRE(window_mode == 0 || window_mode == 1, "csa_fused_attention: window_mode must be 0 or 1");
+  CSA_REQUIRE(!inv_rope || rope_dim == 64, "csa_fused_attention: inv_rope needs rope_dim 64");
+  CSA_REQUIRE(out && aligned16(out) && (out_dtype == CSA_F32 || out_dtype == CSA_BF16), "csa_fused_attention: bad out");
+  AttnParams p{};
+  p.q = q; p.q_f32 = q_dtype == CSA_F32; p.q_pos = q_pos;
+  p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale; p.cap = cap;
+  p.src1 = idx ? SRC1_GATHER : SRC1_DENSE; p.idx = idx; p.k = k; p.m = m;
+  p.kv2 = kv_tok; p.cap2 = tok_cap; p.src2 = window_mode == 0 ? SRC2_WINDOW : SRC2_CACHE; p.W = W;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.sink = sink; p.out = out; p.out_bf16 = out_dtype == CSA_BF16;
   p.inv_rope = inv_rope; p.rope_dim = rope_dim; p.rope_base = rope_base;
   return dispatch<EPI_COMBINE>(p, D, kv_dtype, stream);
 }

@@ -143,3 +143,78 @@ def test_batch_invariance_bit_exact():
         Oa, La = csa.csa_sparse_mqa(tq[b:b + 1].contiguous(), tkv[b:b + 1].contiguous(), ti[b:b + 1].contiguous())
         assert torch.equal(Oa[0], Ob[b]) and torch.equal(La[0], Lb[b])
     csa.check_device_error()
+
+
+def _dequant(cache):
+    return np.concatenate([O.e4m3_decode(cache["kv_nope"].cpu().numpy()) * cache["kv_scale"].cpu().numpy()[:, None],
+                           cache["kv_rope"].float().cpu().numpy()], axis=1)
+
+
+def test_fused_csa_decode_e4m3_caches():
+    """Decode: top-k entries from an e4m3 + bf16-RoPE cache, the 128-row SWA
+    cache and the sink in one softmax, inverse RoPE at the query position."""
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(21)
+    gen = torch.Generator(device="cuda").manual_seed(21)
+    n_seq, cap, H, D, W, k = 4, 2500, 64, 512, 128, 512
+    caches = [synth.decode_csa_cache(cap, D, 128, 64, gen, "cuda") for _ in range(n_seq)]
+    kv_nope = torch.stack([c["kv_nope"] for c in caches]); kv_rope = torch.stack([c["kv_rope"] for c in caches])
+    kv_scale = torch.stack([c["kv_scale"] for c in caches])
+    q = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((n_seq, 1, H, D))))
+    swa = synth.to_bf16_values(rng.standard_normal((n_seq, W, D)))
+    sink = rng.standard_normal(H).astype(np.float32)
+    pos = np.array([4 * cap - 1, 3, 999, 4 * cap - 5], np.int64)
+    idx = np.full((n_seq, 1, k), -1, np.int32)
+    for b in range(n_seq):
+        nv = min(cap, (pos[b] + 1) // 4)
+        n = min(k, nv)
+        idx[b, 0, :n] = np.sort(rng.choice(nv, n, replace=False)) if nv else []
+    out = csa.csa_fused_attention(cuda(q, torch.bfloat16), kv_nope, cuda(swa, torch.bfloat16), cuda(pos), W,
+                                  cuda(sink), idx=cuda(idx), kv_rope=kv_rope, kv_scale=kv_scale, window_mode=1,
+                                  inv_rope=True, rope_dim=64, out_dtype=torch.float32)
+    csa.check_device_error()
+    for b in range(n_seq):
+        kv = _dequant(caches[b])
+        Op, Lp = O.sparse_attention_partial(q[b], kv, idx[b])
+        nrow = min(W, pos[b] + 1)
+        ref = O.window_sink_combine(q[b], None, [pos[b]], W, sink, Op, Lp, inv_rope=True, window_rows=[swa[b][:nrow]])
+        assert_close(host(out)[b], ref, what=f"fused CSA decode b={b}")
+
+
+def test_fused_hca_decode_e4m3_dense():
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(22)
+    gen = torch.Generator(device="cuda").manual_seed(22)
+    n_seq, cap, H, D, W, m = 3, 700, 64, 512, 128, 128
+    caches = [synth.decode_csa_cache(cap, D, 128, 64, gen, "cuda") for _ in range(n_seq)]
+    kv_nope = torch.stack([c["kv_nope"] for c in caches]); kv_rope = torch.stack([c["kv_rope"] for c in caches])
+    kv_scale = torch.stack([c["kv_scale"] for c in caches])
+    q = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((n_seq, 1, H, D))))
+    swa = synth.to_bf16_values(rng.standard_normal((n_seq, W, D)))
+    sink = rng.standard_normal(H).astype(np.float32)
+    pos = np.array([128 * 700 - 1, 130, 128 * 333 + 17], np.int64)
+    out = csa.csa_fused_attention(cuda(q, torch.bfloat16), kv_nope, cuda(swa, torch.bfloat16), cuda(pos), W,
+                                  cuda(sink), m=m, kv_rope=kv_rope, kv_scale=kv_scale, window_mode=1,
+                                  inv_rope=True, rope_dim=64, out_dtype=torch.float32)
+    csa.check_device_error()
+    for b in range(n_seq):
+        kv = _dequant(caches[b])
+        ref = O.hca_decode(q[b][0], kv, swa[b][:min(W, pos[b] + 1)], sink, int(pos[b]), m=m)
+        assert_close(host(out)[b][0], ref, what=f"fused HCA decode b={b}")
+
+
+def test_fused_equals_separate_calls():
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(23)
+    S, ne, H, D, k, W = 400, 100, 64, 512, 64, 128
+    q = cuda(synth.to_bf16_values(O.rmsnorm(rng.standard_normal((1, S, H, D)))), torch.bfloat16)
+    kv = cuda(synth.to_bf16_values(O.rmsnorm(rng.standard_normal((1, ne, D)))), torch.bfloat16)
+    kt = cuda(synth.to_bf16_values(O.rmsnorm(rng.standard_normal((1, S, D)))), torch.bfloat16)
+    idx = cuda(np.stack([_rand_idx(rng, S, k, ne, [64, 0, 5, 33])]))
+    sink = cuda(rng.standard_normal(H).astype(np.float32))
+    pos = cuda(np.array([0], np.int64))
+    Op, Lp = csa.csa_sparse_mqa(q, kv, idx)
+    sep = csa.swa_sink_combine(q, kt, pos, W, sink, Op, Lp, inv_rope=True, out_dtype=torch.float32)
+    fus = csa.csa_fused_attention(q, kv, kt, pos, W, sink, idx=idx, inv_rope=True, out_dtype=torch.float32)
+    csa.check_device_error()
+    assert_close(host(fus), host(sep), max_abs=5e-3, rel_l2=1e-3, what="fused vs separate")

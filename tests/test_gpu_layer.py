@@ -17,12 +17,12 @@ def _lib():
     lib_loaded()
 
 
-def _gpu_csa(inp, cfg, dt):
+def _gpu_csa(inp, cfg, dt, fused=True):
     import long_context_compressed_02_b200 as csa
     out, idx = csa.csa_layer_prefill(
         cuda(inp["q"], dt), cuda(inp["C"], dt), cuda(inp["Z"], dt), cuda(inp["B"]), cuda(inp["qI_codes"]),
         cuda(inp["w"]), cuda(inp["kI_codes"]), cuda(inp["sink"]), k=cfg["k"], m=cfg["m"], W=cfg["W"],
-        norm_rope=cfg["norm_rope"], inv_rope=cfg["inv_rope"], return_idx=True)
+        norm_rope=cfg["norm_rope"], inv_rope=cfg["inv_rope"], return_idx=True, fused=fused)
     csa.check_device_error()
     return out, idx
 
@@ -33,18 +33,19 @@ def _oracle_csa(inp, cfg, rows=None, store=None):
                        norm_rope=cfg["norm_rope"], inv_rope=cfg["inv_rope"], store_round=store, rows=rows)
 
 
-def test_tiny_csa_layer():
+@pytest.mark.parametrize("fused", [True, False])
+def test_tiny_csa_layer(fused):
     inp, cfg = synth.prefill_inputs("tiny_csa")
-    out, idx = _gpu_csa(inp, cfg, torch.float32)
+    out, idx = _gpu_csa(inp, cfg, torch.float32, fused)
     ref, ridx = _oracle_csa(inp, cfg)
     assert np.array_equal(idx.cpu().numpy(), ridx)
     assert_close(host(out), ref, what="tiny CSA layer")
 
 
-@pytest.mark.parametrize("S", [1534, 2048])
-def test_flash_shaped_csa_layer(S):
+@pytest.mark.parametrize("S,fused", [(1534, True), (2048, True), (2048, False)])
+def test_flash_shaped_csa_layer(S, fused):
     inp, cfg = synth.prefill_inputs("csa_prefill", S=S, grid=True)
-    out, idx = _gpu_csa(inp, cfg, torch.bfloat16)
+    out, idx = _gpu_csa(inp, cfg, torch.bfloat16, fused)
     ref, ridx = _oracle_csa(inp, cfg, store=O.bf16_round)
     assert np.array_equal(idx.cpu().numpy(), ridx)
     assert_close(host(out), ref, what="Flash-shaped CSA layer")
@@ -65,13 +66,13 @@ def test_csa_layer_causality_bit_exact():
     assert not torch.equal(out[t + 1:], base[t + 1:])
 
 
-@pytest.mark.parametrize("S", [128 * 6 + 37, 129])
-def test_hca_layer(S):
+@pytest.mark.parametrize("S,fused", [(128 * 6 + 37, True), (129, True), (128 * 6 + 37, False)])
+def test_hca_layer(S, fused):
     import long_context_compressed_02_b200 as csa
     inp, cfg = synth.prefill_inputs("hca_prefill", S=S)
     out = csa.hca_layer_prefill(cuda(inp["q"], torch.bfloat16), cuda(inp["C"], torch.bfloat16),
                                 cuda(inp["Z"], torch.bfloat16), cuda(inp["B"]), cuda(inp["sink"]),
-                                m=128, W=128, norm_rope=True, inv_rope=True)
+                                m=128, W=128, norm_rope=True, inv_rope=True, fused=fused)
     csa.check_device_error()
     ref = O.hca_layer(inp["q"], inp["C"], inp["Z"], inp["B"], inp["sink"], m=128, W=128, norm_rope=True,
                       inv_rope=True, store_round=O.bf16_round)
