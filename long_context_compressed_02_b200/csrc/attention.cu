@@ -687,6 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       named_bar_sync(1, 128);   // s_red / bc reuse across items
     }
   }
+  __syncwarp();                 // reconverge role warps before the CTA barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {

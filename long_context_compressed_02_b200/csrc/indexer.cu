@@ -73,7 +73,8 @@ bool make_byte_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t r
 }
 
 // ------------------------------------------------------------------ scores
-constexpr int kIdxThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kIdxThreads = 320;      // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kEpiThreads = 256;
 constexpr int kStages = 8;
 
 struct IdxParams {
@@ -100,6 +101,12 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   *abort_flag = 1;
   atomicOr(&g_err_idx, DEV_ERR_TIMEOUT_MBAR);
   return false;
+}
+
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
 }
 
 __global__ void __launch_bounds__(kIdxThreads, 1)
@@ -130,12 +137,14 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   uint64_t* qbar = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(qbar + 1);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
-  float* s_w = reinterpret_cast<float*>(s_abort + 1);   // [N] = w * qs per column
+  int* s_nv = s_abort + 1;                                    // [TQ] visible entries per token
+  float* s_w = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(s_nv + p.TQ) + 15) & ~uintptr_t(15));   // [N] = w * qs per column
 
   const uint32_t tmem_cols = p.N <= 16 ? 32u : (p.N <= 32 ? 64u : (p.N <= 64 ? 128u : (p.N <= 128 ? 256u : 512u)));
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 128); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiThreads); }
     mbar_init(qbar, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -150,6 +159,10 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     }
     s_w[c] = v;
   }
+  for (int tq = tid; tq < p.TQ; tq += kIdxThreads) {
+    const int t = t0 + tq;
+    s_nv[tq] = t < p.T ? (int)min(p.cap, (pos0 + t + 1) / p.m) : 0;
+  }
   if (warp == 1) tmem_alloc(s_tmem, tmem_cols);
   tc_fence_before();
   __syncthreads();
@@ -160,68 +173,103 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   const uint32_t swz = p.DI == 128 ? SWZ_128B : (p.DI == 64 ? SWZ_64B : SWZ_32B);
   const uint32_t sbo = 8u * p.DI;
 
-  if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    tma_prefetch_desc(&tmap_k);
-    tma_prefetch_desc(&tmap_q);
-    mbar_expect_tx(qbar, b_bytes);
-    tma_load_2d(sB, &tmap_q, 0, (int32_t)(((int64_t)b * p.T + t0) * p.HI), qbar);
-    for (int it = 0; it < n_tiles; ++it) {
-      const int s = it % kStages;
-      const uint32_t ph = (it / kStages) & 1;
-      if (!wait_bar(&empty[s], ph ^ 1, abort_flag)) break;
-      mbar_expect_tx(&full[s], a_bytes);
-      tma_load_2d(sA + s * a_bytes, &tmap_k, 0, (int32_t)((int64_t)b * p.cap + (int64_t)(tile0 + it) * 128), &full[s]);
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    const uint32_t idesc = make_idesc(128, p.N, 0, 0, 0, 0);
-    const uint32_t sB_addr = smem_u32(sB), sA_addr = smem_u32(sA);
-    if (wait_bar(qbar, 0, abort_flag)) {
+  if (warp == 0) {
+    // ---------------- TMA producer (lane 0)
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_q);
+      mbar_expect_tx(qbar, b_bytes);
+      tma_load_2d(sB, &tmap_q, 0, (int32_t)(((int64_t)b * p.T + t0) * p.HI), qbar);
       for (int it = 0; it < n_tiles; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
-        const int acc = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
-        if (!wait_bar(&full[s], ph, abort_flag)) break;
-        if (!wait_bar(&tempty[acc], aph ^ 1, abort_flag)) break;
-        tc_fence_after();
-        for (int kk = 0; kk < p.DI / 32; ++kk) {
-          uint64_t ad = smem_desc(sA_addr + s * a_bytes + kk * 32, 16, sbo, swz);
-          uint64_t bd = smem_desc(sB_addr + kk * 32, 16, sbo, swz);
-          mma_f8(tmem + acc * p.N, ad, bd, idesc, kk > 0);
-        }
-        mma_commit(&empty[s]);
-        mma_commit(&tfull[acc]);
+        if (!wait_bar(&empty[s], ph ^ 1, abort_flag)) break;
+        mbar_expect_tx(&full[s], a_bytes);
+        tma_load_2d(sA + s * a_bytes, &tmap_k, 0, (int32_t)((int64_t)b * p.cap + (int64_t)(tile0 + it) * 128), &full[s]);
       }
     }
-  } else if (warp >= 2) {
-    // ---------------- epilogue: 128 threads, one key (TMEM lane) each
-    const int sp = warp & 3;                       // TMEM sub-partition of this warp
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (lane 0)
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(128, p.N, 0, 0, 0, 0);
+      const uint32_t sB_addr = smem_u32(sB), sA_addr = smem_u32(sA);
+      if (wait_bar(qbar, 0, abort_flag)) {
+        for (int it = 0; it < n_tiles; ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          const int acc = it & 1;
+          const uint32_t aph = (it >> 1) & 1;
+          if (!wait_bar(&full[s], ph, abort_flag)) break;
+          if (!wait_bar(&tempty[acc], aph ^ 1, abort_flag)) break;
+          tc_fence_after();
+          for (int kk = 0; kk < p.DI / 32; ++kk) {
+            uint64_t ad = smem_desc(sA_addr + s * a_bytes + kk * 32, 16, sbo, swz);
+            uint64_t bd = smem_desc(sB_addr + kk * 32, 16, sbo, swz);
+            mma_f8(tmem + acc * p.N, ad, bd, idesc, kk > 0);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&tfull[acc]);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: 8 warps, two per TMEM sub-partition; each
+    // thread owns one key (TMEM lane) and half of the token columns (all of
+    // them when the block holds a single token).
+    const int ew = warp - 2;
+    const int sp = warp & 3;
+    const int half = ew >> 2;
+    const bool split = p.TQ >= 2 && p.N >= 64;
+    const int c_begin = split ? half * (p.N >> 1) : 0;
+    const int c_end = split ? c_begin + (p.N >> 1) : (half == 0 ? p.N : 0);
+    const int log2hi = __ffs(p.HI) - 1;
+    const uint32_t w_addr = smem_u32(s_w);
     const int key_in_tile = sp * 32 + lane;
     for (int it = 0; it < n_tiles; ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
-      if (!wait_bar(&tfull[acc], aph, abort_flag)) break;
-      tc_fence_after();
       const int64_t key = (int64_t)(tile0 + it) * 128 + key_in_tile;
       const float ksc = (key < p.cap) ? (p.ks ? p.ks[(int64_t)b * p.cap + key] : 1.f) : 0.f;
+      if (!wait_bar(&tfull[acc], aph, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N;
       float run = 0.f;
-      for (int cc = 0; cc < p.N; cc += 16) {
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N + cc, v);
+      for (int cc = c_begin; cc < c_end; cc += 32) {
+        float v[32];
+        tmem_ld32(tb + cc, v);
         tmem_wait_ld();
+        float pr[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = cc + i;
-          run = fmaf(s_w[col], fmaxf(v[i], 0.f), run);
-          if (((col + 1) & (p.HI - 1)) == 0) {
-            const int t = t0 + col / p.HI;
-            if (t < p.T) {
-              const int64_t nv = min(p.cap, (pos0 + t + 1) / p.m);
-              if (key < nv) p.scores[((int64_t)b * p.T + t) * p.cap + key] = run * ksc;
-            }
+        for (int i = 0; i < 8; ++i) {
+          const float4 w4 = ld_shared_f4(w_addr + (cc + 4 * i) * 4);
+          pr[4 * i + 0] = w4.x * fmaxf(v[4 * i + 0], 0.f);
+          pr[4 * i + 1] = w4.y * fmaxf(v[4 * i + 1], 0.f);
+          pr[4 * i + 2] = w4.z * fmaxf(v[4 * i + 2], 0.f);
+          pr[4 * i + 3] = w4.w * fmaxf(v[4 * i + 3], 0.f);
+        }
+        // pairwise sums inside each group of min(HI, 32) head columns
+#pragma unroll
+        for (int lv = 0; lv < 5; ++lv) {
+          const int w = 1 << lv;
+          if (w < p.HI) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2 * w) pr[i] += pr[i + w];
+          }
+        }
+        if (p.HI >= 32) {
+          run += pr[0];
+          if (((cc + 32) & (p.HI - 1)) == 0) {
+            const int tq = (cc + 31) >> log2hi;
+            if (key < s_nv[tq]) p.scores[((int64_t)b * p.T + t0 + tq) * p.cap + key] = run * ksc;
             run = 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if ((j & (p.HI - 1)) == 0) {
+              const int tq = (cc + j) >> log2hi;
+              if (key < s_nv[tq]) p.scores[((int64_t)b * p.T + t0 + tq) * p.cap + key] = pr[j] * ksc;
+            }
           }
         }
       }
@@ -229,6 +277,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       mbar_arrive(&tempty[acc]);
     }
   }
+  __syncwarp();                 // reconverge role warps before the CTA barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -470,11 +519,11 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
                 kChunk, (long long)L.n_chunks * k, kMergeCap);
   CSA_REQUIRE(L.n_chunks <= 64, "csa_index_topk: cap too large");
 
-  // token block: N = TQ * HI columns, a multiple of 16 and at most 256
+  // token block: N = TQ * HI columns, a multiple of 32 and at most 256
   int TQ = 256 / HI;
-  while (TQ > 1 && (TQ / 2) * HI >= 16 && TQ / 2 >= T) TQ /= 2;
+  while (TQ > 1 && (TQ / 2) * HI >= 32 && TQ / 2 >= T) TQ /= 2;
   const int N = TQ * HI;
-  if (N % 16 != 0) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: HI=%d gives no valid MMA width", HI);
+  if (N % 32 != 0) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: HI=%d gives no valid MMA width", HI);
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   IdxParams ip{};
@@ -498,7 +547,7 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
     return fail(CSA_ERR_CUDA, "csa_index_topk: cuTensorMapEncodeTiled failed");
 
   const size_t smem = 1024 + ((N * DI + 1023) / 1024) * 1024 + (size_t)kStages * 128 * DI +
-                      (2 * kStages + 5) * 8 + 16 + N * 4;
+                      (2 * kStages + 5) * 8 + 8 + TQ * 4 + 16 + N * 4;
   cudaFuncSetAttribute(indexer_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((unsigned)n_kchunks, (unsigned)n_qblocks, (unsigned)n_seq);
   indexer_scores_kernel<<<grid, kIdxThreads, smem, stream>>>(mk, mq, ip);
