@@ -30,11 +30,13 @@
 // swizzle) and a slab pair is refilled as soon as the PV MMA of its 128-column
 // tile retires, so loads overlap the tail of the previous chunk's MMAs.
 #include <algorithm>
+#include <cstring>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <math_constants.h>
 #include "common.cuh"
 #include "tc.cuh"
+#include "tmap.cuh"
 
 namespace csa {
 
@@ -89,10 +91,15 @@ struct AttnParams {
   void* out;
   int out_bf16, inv_rope, rope_dim;
   float rope_base;
+  int tma_q, tma_kv, tma_tok;   // TMA tile loads for bf16 queries / dense entries / window rows
 };
 
+// Chunk order: the window rows (source 2) come first, so that they start on a
+// 128-row chunk boundary and load as one TMA box per slab; the compressed
+// rows (source 1) follow from the next chunk boundary.
 struct RowSet {
   int n1, n2, n;            // rows from source 1, source 2, total
+  int nc2, nchunks;         // window chunks, all chunks
   int64_t lo2;              // first window row
   const int32_t* idx;       // gather list (source 1)
 };
@@ -117,7 +124,7 @@ __device__ __forceinline__ int count_valid_warp(const int32_t* row, int k, int l
 
 // Whole-warp call: every lane gets the same row set.
 __device__ __forceinline__ RowSet row_set_warp(const AttnParams& p, int b, int t, int lane) {
-  RowSet r{0, 0, 0, 0, nullptr};
+  RowSet r{0, 0, 0, 0, 0, 0, nullptr};
   const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
   if (p.src1 == SRC1_GATHER) {
     r.idx = p.idx + ((int64_t)b * p.T + t) * p.k;
@@ -134,14 +141,19 @@ __device__ __forceinline__ RowSet row_set_warp(const AttnParams& p, int b, int t
     r.n2 = (int)min(min((int64_t)p.W, p.cap2), pos + 1);
   }
   r.n = r.n1 + r.n2;
+  r.nc2 = (r.n2 + kRows - 1) / kRows;
+  r.nchunks = r.nc2 + (r.n1 + kRows - 1) / kRows;
   return r;
 }
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  // a few tight polls, then back off with nanosleep so that waiting warps do not
+  // flood the shared-memory pipe that the loads and stores of other warps use
   uint64_t start = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0) {
+    if (i > 8) __nanosleep(i < 64 ? 32 : 128);
+    if ((i & 63u) == 0) {
       if (*abort_flag) return false;
       const uint64_t now = global_ns();
       if (start == 0) start = now;
@@ -153,6 +165,14 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return false;
 }
 
+// 2^x on the SFU (flush-to-zero: results below 2^-126 become 0, which only
+// drops probabilities that cannot affect an fp32 softmax sum).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -161,6 +181,20 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // 8 consecutive values -> one 16-byte chunk of bf16
 __device__ __forceinline__ uint4 to_bf16x8(const float* v) {
   return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+}
+
+// cp.async.wait_group needs an immediate: dispatch the (unrolled) count.
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+  }
 }
 
 __device__ __forceinline__ void st_shared16(uint8_t* dst, uint4 v) {
@@ -267,8 +301,30 @@ __device__ __forceinline__ void load_tok_slab(const AttnParams& p, int b, int64_
   }
 }
 
+// BF16 stores, cp.async: one 128-byte slab of 32 chunk rows per loader warp.
+// Lane l moves 16 bytes of row 4j + l/8 (j = 0..7), so each warp instruction
+// reads 4 whole 128-byte row segments (full L2 sectors) instead of 32 scattered
+// 16-byte pieces.  row / valid / win are the caller's own chunk row (lane).
+template <int D>
+__device__ __forceinline__ void gather_slab_bf16(const AttnParams& p, int b, int64_t row, bool valid, bool win,
+                                                 int sl, uint8_t* slab_base, int warp_row0, int lane) {
+  const int q = lane & 7;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int rl = 4 * j + (lane >> 3);
+    const int64_t rr = __shfl_sync(0xffffffffu, row, rl);
+    const bool rv = __shfl_sync(0xffffffffu, valid, rl);
+    const bool rw = __shfl_sync(0xffffffffu, win, rl);
+    const uint8_t* base = rw ? reinterpret_cast<const uint8_t*>(p.kv2) + ((int64_t)b * p.cap2 + (rv ? rr : 0)) * D * 2
+                             : reinterpret_cast<const uint8_t*>(p.kv) + ((int64_t)b * p.cap + (rv ? rr : 0)) * D * 2;
+    cp_async16(slab_base + swz128(warp_row0 + rl, q), base + 128 * sl + 16 * q, rv ? 16u : 0u);
+  }
+}
+
 template <int D, int KV, int EPI>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(kThreads, 1)
+attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap map_q,
+            const __grid_constant__ CUtensorMap map_kv, const __grid_constant__ CUtensorMap map_tok) {
   constexpr int NS = D / 64;                 // 128-byte slabs per row
   constexpr int NT = D / 128;                // O^T tiles
   constexpr uint32_t kQSlab = kNQ * 128;     // 8 KB
@@ -278,7 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   constexpr bool kAsync = (KV == KV_BF16);                  // cp.async for every row of a bf16 store
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by offsetting the shared array itself, so accesses stay in the shared window
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + NS * kQSlab;
   uint8_t* sP = sKV + NS * kKSlab;
@@ -325,12 +382,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       // ---- Q tile: 64 rows x NS slabs of 128 B
       if (!wait_bar(q_free, (qcount & 1) ^ 1, abort_flag)) { ok = false; break; }
       ++qcount;
-      for (int u = lt; u < kNQ * NS; u += 128) {
-        const int r = u % kNQ, s = u / kNQ;
-        uint8_t* dst = sQ + s * kQSlab;
-        const bool v = r < p.H;
-        const int64_t qrow = ((int64_t)b * p.T + t) * p.H + (v ? r : 0);
-        if (p.q_f32) {
+      if (p.tma_q) {
+        // 64 query rows (the token's heads; rows past H belong to the next token or
+        // are zero-filled, and their columns are never written out)
+        if (lt == 0) {
+          mbar_expect_tx(q_full, kNQ * D * 2);
+#pragma unroll 1
+          for (int s = 0; s < NS; ++s)
+            tma_load_2d(sQ + s * kQSlab, &map_q, 64 * s, (int32_t)(((int64_t)b * p.T + t) * p.H), q_full);
+        }
+      } else if (p.q_f32) {
+        for (int u = lt; u < kNQ * NS; u += 128) {
+          const int r = u % kNQ, s = u / kNQ;
+          uint8_t* dst = sQ + s * kQSlab;
+          const bool v = r < p.H;
+          const int64_t qrow = ((int64_t)b * p.T + t) * p.H + (v ? r : 0);
           const float* src = reinterpret_cast<const float*>(p.q) + qrow * D + 64 * s;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -345,25 +411,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             }
             st_shared16(dst + swz128(r, q), to_bf16x8(x));
           }
-        } else {
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(p.q) + (qrow * D + 64 * s) * 2;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) cp_async16(dst + swz128(r, q), src + 16 * q, v ? 16u : 0u);
+        }
+      } else {
+        // consecutive lanes take consecutive 16-byte pieces of one query row
+        constexpr int kPieces = D / 8;                       // 16-byte pieces per row
+        const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q) + ((int64_t)b * p.T + t) * p.H * D * 2;
+        for (int u = lt; u < kNQ * kPieces; u += 128) {
+          const int r = u / kPieces, c = u % kPieces;
+          const bool v = r < p.H;
+          cp_async16(sQ + (c >> 3) * kQSlab + swz128(r, c & 7), qb + ((int64_t)(v ? r : 0) * D) * 2 + 16 * c,
+                     v ? 16u : 0u);
         }
       }
-      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-      fence_proxy_async_smem();
-      mbar_arrive(q_full);
+      if (!p.tma_q || lt != 0) {
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+        fence_proxy_async_smem();
+        mbar_arrive(q_full);
+      }
       // ---- KV chunks
-      const int n_chunks = (rs.n + kRows - 1) / kRows;
-      for (int c = 0; c < n_chunks && ok; ++c, ++g) {
-        const int r = c * kRows + lt;
-        bool valid = r < rs.n;
-        const bool win = r >= rs.n1;                 // source-2 (window) row
+      for (int c = 0; c < rs.nchunks && ok; ++c, ++g) {
+        const bool win = c < rs.nc2;                   // window chunk (source 2)
+        const int cl = win ? c : c - rs.nc2;
+        const int r = cl * kRows + lt;
+        bool valid = r < (win ? rs.n2 : rs.n1);
         int64_t row = 0;
         if (valid) {
           if (win) {
-            row = rs.lo2 + (r - rs.n1);
+            row = rs.lo2 + r;
           } else if (rs.idx) {
             row = rs.idx[r];
             if (row < 0 || row >= p.cap) { atomicOr(&g_err_attn, DEV_ERR_BAD_INDEX); valid = false; row = 0; }
@@ -371,34 +445,61 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
             row = r;
           }
         }
+        // TMA boxes load whole 128-row blocks: used when every row of the box is
+        // either in the set or a real row of the same tensor (prefill window rows
+        // past the query are later tokens; masked rows then hold finite data).
+        // Partial chunks of caches, whose tail rows may be unwritten, take the
+        // zero-filling path instead.
+        const int nset = win ? rs.n2 : rs.n1;
+        const bool full = (cl + 1) * kRows <= nset;
+        const bool tma = win ? (p.tma_tok != 0 && (p.src2 == SRC2_WINDOW || full))
+                             : (rs.idx == nullptr && p.tma_kv != 0 && full);
+        if (tma) {
+          // one box of 128 rows x 64 columns per slab; rows past the set are masked later
+          const int32_t y0 = win ? (int32_t)((int64_t)b * p.cap2 + rs.lo2 + (int64_t)cl * kRows)
+                                 : (int32_t)((int64_t)b * p.cap + (int64_t)cl * kRows);
+          for (int tt = 0; tt < NT; ++tt) {
+            if (!wait_bar(&pv_done[tt], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int sl = 2 * tt + h;
+              if (lt == 0) {
+                mbar_expect_tx(&kv_full[sl], kKSlab);
+                tma_load_2d(sKV + sl * kKSlab, win ? &map_tok : &map_kv, 64 * sl, y0, &kv_full[sl]);
+              } else {
+                mbar_arrive(&kv_full[sl]);
+              }
+            }
+          }
+          continue;
+        }
+        // every slab pair is issued as soon as the PV tile that read it retires;
+        // completions are then retired in order (cp.async groups, one per slab)
         for (int tt = 0; tt < NT; ++tt) {
           if (!wait_bar(&pv_done[tt], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int sl = 2 * tt + h;
-            if (win) load_tok_slab<D, KV2, kAsync>(p, b, row, valid, sl, sKV + sl * kKSlab, lt);
+            if constexpr (kAsync) gather_slab_bf16<D>(p, b, row, valid, win, sl, sKV + sl * kKSlab, lt & ~31, lane);
+            else if (win) load_tok_slab<D, KV2, kAsync>(p, b, row, valid, sl, sKV + sl * kKSlab, lt);
             else     load_kv_slab<D, KV>(p, b, row, valid, sl, sKV + sl * kKSlab, lt);
-            if constexpr (kAsync) asm volatile("cp.async.commit_group;" ::: "memory");
-          }
-          if constexpr (kAsync) {
-            if (tt > 0) {
-              asm volatile("cp.async.wait_group 2;" ::: "memory");
+            if constexpr (kAsync) {
+              asm volatile("cp.async.commit_group;" ::: "memory");
+            } else {
               fence_proxy_async_smem();
-              mbar_arrive(&kv_full[2 * tt - 2]);
-              mbar_arrive(&kv_full[2 * tt - 1]);
+              mbar_arrive(&kv_full[sl]);
             }
-          } else {
-            fence_proxy_async_smem();
-            mbar_arrive(&kv_full[2 * tt]);
-            mbar_arrive(&kv_full[2 * tt + 1]);
           }
         }
         if constexpr (kAsync) {
           if (ok) {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-            fence_proxy_async_smem();
-            mbar_arrive(&kv_full[2 * NT - 2]);
-            mbar_arrive(&kv_full[2 * NT - 1]);
+            // NS groups outstanding, oldest first: retire them one by one
+#pragma unroll
+            for (int sl = 0; sl < NS; ++sl) {
+              cp_async_wait_pending(NS - 1 - sl);
+              fence_proxy_async_smem();
+              mbar_arrive(&kv_full[sl]);
+            }
           }
         }
       }
@@ -408,7 +509,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
     // ============================ MMA issuer (lane 0; the warp computes row sets)
     const uint32_t idesc_s = make_idesc(128, kNQ, 1, 1, 0, 0);
     const uint32_t idesc_o = make_idesc(128, kNQ, 1, 1, 1, 1);
-    const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV), aP = smem_u32(sP);
+    // Descriptors differ only in the start-address field (bits 0..13, address >> 4):
+    // build each base once and add compile-time offsets, so an MMA costs one add.
+    const uint64_t dS_A = smem_desc(smem_u32(sKV), 16, 1024, SWZ_128B);       // KV chunk, K-major
+    const uint64_t dS_B = smem_desc(smem_u32(sQ), 16, 1024, SWZ_128B);        // Q tile, K-major
+    const uint64_t dO_A = smem_desc(smem_u32(sKV), kKSlab, 1024, SWZ_128B);   // KV chunk as V^T, MN-major
+    const uint64_t dO_B = smem_desc(smem_u32(sP), 16, 1024, SWZ_128B);        // P^T, MN-major
     uint32_t g = 0, qcount = 0, icount = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -418,17 +524,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       if (lane == 0) {
         if (!wait_bar(q_full, qcount & 1, abort_flag)) ok = false;
         ++qcount;
-        const int n_chunks = (rs.n + kRows - 1) / kRows;
+        const int n_chunks = rs.nchunks;
         for (int c = 0; c < n_chunks && ok; ++c, ++g) {
+#pragma unroll 1
           for (int s = 0; s < NS; ++s) {
             if (!wait_bar(&kv_full[s], g & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              uint64_t ad = smem_desc(aKV + s * kKSlab + kk * 32, 16, 1024, SWZ_128B);
-              uint64_t bd = smem_desc(aQ + s * kQSlab + kk * 32, 16, 1024, SWZ_128B);
-              mma_bf16(tmem, ad, bd, idesc_s, (s | kk) != 0);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem, dS_A + ((s * kKSlab + kk * 32) >> 4), dS_B + ((s * kQSlab + kk * 32) >> 4), idesc_s,
+                       (s | kk) != 0);
           }
           if (!ok) break;
           mma_commit(s_done);
@@ -436,13 +541,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
           if (!wait_bar(p_full, g & 1, abort_flag)) { ok = false; break; }
           if (c == 0 && !wait_bar(epi_done, (icount & 1) ^ 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t acc0 = c > 0 ? 1u : 0u;
+#pragma unroll 1
           for (int tt = 0; tt < NT; ++tt) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              uint64_t ad = smem_desc(aKV + (2 * tt) * kKSlab + kk * 2048, kKSlab, 1024, SWZ_128B);
-              uint64_t bd = smem_desc(aP + kk * 2048, 16, 1024, SWZ_128B);
-              mma_bf16(tmem + 64 + 64 * tt, ad, bd, idesc_o, (c > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16(tmem + 64 + 64 * tt, dO_A + ((2 * tt * kKSlab + kk * 2048) >> 4), dO_B + ((kk * 2048) >> 4),
+                       idesc_o, kk > 0 ? 1u : acc0);
             mma_commit(&pv_done[tt]);
           }
         }
@@ -473,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
       }
       float m_own[2] = {-CUDART_INF_F, -CUDART_INF_F};   // running max of columns lane, 32 + lane
       float l_own[2] = {0.f, 0.f};
-      const int n_chunks = (rs.n + kRows - 1) / kRows;
+      const int n_chunks = rs.nchunks;
       for (int c = 0; c < n_chunks && ok; ++c, ++g) {
         if (!wait_bar(s_done, g & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -481,9 +586,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_ld16(tmem + lane_base + 16 * q, x + 16 * q);
         tmem_wait_ld();
-        const bool valid = c * kRows + e < rs.n;
+        const bool valid = c < rs.nc2 ? c * kRows + e < rs.n2 : (c - rs.nc2) * kRows + e < rs.n1;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) x[j] = valid ? x[j] * p.scale_log2 : -CUDART_INF_F;
+        for (int j = 0; j < 64; ++j) x[j] = valid ? x[j] : -CUDART_INF_F;   // raw logits; scale folded below
         // column maxima over this warp's 32 rows: lane ends with columns lane, 32 + lane
         float cm[2];
 #pragma unroll
@@ -512,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int col = 32 * h + lane;
-          float mx = fmaxf(fmaxf(red[col], red[64 + col]), fmaxf(red[128 + col], red[192 + col]));
+          float mx = fmaxf(fmaxf(red[col], red[64 + col]), fmaxf(red[128 + col], red[192 + col])) * p.scale_log2;
           float mn = (mx > m_own[h] + kTau) ? mx : m_own[h];
           alpha[h] = exp2f(m_own[h] - mn);             // 0 on the first chunk
           if (mn != m_own[h] && c > 0) need_rescale = true;
@@ -523,11 +628,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         need_rescale = __any_sync(0xffffffffu, need_rescale);
         __syncwarp();
         float p_[64];
+        const float sl2 = p.scale_log2;
 #pragma unroll
         for (int j = 0; j < 64; j += 4) {
           float4 mm = *reinterpret_cast<const float4*>(bc_m + j);
-          p_[j] = exp2f(x[j] - mm.x); p_[j + 1] = exp2f(x[j + 1] - mm.y);
-          p_[j + 2] = exp2f(x[j + 2] - mm.z); p_[j + 3] = exp2f(x[j + 3] - mm.w);
+          p_[j] = fast_exp2(fmaf(x[j], sl2, -mm.x)); p_[j + 1] = fast_exp2(fmaf(x[j + 1], sl2, -mm.y));
+          p_[j + 2] = fast_exp2(fmaf(x[j + 2], sl2, -mm.z)); p_[j + 3] = fast_exp2(fmaf(x[j + 3], sl2, -mm.w));
         }
         // P^T row e -> shared memory (MN-major B operand of the PV MMA)
 #pragma unroll
@@ -608,10 +714,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         tc_fence_after();
       }
       const int64_t obase = ((int64_t)b * p.T + t) * p.H;
+      // Each 128-d tile is written in two halves of 32 heads.  Phase A: every
+      // thread (one TMEM lane = one d) scales its accumulators and stages them
+      // as fp32 [32 heads][128 d] in sP (free once the last PV retired).
+      // Phase B: the 128 threads walk the staged rows in order, add the
+      // compressed-branch partial, apply the inverse RoPE, and store 16-byte
+      // vectors, so every global write is a full, coalesced row segment.
+      float* stage = reinterpret_cast<float*>(sP);
+      const int r0 = D - p.rope_dim;
       for (int tt = 0; tt < NT; ++tt) {
-        const int d = tt * 128 + e;
-        const bool rope_tile = EPI == EPI_COMBINE && p.inv_rope && tt == NT - 1;
-        // 32 query rows at a time keeps the live set small
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
           float o[32];
@@ -623,57 +734,69 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = 0.f;
           }
-          if (EPI == EPI_PARTIAL) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int c = 32 * hh + i;
-              if (c < p.H) p.O_part[(obase + c) * D + d] = o[i] * bc_m[64 + c];
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int c = 32 * hh + i;
-              float v = o[i] * bc_m[64 + c];
-              if (p.O_in && c < p.H) v = fmaf(bc_m[128 + c], p.O_in[(obase + c) * D + d], v);
-              o[i] = v;
-            }
-            const int r0 = D - p.rope_dim;
-            if (rope_tile) {
-              // pairs (d, d + 32) of the last 64 dims sit in warps 2 and 3: swap through sP
-              float* ex = reinterpret_cast<float*>(sP);
-              named_bar_sync(2, 128);
-              if (d >= r0) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) ex[i * 64 + (d - r0)] = o[i];
+          for (int i = 0; i < 32; ++i) stage[i * 128 + e] = o[i] * bc_m[64 + 32 * hh + i];
+          named_bar_sync(2, 128);
+          // phase B: 16 threads per head row, 8 consecutive d each
+          const int cl0 = e >> 4, dl = (e & 15) * 8;
+#pragma unroll 1
+          for (int cl = cl0; cl < 32; cl += 8) {
+            const int c = 32 * hh + cl;
+            if (c >= p.H) break;
+            float v[8];
+            const float4 a0 = *reinterpret_cast<const float4*>(stage + cl * 128 + dl);
+            const float4 a1 = *reinterpret_cast<const float4*>(stage + cl * 128 + dl + 4);
+            v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w; v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+            const int d0 = tt * 128 + dl;
+            const int64_t grow = (obase + c) * D + d0;
+            if (EPI == EPI_COMBINE) {
+              if (p.O_in) {
+                const float cp = bc_m[128 + c];
+                const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.O_in + grow));
+                const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.O_in + grow) + 1);
+                v[0] = fmaf(cp, b0.x, v[0]); v[1] = fmaf(cp, b0.y, v[1]); v[2] = fmaf(cp, b0.z, v[2]);
+                v[3] = fmaf(cp, b0.w, v[3]); v[4] = fmaf(cp, b1.x, v[4]); v[5] = fmaf(cp, b1.y, v[5]);
+                v[6] = fmaf(cp, b1.z, v[6]); v[7] = fmaf(cp, b1.w, v[7]);
               }
-              named_bar_sync(2, 128);
-              if (d >= r0) {
-                const int jj = d - r0, half = p.rope_dim / 2;
-                const float2 csj = cs[jj % half];
+              if (p.inv_rope && d0 >= r0) {
+                // inverse rotation by -pos: (a, b) -> (a cos + b sin, -a sin + b cos)
+                const int half = p.rope_dim / 2;
+                const int jj0 = d0 - r0;
+                const bool first = jj0 < half;
+                const int pd = dl + (first ? half : -half);
+                float w[8];
+                const float4 c0 = *reinterpret_cast<const float4*>(stage + cl * 128 + pd);
+                const float4 c1 = *reinterpret_cast<const float4*>(stage + cl * 128 + pd + 4);
+                w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w; w[4] = c1.x; w[5] = c1.y; w[6] = c1.z; w[7] = c1.w;
+                if (p.O_in) {
+                  const float cp = bc_m[128 + c];
+                  const int64_t prow = grow + (first ? half : -half);
+                  const float4 e0 = __ldg(reinterpret_cast<const float4*>(p.O_in + prow));
+                  const float4 e1 = __ldg(reinterpret_cast<const float4*>(p.O_in + prow) + 1);
+                  w[0] = fmaf(cp, e0.x, w[0]); w[1] = fmaf(cp, e0.y, w[1]); w[2] = fmaf(cp, e0.z, w[2]);
+                  w[3] = fmaf(cp, e0.w, w[3]); w[4] = fmaf(cp, e1.x, w[4]); w[5] = fmaf(cp, e1.y, w[5]);
+                  w[6] = fmaf(cp, e1.z, w[6]); w[7] = fmaf(cp, e1.w, w[7]);
+                }
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                  // inverse rotation by -pos: (a, b) -> (a cos + b sin, -a sin + b cos)
-                  if (jj < half) o[i] = o[i] * csj.x + ex[i * 64 + jj + half] * csj.y;
-                  else           o[i] = o[i] * csj.x - ex[i * 64 + jj - half] * csj.y;
+                for (int i = 0; i < 8; ++i) {
+                  const float2 csj = cs[(jj0 + i) % half];
+                  v[i] = first ? v[i] * csj.x + w[i] * csj.y : v[i] * csj.x - w[i] * csj.y;
                 }
               }
-            }
-            if (p.out_bf16) {
-              __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int c = 32 * hh + i;
-                if (c < p.H) out[(obase + c) * D + d] = __float2bfloat16_rn(o[i]);
+              if (p.out_bf16) {
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + grow) = to_bf16x8(v);
+              } else {
+                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + grow);
+                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
               }
             } else {
-              float* out = reinterpret_cast<float*>(p.out);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int c = 32 * hh + i;
-                if (c < p.H) out[(obase + c) * D + d] = o[i];
-              }
+              float4* dst = reinterpret_cast<float4*>(p.O_part + grow);
+              dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+              dst[1] = make_float4(v[4], v[5], v[6], v[7]);
             }
           }
+          named_bar_sync(2, 128);   // staging buffer reused by the next half
         }
       }
       if (rs.n > 0) {
@@ -696,8 +819,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
   }
 }
 
+struct AttnMaps {
+  CUtensorMap q, kv, tok;
+};
+
 template <int D, int KV, int EPI>
-csa_status_t launch_attn(const AttnParams& p, cudaStream_t st) {
+csa_status_t launch_attn(const AttnParams& p, const AttnMaps& m, cudaStream_t st) {
   constexpr int NS = D / 64, NT = D / 128;
   const size_t smem = 1024 + NS * (kNQ * 128) + NS * (kRows * 128) + kRows * 128 +
                       (2 * 4 * 64 + 4 * 3 * 64) * 4 + 64 * 8 + (5 + NS + NT) * 8 + 16;
@@ -707,20 +834,50 @@ csa_status_t launch_attn(const AttnParams& p, cudaStream_t st) {
   const int64_t items = (int64_t)p.n_seq * p.T;
   if (items == 0) return CSA_OK;
   const int grid = (int)std::min<int64_t>(items, num_sms());
-  kern<<<grid, kThreads, smem, st>>>(p);
+  kern<<<grid, kThreads, smem, st>>>(p, m.q, m.kv, m.tok);
   return check_launch("attention");
 }
 
-template <int EPI>
-csa_status_t dispatch(const AttnParams& p, int D, csa_dtype_t kv_dtype, cudaStream_t st) {
-  if (D == 512) {
-    if (kv_dtype == CSA_BF16) return launch_attn<512, KV_BF16, EPI>(p, st);
-    if (kv_dtype == CSA_F32) return launch_attn<512, KV_F32, EPI>(p, st);
-    return launch_attn<512, KV_FP8, EPI>(p, st);
+// Builds the tile maps that apply (bf16 rows, 64 x 128-row boxes, 128-byte
+// swizzle) and sets the matching flags; other maps stay zero and unused.
+csa_status_t build_maps(AttnParams& p, AttnMaps& m, int D, csa_dtype_t q_dtype, csa_dtype_t kv_dtype,
+                        csa_dtype_t tok_dtype) {
+  memset(&m, 0, sizeof(m));
+  const int64_t rows_q = (int64_t)p.n_seq * p.T * p.H;
+  if (q_dtype == CSA_BF16 && rows_q > 0 && rows_q < ((int64_t)1 << 31)) {
+    if (!encode_2d(&m.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, D, rows_q, 64, kNQ, CU_TENSOR_MAP_SWIZZLE_128B))
+      return fail(CSA_ERR_CUDA, "attention: cuTensorMapEncodeTiled (queries) failed");
+    p.tma_q = 1;
   }
-  if (kv_dtype == CSA_BF16) return launch_attn<128, KV_BF16, EPI>(p, st);
-  if (kv_dtype == CSA_F32) return launch_attn<128, KV_F32, EPI>(p, st);
-  return launch_attn<128, KV_FP8, EPI>(p, st);
+  const int64_t rows_kv = (int64_t)p.n_seq * p.cap;
+  if (p.src1 == SRC1_DENSE && kv_dtype == CSA_BF16 && rows_kv < ((int64_t)1 << 31)) {
+    if (!encode_2d(&m.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.kv, D, rows_kv, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B))
+      return fail(CSA_ERR_CUDA, "attention: cuTensorMapEncodeTiled (entries) failed");
+    p.tma_kv = 1;
+  }
+  const int64_t rows_tok = (int64_t)p.n_seq * p.cap2;
+  if (p.src2 != SRC2_NONE && tok_dtype == CSA_BF16 && rows_tok < ((int64_t)1 << 31)) {
+    if (!encode_2d(&m.tok, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.kv2, D, rows_tok, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B))
+      return fail(CSA_ERR_CUDA, "attention: cuTensorMapEncodeTiled (window) failed");
+    p.tma_tok = 1;
+  }
+  return CSA_OK;
+}
+
+template <int EPI>
+csa_status_t dispatch(AttnParams& p, int D, csa_dtype_t q_dtype, csa_dtype_t kv_dtype, csa_dtype_t tok_dtype,
+                      cudaStream_t st) {
+  AttnMaps m;
+  csa_status_t s = build_maps(p, m, D, q_dtype, kv_dtype, tok_dtype);
+  if (s != CSA_OK) return s;
+  if (D == 512) {
+    if (kv_dtype == CSA_BF16) return launch_attn<512, KV_BF16, EPI>(p, m, st);
+    if (kv_dtype == CSA_F32) return launch_attn<512, KV_F32, EPI>(p, m, st);
+    return launch_attn<512, KV_FP8, EPI>(p, m, st);
+  }
+  if (kv_dtype == CSA_BF16) return launch_attn<128, KV_BF16, EPI>(p, m, st);
+  if (kv_dtype == CSA_F32) return launch_attn<128, KV_F32, EPI>(p, m, st);
+  return launch_attn<128, KV_FP8, EPI>(p, m, st);
 }
 
 csa_status_t check_common(const char* fn, const void* q, csa_dtype_t q_dtype, const void* kv, csa_dtype_t kv_dtype,
@@ -760,7 +917,7 @@ extern "C" csa_status_t csa_sparse_mqa(const void* q, csa_dtype_t q_dtype, const
   p.cap = cap; p.src1 = SRC1_GATHER; p.idx = idx; p.k = k; p.m = 1; p.src2 = SRC2_NONE;
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = O_part; p.lse_part = lse_part; p.rope_dim = rope_dim;
-  return dispatch<EPI_PARTIAL>(p, D, kv_dtype, stream);
+  return dispatch<EPI_PARTIAL>(p, D, q_dtype, kv_dtype, kv_dtype, stream);
 }
 
 extern "C" csa_status_t hca_dense_attn(const void* q, csa_dtype_t q_dtype, const void* kv,
@@ -778,7 +935,7 @@ extern "C" csa_status_t hca_dense_attn(const void* q, csa_dtype_t q_dtype, const
   p.cap = cap; p.q_pos = q_pos; p.src1 = SRC1_DENSE; p.m = m; p.src2 = SRC2_NONE;
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = O_part; p.lse_part = lse_part; p.rope_dim = rope_dim;
-  return dispatch<EPI_PARTIAL>(p, D, kv_dtype, stream);
+  return dispatch<EPI_PARTIAL>(p, D, q_dtype, kv_dtype, kv_dtype, stream);
 }
 
 extern "C" csa_status_t swa_sink_combine(const void* q, csa_dtype_t q_dtype, const void* kv_tok,
@@ -804,7 +961,7 @@ extern "C" csa_status_t swa_sink_combine(const void* q, csa_dtype_t q_dtype, con
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_in = O_part; p.lse_in = lse_part; p.sink = sink; p.out = out; p.out_bf16 = out_dtype == CSA_BF16;
   p.inv_rope = inv_rope; p.rope_dim = rope_dim; p.rope_base = rope_base;
-  return dispatch<EPI_COMBINE>(p, D, kv_dtype, stream);
+  return dispatch<EPI_COMBINE>(p, D, q_dtype, kv_dtype, kv_dtype, stream);
 }
 
 extern "C" csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, const void* kv, csa_dtype_t kv_dtype,
@@ -833,5 +990,5 @@ extern "C" csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, 
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
   p.sink = sink; p.out = out; p.out_bf16 = out_dtype == CSA_BF16;
   p.inv_rope = inv_rope; p.rope_dim = rope_dim; p.rope_base = rope_base;
-  return dispatch<EPI_COMBINE>(p, D, kv_dtype, stream);
+  return dispatch<EPI_COMBINE>(p, D, q_dtype, kv_dtype, tok_dtype, stream);
 }

@@ -28,6 +28,7 @@
 #include <math_constants.h>
 #include "common.cuh"
 #include "tc.cuh"
+#include "tmap.cuh"
 
 namespace csa {
 
@@ -43,33 +44,12 @@ uint32_t read_clear_err_indexer() {
 namespace {
 
 // ------------------------------------------------------------------ TMA maps
-PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 // 2-D byte tensor [rows, row_bytes] with boxes of [box_rows, row_bytes],
 // swizzled to match the tcgen05 K-major layout of the same width.
 bool make_byte_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes, uint32_t box_rows) {
-  auto enc = tmap_encoder();
-  if (!enc) return false;
   CUtensorMapSwizzle swz = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                          : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-  cuuint64_t gdim[2] = {row_bytes, rows};
-  cuuint64_t gstride[1] = {row_bytes};
-  cuuint32_t box[2] = {row_bytes, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), gdim, gstride, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, row_bytes, rows, row_bytes, box_rows, swz);
 }
 
 // ------------------------------------------------------------------ scores
@@ -88,10 +68,13 @@ struct IdxParams {
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  // a few tight polls, then back off with nanosleep so that waiting warps do not
+  // flood the shared-memory pipe that the loads and stores of other warps use
   uint64_t start = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0) {
+    if (i > 8) __nanosleep(i < 64 ? 32 : 128);
+    if ((i & 63u) == 0) {
       if (*abort_flag) return false;
       const uint64_t now = global_ns();
       if (start == 0) start = now;
@@ -113,7 +96,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                       IdxParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // aligned by offsetting the shared array itself, so accesses stay in the shared window
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int b = blockIdx.z, qb = blockIdx.y, chunk = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t0 = qb * p.TQ;
