@@ -149,6 +149,61 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None):
+    """CSA decode at 2^20 context, batch 16 (one new token per sequence): indexer
+    scan over the e4m3 key cache + top-k, then the fused attention over the 512
+    selected e4m3 entries, the 128-row bf16 SWA cache and the sink."""
+    inp, cfg = synth.decode_inputs_device("csa_decode_1m", dev, seed=1, batch=batch)
+    Bn, ne, k, W, H, D, HI, DI = (cfg[x] for x in ("batch", "n_e", "k", "W", "H", "D", "HI", "DI"))
+    ws = torch.empty(csa.csa_index_topk_workspace(Bn, 1, ne, k), dtype=torch.uint8, device=dev)
+    idx = torch.empty(Bn, 1, k, dtype=torch.int32, device=dev)
+    out = torch.empty(Bn, 1, H, D, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        csa.csa_index_topk(inp["qI"], inp["w"], inp["kI"], inp["q_pos"], 4, k, qI_scale=inp["qI_scale"],
+                           kI_scale=inp["kI_scale"], workspace=ws, idx=idx)
+        if ev is not None:
+            ev[1].record(stream)
+        csa.csa_fused_attention(inp["q"], inp["kv_nope"], inp["swa"], inp["q_pos"], W, inp["sink"], idx=idx,
+                                kv_rope=inp["kv_rope"], kv_scale=inp["kv_scale"], window_mode=1, inv_rope=True,
+                                rope_dim=64, out=out)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(3, warmup)):
+        step()
+    csa.check_device_error()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    t_idx = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    t_att = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms = float(np.mean([e[0].elapsed_time(e[2]) for e in evs]))
+    # algorithmic bytes: every visible indexer key + scale, the selected e4m3 rows
+    # (448 + 128 + 4 bytes), the SWA rows, the queries; plus the fp32 score row
+    # written and read once by the selection
+    scan = Bn * ne * (DI + 4)
+    gather = Bn * k * (D - 64 + 128 + 4)
+    swa = Bn * W * D * 2
+    qbytes = Bn * (H * D * 2 + HI * DI + HI * 8)
+    algo = scan + gather + swa + qbytes
+    hbm, _, _, src = _peaks()
+    ach_idx = scan / (t_idx * 1e-3) / 1e9
+    return {"workload": "csa_decode_1m", "batch": Bn, "context": cfg["ctx"], "entries": ne, "top_k": k,
+            "tokens_per_s": Bn / (ms * 1e-3), "ms_per_step": ms, "kernels_ms": {"index_topk": t_idx,
+                                                                                 "fused_attention": t_att},
+            "algorithmic_bytes_per_step": algo,
+            "hbm_frac_step": algo / (ms * 1e-3) / 1e9 / hbm,
+            "roofline": {"kernel": "index_topk", "bound": "hbm", "achieved": ach_idx, "peak": hbm, "unit": "GB/s",
+                         "frac": ach_idx / hbm, "traffic": None, "peak_source": f"{src} copy bandwidth"}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -158,6 +213,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--S", type=int, default=None, help="shorter sequence (profiling cases only)")
+    ap.add_argument("--no-decode", action="store_true", help="skip the 1M-context decode leg")
+    ap.add_argument("--decode-batch", type=int, default=None, help="fewer decode sequences (profiling cases only)")
+    ap.add_argument("--no-prefill", action="store_true", help="run only the decode leg (profiling cases only)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -180,6 +238,11 @@ def main():
     build.build()
     csa.lib()
 
+    if args.no_prefill:
+        d = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch)
+        if rank == 0:
+            print(json.dumps({"decode_1m": d}), flush=True)
+        return
     inp, cfg = synth.prefill_inputs_device(WORKLOAD, dev, seed=rank, S=args.S)
     S, H, D, m, k, W, HI, DI = (cfg[x] for x in ("S", "H", "D", "m", "k", "W", "HI", "DI"))
     ne = S // m
@@ -288,6 +351,10 @@ def main():
         roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s", "frac": None,
                 "traffic": None}
 
+    decode = None
+    if not args.no_decode and args.S is None:
+        decode = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = host_inputs(inp)
@@ -313,7 +380,7 @@ def main():
                            "flops_per_step": {"sparse_mqa": fl_sparse, "swa_window": fl_window,
                                               "indexer_fp8": fl_index}},
                 "prefill_tokens_per_s": world * S / (ms * 1e-3),
-                "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -183,60 +183,85 @@ compress_kernel(const Tin* __restrict__ C, const Tin* __restrict__ Z, const Tin*
   if (owner) Vec8<Tout>::store(out + i * D + ch0, x);
 }
 
+// cos/sin for RoPE pair j at position pos: the angle pos * base^(-2j/r) is formed
+// and reduced modulo 2*pi in double (positions reach 2^20 and beyond), then the
+// reduced angle is evaluated in single precision.
+__device__ __forceinline__ float2 rope_cs_fast(int64_t pos, int j, int rope_dim, float rope_base) {
+  const double inv_freq = exp2(-2.0 * (double)j / (double)rope_dim * log2((double)rope_base));
+  double a = (double)pos * inv_freq;
+  a -= floor(a * 0.15915494309189535) * 6.283185307179586;
+  float sn, cs;
+  sincosf((float)a, &sn, &cs);
+  return make_float2(cs, sn);
+}
+
 // Rows of `rows_per_pos` share one position; a CTA handles `ppb` positions.
-// Each warp normalises whole rows: lane owns D/32 consecutive channels.
+// A warp normalises two rows at a time; lane owns D/32 consecutive channels.
+// Lanes holding RoPE dims also load their partner channels (d -+ half) directly,
+// so the rotation needs no cross-lane exchange.
 template <typename Tin, typename Tout, int CPL>
 __global__ void __launch_bounds__(kThreads)
 rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int D, int rows_per_pos, int64_t pos0,
                     int ppb, int norm, int rope_dim, float rope_base, float eps, Tout* __restrict__ out) {
-  __shared__ float2 s_cs[8][64];
+  constexpr int RPW = 2;
+  __shared__ float2 s_cs[32][32];   // [position in CTA][pair]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t p_first = (int64_t)blockIdx.x * ppb;
   const int half = rope_dim / 2;
   for (int e = tid; e < ppb * half; e += kThreads) {
-    int pl = e / half, j = e % half;
-    float c, s;
-    rope_cs(pos0 + p_first + pl, j, rope_dim, rope_base, &c, &s);
-    s_cs[pl][j] = make_float2(c, s);
+    const int pl = e / half, j = e % half;
+    s_cs[pl][j] = rope_cs_fast(pos0 + p_first + pl, j, rope_dim, rope_base);
   }
   __syncthreads();
   const int64_t r_begin = p_first * rows_per_pos;
   const int64_t r_end = min(rows, (p_first + ppb) * rows_per_pos);
-  for (int64_t r = r_begin + warp; r < r_end; r += kThreads / 32) {
-    float v[CPL];
-    const Tin* src = x + r * D + lane * CPL;
+  const int r0d = D - rope_dim;
+  const int d0 = lane * CPL;
+  const bool in_rope = rope_dim > 0 && d0 >= r0d;
+  const bool first_half = d0 < r0d + half;
+  const int pd0 = first_half ? d0 + half : d0 - half;     // partner channels
+  for (int64_t rb = r_begin + warp * RPW; rb < r_end; rb += (kThreads / 32) * RPW) {
+    float v[RPW][CPL], u[RPW][CPL];
 #pragma unroll
-    for (int c = 0; c < CPL; c += 8) Vec8<Tin>::load(src + c, v + c);
-    if (norm) {
-      float ss = 0.f;
+    for (int k = 0; k < RPW; ++k) {
+      const int64_t r = min(rb + k, r_end - 1);
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) ss = fmaf(v[c], v[c], ss);
+      for (int c = 0; c < CPL; c += 8) Vec8<Tin>::load(x + r * D + d0 + c, v[k] + c);
+      if (in_rope) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      float inv = rsqrtf(ss / (float)D + eps);
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) v[c] *= inv;
-    }
-    if (rope_dim > 0) {
-      const int pl = (int)(r / rows_per_pos - p_first);
-      const int r0 = D - rope_dim;
-      const int partner = half / CPL;   // lane distance between (d, d + half)
-      float w[CPL];
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        float up = __shfl_down_sync(0xffffffffu, v[c], partner);
-        float dn = __shfl_up_sync(0xffffffffu, v[c], partner);
-        int d = lane * CPL + c;
-        if (d < r0) { w[c] = v[c]; continue; }
-        int j = (d - r0) % half;
-        float2 cs = s_cs[pl][j];
-        w[c] = (d < r0 + half) ? v[c] * cs.x - up * cs.y : dn * cs.y + v[c] * cs.x;
+        for (int c = 0; c < CPL; c += 8) Vec8<Tin>::load(x + r * D + pd0 + c, u[k] + c);
       }
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) v[c] = w[c];
     }
 #pragma unroll
-    for (int c = 0; c < CPL; c += 8) Vec8<Tout>::store(out + r * D + lane * CPL + c, v + c);
+    for (int k = 0; k < RPW; ++k) {
+      const int64_t r = rb + k;
+      float inv = 1.f;
+      if (norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) ss = fmaf(v[k][c], v[k][c], ss);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        inv = rsqrtf(ss / (float)D + eps);
+      }
+      float o[CPL];
+      if (in_rope) {
+        const int pl = (int)(min(r, r_end - 1) / rows_per_pos - p_first);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          const float2 cs = s_cs[pl][(d0 + c - r0d) % half];
+          const float a = v[k][c] * inv, bb = u[k][c] * inv;
+          o[c] = first_half ? a * cs.x - bb * cs.y : bb * cs.y + a * cs.x;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) o[c] = v[k][c] * inv;
+      }
+      if (r < r_end) {
+#pragma unroll
+        for (int c = 0; c < CPL; c += 8) Vec8<Tout>::store(out + r * D + d0 + c, o + c);
+      }
+    }
   }
 }
 
@@ -266,7 +291,7 @@ csa_status_t launch_compress(const void* C, const void* Z, const void* Cb, const
 template <typename Tin, typename Tout, int CPL>
 csa_status_t launch_norm(const void* x, int64_t rows, int D, int rpp, int64_t pos0, int norm, int rope_dim,
                          float rope_base, float eps, void* out, cudaStream_t st) {
-  int ppb = rpp >= 8 ? 1 : 8 / rpp;
+  int ppb = rpp >= 32 ? 1 : 32 / rpp;      // 32 rows per CTA pass (8 warps x 4 rows)
   int64_t npos = (rows + rpp - 1) / rpp;
   int64_t grid = (npos + ppb - 1) / ppb;
   if (grid == 0) return CSA_OK;

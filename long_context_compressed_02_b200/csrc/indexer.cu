@@ -209,11 +209,17 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     const int log2hi = __ffs(p.HI) - 1;
     const uint32_t w_addr = smem_u32(s_w);
     const int key_in_tile = sp * 32 + lane;
+    auto key_scale = [&](int it) -> float {
+      const int64_t key = (int64_t)(tile0 + it) * 128 + key_in_tile;
+      return (key < p.cap && it < n_tiles) ? (p.ks ? __ldg(p.ks + (int64_t)b * p.cap + key) : 1.f) : 0.f;
+    };
+    float ksc_next = key_scale(0);
     for (int it = 0; it < n_tiles; ++it) {
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       const int64_t key = (int64_t)(tile0 + it) * 128 + key_in_tile;
-      const float ksc = (key < p.cap) ? (p.ks ? p.ks[(int64_t)b * p.cap + key] : 1.f) : 0.f;
+      const float ksc = ksc_next;
+      ksc_next = key_scale(it + 1);          // issued a tile ahead: off the critical path
       if (!wait_bar(&tfull[acc], aph, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N;
@@ -281,6 +287,7 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 struct SelectSmem {
+  uint32_t whist[kTopkThreads / 32][256];
   uint32_t hist[256];
   uint64_t warp_tot[kTopkThreads / 32];
   uint32_t digit, above;
@@ -315,11 +322,20 @@ __device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id
     uint32_t prefix = 0, mask = 0;
     int remaining = k;
     for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kTopkThreads) ss.hist[i] = 0;
+      for (int i = tid; i < 256 * (kTopkThreads / 32); i += kTopkThreads) (&ss.whist[0][0])[i] = 0;
       __syncthreads();
+      // per-warp private histograms: scores share their top bits, so a single
+      // histogram would serialise every warp on one bin
       for (int e = tid; e < n; e += kTopkThreads) {
         const uint32_t key = keys[e];
-        if ((key & mask) == prefix) atomicAdd(&ss.hist[(key >> shift) & 255u], 1u);
+        if ((key & mask) == prefix) atomicAdd(&ss.whist[tid >> 5][(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      for (int i = tid; i < 256; i += kTopkThreads) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int w = 0; w < kTopkThreads / 32; ++w) t += ss.whist[w][i];
+        ss.hist[i] = t;
       }
       __syncthreads();
       if (tid < 32) {
@@ -546,7 +562,8 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
   tp.cand_cnt = reinterpret_cast<int32_t*>(ws + L.cand_cnt);
   const int64_t rows = (int64_t)n_seq * T;
   CSA_REQUIRE(rows <= 0x7fffffff, "csa_index_topk: too many rows");
-  const size_t smem1 = kChunk * sizeof(uint32_t);
+  // key buffer sized to the longest chunk actually present (rows of <= 16384 entries)
+  const size_t smem1 = (size_t)std::min<int64_t>(kChunk, cap) * sizeof(uint32_t);
   cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   dim3 g1((unsigned)rows, (unsigned)L.n_chunks);
   topk_chunk_kernel<<<g1, kTopkThreads, smem1, stream>>>(tp);

@@ -178,3 +178,51 @@ def prefill_inputs_device(name: str, device, seed: int = 0, S: int | None = None
         out["kI_codes"] = kI.to(torch.float8_e4m3fn).view(torch.uint8)
         out["w"] = w.contiguous()
     return out, dict(cfg, S=S)
+
+
+def decode_inputs_device(name: str, device, seed: int = 0, grid: bool = False, batch: int | None = None,
+                         ctx: int | None = None):
+    """Batched decode-step inputs for `csa_decode_1m` on `device` (torch's seeded
+    generator), stacked over the batch:
+      kv_nope [B, n_e, D-64] e4m3, kv_rope [B, n_e, 64] bf16, kv_scale [B, n_e] f32,
+      kI [B, n_e, DI] e4m3, kI_scale [B, n_e] f32 (row scales 2^U{-2..2}, codes N(0,1)/scale),
+      q [B, 1, H, D] bf16, qI [B, 1, HI, DI] e4m3, qI_scale [B, 1, HI], w [B, 1, HI] f32,
+      swa [B, W, D] bf16, sink [H] f32, q_pos [B] int64 (= context - 1).
+    grid=True puts the indexer values on the 1/8 grid (w on 1/16) with unit scales."""
+    cfg = dict(WORKLOADS[name])
+    B = cfg["batch"] if batch is None else batch
+    L = cfg["ctx"] if ctx is None else ctx
+    H, D, HI, DI, W, r = cfg["H"], cfg["D"], cfg["HI"], cfg["DI"], cfg["W"], cfg["rope_dim"]
+    m = cfg["m"]
+    ne = L // m
+    g = torch.Generator(device=device).manual_seed(seed)
+
+    def pow2(*shape):
+        return torch.pow(2.0, torch.randint(-2, 3, shape, generator=g, device=device).float())
+
+    out = {}
+    sc = pow2(B, ne)
+    out["kv_nope"] = (torch.randn(B, ne, D - r, generator=g, device=device) / sc[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    out["kv_rope"] = torch.randn(B, ne, r, generator=g, device=device).to(torch.bfloat16)
+    out["kv_scale"] = sc
+    ks = pow2(B, ne)
+    y = torch.randn(B, ne, DI, generator=g, device=device)
+    qs = pow2(B, 1, HI)
+    x = torch.randn(B, 1, HI, DI, generator=g, device=device)
+    if grid:
+        y, x = torch.round(y * 8) / 8, torch.round(x * 8) / 8
+        ks, qs = torch.ones_like(ks), torch.ones_like(qs)
+        w = torch.floor(torch.rand(B, 1, HI, generator=g, device=device) * 16) / 16
+    else:
+        y, x = y / ks[..., None], x / qs[..., None]
+        w = torch.rand(B, 1, HI, generator=g, device=device)
+    out["kI"] = y.to(torch.float8_e4m3fn).view(torch.uint8)
+    out["kI_scale"] = ks
+    out["qI"] = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    out["qI_scale"] = qs
+    out["w"] = w.contiguous()
+    out["q"] = torch.randn(B, 1, H, D, generator=g, device=device).to(torch.bfloat16)
+    out["swa"] = torch.randn(B, W, D, generator=g, device=device).to(torch.bfloat16)
+    out["sink"] = torch.randn(H, generator=g, device=device)
+    out["q_pos"] = torch.full((B,), L - 1, dtype=torch.int64, device=device)
+    return out, dict(cfg, batch=B, ctx=L, n_e=ne)

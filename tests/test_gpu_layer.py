@@ -88,3 +88,48 @@ def test_flash_prefill_full_size_sampled_rows():
     ref, ridx = _oracle_csa(inp, cfg, rows=rows, store=O.bf16_round)
     assert np.array_equal(idx.cpu().numpy()[rows], ridx)
     assert_close(host(out[torch.from_numpy(rows).cuda()]), ref, what="full-size sampled rows")
+
+
+@pytest.mark.parametrize("grid", [True, False])
+def test_csa_decode_1m_full_size_sampled(grid):
+    """The 1M-context decode workload (16 sequences x 2^18 e4m3 entries): the
+    indexer + top-k and the fused attention through the C ABI; two sequences
+    checked against the oracle (bit-exact selection on grid values; on
+    continuous values the selection may differ only within the fp32 rounding
+    bound, and the output is compared when the sets agree)."""
+    import long_context_compressed_02_b200 as csa
+    inp, cfg = synth.decode_inputs_device("csa_decode_1m", "cuda", seed=3, grid=grid)
+    Bn, ne, k, W, H, D = (cfg[x] for x in ("batch", "n_e", "k", "W", "H", "D"))
+    idx = csa.csa_index_topk(inp["qI"], inp["w"], inp["kI"], inp["q_pos"], 4, k, qI_scale=inp["qI_scale"],
+                             kI_scale=inp["kI_scale"])
+    out = csa.csa_fused_attention(inp["q"], inp["kv_nope"], inp["swa"], inp["q_pos"], W, inp["sink"], idx=idx,
+                                  kv_rope=inp["kv_rope"], kv_scale=inp["kv_scale"], window_mode=1, inv_rope=True,
+                                  rope_dim=64, out_dtype=torch.float32)
+    csa.check_device_error()
+    t = cfg["ctx"] - 1
+    for b in (0, 9):
+        kI = O.e4m3_decode(inp["kI"][b].cpu().numpy()) * inp["kI_scale"][b].cpu().numpy()[:, None]
+        qI = O.e4m3_decode(inp["qI"][b, 0].cpu().numpy()) * inp["qI_scale"][b, 0].cpu().numpy()[:, None]
+        w = inp["w"][b, 0].cpu().numpy()
+        s = O.indexer_scores(qI[None], w[None], kI, [ne])
+        ridx = O.topk_select(s, [ne], k)[0]
+        gidx = idx[b, 0].cpu().numpy()
+        if grid:
+            assert np.array_equal(gidx, ridx)
+        else:
+            kth = np.sort(s[0])[::-1][k - 1]
+            bound = 1e-5 * (np.abs(w)[:, None] * np.abs(qI @ kI.T)).sum(axis=0).max()
+            for e in set(gidx.tolist()) ^ set(ridx.tolist()):
+                assert abs(s[0, e] - kth) <= bound
+            if not np.array_equal(gidx, ridx):
+                continue
+        # dequantise only the selected rows: the attention reads nothing else
+        kv = np.zeros((ne, D))
+        sel = ridx[ridx >= 0]
+        kv[sel, :D - 64] = O.e4m3_decode(inp["kv_nope"][b][torch.from_numpy(sel).cuda()].cpu().numpy()) * \
+            inp["kv_scale"][b][torch.from_numpy(sel).cuda()].cpu().numpy()[:, None]
+        kv[sel, D - 64:] = inp["kv_rope"][b][torch.from_numpy(sel).cuda()].float().cpu().numpy()
+        q = inp["q"][b, 0].float().cpu().numpy()
+        ref, _ = O.csa_decode(q, qI, w, kI, kv, inp["swa"][b].float().cpu().numpy(), inp["sink"].cpu().numpy(),
+                              t, k=k, m=4, inv_rope=True)
+        assert_close(host(out)[b, 0], ref, what=f"decode 1M b={b}")
