@@ -158,6 +158,9 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None):
     ws = torch.empty(csa.csa_index_topk_workspace(Bn, 1, ne, k), dtype=torch.uint8, device=dev)
     idx = torch.empty(Bn, 1, k, dtype=torch.int32, device=dev)
     out = torch.empty(Bn, 1, H, D, dtype=torch.bfloat16, device=dev)
+    # split each token's 5 chunks (4 x 128 selected entries + the window) over CTAs
+    n_split = max(1, min(5, csa.num_sms() // Bn))
+    aws = torch.empty(csa.csa_fused_attention_workspace(Bn, 1, H, D, n_split), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
@@ -169,7 +172,7 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None):
             ev[1].record(stream)
         csa.csa_fused_attention(inp["q"], inp["kv_nope"], inp["swa"], inp["q_pos"], W, inp["sink"], idx=idx,
                                 kv_rope=inp["kv_rope"], kv_scale=inp["kv_scale"], window_mode=1, inv_rope=True,
-                                rope_dim=64, out=out)
+                                rope_dim=64, out=out, n_split=n_split, workspace=aws)
         if ev is not None:
             ev[2].record(stream)
 
@@ -195,7 +198,7 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None):
     algo = scan + gather + swa + qbytes
     hbm, _, _, src = _peaks()
     ach_idx = scan / (t_idx * 1e-3) / 1e9
-    return {"workload": "csa_decode_1m", "batch": Bn, "context": cfg["ctx"], "entries": ne, "top_k": k,
+    return {"workload": "csa_decode_1m", "batch": Bn, "attention_splits": n_split, "context": cfg["ctx"], "entries": ne, "top_k": k,
             "tokens_per_s": Bn / (ms * 1e-3), "ms_per_step": ms, "kernels_ms": {"index_topk": t_idx,
                                                                                  "fused_attention": t_att},
             "algorithmic_bytes_per_step": algo,

@@ -231,6 +231,25 @@ csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, const void*
                                  int D, int rope_dim, float rope_base, int inv_rope, float scale,
                                  void* out, csa_dtype_t out_dtype, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * csa_fused_attention_splitkv — csa_fused_attention with each query token's
+ * row set split into n_split consecutive chunk ranges processed in parallel
+ * (more CTAs when there are few query tokens, e.g. decode), followed by a merge
+ * of the n_split partial results and the sink in one softmax and the optional
+ * inverse RoPE.  Same result as csa_fused_attention up to rounding.
+ *   n_split in [1, 16]; workspace of csa_fused_attention_workspace(n_seq, T, H, D,
+ *   n_split) bytes (partials: fp32 [n_seq*T*n_split, H, D] + lse).
+ * ------------------------------------------------------------------------- */
+size_t csa_fused_attention_workspace(int n_seq, int T, int H, int D, int n_split);
+csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q_dtype, const void* kv, csa_dtype_t kv_dtype,
+                                         const void* kv_rope, const float* kv_scale, int64_t cap,
+                                         const int32_t* idx, int k, int m, const void* kv_tok,
+                                         csa_dtype_t tok_dtype, int64_t tok_cap, int W, int window_mode,
+                                         const int64_t* q_pos, const float* sink, int n_seq, int T, int H,
+                                         int D, int rope_dim, float rope_base, int inv_rope, float scale,
+                                         int n_split, void* workspace, size_t ws_bytes, void* out,
+                                         csa_dtype_t out_dtype, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

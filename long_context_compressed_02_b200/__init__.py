@@ -55,6 +55,9 @@ def lib():
         "csa_fused_attention": ([P, I, P, I, P, P, I64, P, I, I, P, I, I64, I, I, P, P, I, I, I, I, I, F, I, F,
                                  P, I, P], I),
         "csa_index_topk_noalloc": ([P, P, P, P, P, P, I, I, I, I, I64, I, I, P, P], I),
+        "csa_fused_attention_workspace": ([I, I, I, I, I], SZ),
+        "csa_fused_attention_splitkv": ([P, I, P, I, P, P, I64, P, I, I, P, I, I64, I, I, P, P, I, I, I, I, I, F, I, F,
+                                         I, P, SZ, P, I, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -86,6 +89,15 @@ def _dev(t, name):
         raise CsaError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise CsaError(f"{name} must be contiguous")
+
+
+def num_sms(device=None):
+    """Streaming multiprocessors of the current (or given) CUDA device."""
+    return torch.cuda.get_device_properties(torch.cuda.current_device() if device is None else device).multi_processor_count
+
+
+def csa_fused_attention_workspace(n_seq, T, H, D, n_split):
+    return int(lib().csa_fused_attention_workspace(n_seq, T, H, D, n_split))
 
 
 def check_device_error(stream=None):
@@ -210,7 +222,7 @@ def swa_sink_combine(q, kv_tok, q_pos, W, sink, O_part=None, lse_part=None, *, w
 
 def csa_fused_attention(q, kv, kv_tok, q_pos, W, sink, *, idx=None, m=1, kv_rope=None, kv_scale=None,
                         window_mode=0, inv_rope=False, rope_dim=None, rope_base=10000.0, scale=None,
-                        out_dtype=None, out=None, stream=None):
+                        out_dtype=None, out=None, n_split=1, workspace=None, stream=None):
     """Compressed rows (idx given: gathered top-k entries; else the dense prefix
     of complete m-entries) + raw window rows + sink in one softmax, then the
     optional inverse RoPE.  q [n_seq, T, H, D]; kv [n_seq, cap, D] (or e4m3 +
@@ -226,6 +238,16 @@ def csa_fused_attention(q, kv, kv_tok, q_pos, W, sink, *, idx=None, m=1, kv_rope
         out = torch.empty((n_seq, T, H, D), dtype=out_dtype, device=q.device)
     k = 0 if idx is None else idx.shape[-1]
     kvd, kvp, kvr, kvs = _kv_args(kv, kv_rope, kv_scale)
+    if n_split > 1:
+        need = int(lib().csa_fused_attention_workspace(n_seq, T, H, D, n_split))
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        _check(lib().csa_fused_attention_splitkv(
+            _ptr(q), _DT[q.dtype], kvp, kvd, kvr, kvs, kv.shape[1], _ptr(idx), k, m, _ptr(kv_tok), _DT[kv_tok.dtype],
+            kv_tok.shape[1], W, window_mode, _ptr(q_pos), _ptr(sink), n_seq, T, H, D, rope_dim, rope_base,
+            int(inv_rope), scale, n_split, _ptr(workspace), workspace.numel(), _ptr(out), _DT[out.dtype],
+            _stream(stream)), "csa_fused_attention_splitkv")
+        return out
     _check(lib().csa_fused_attention(_ptr(q), _DT[q.dtype], kvp, kvd, kvr, kvs, kv.shape[1], _ptr(idx), k, m,
                                      _ptr(kv_tok), _DT[kv_tok.dtype], kv_tok.shape[1], W, window_mode, _ptr(q_pos),
                                      _ptr(sink), n_seq, T, H, D, rope_dim, rope_base, int(inv_rope), scale,

@@ -92,6 +92,7 @@ struct AttnParams {
   int out_bf16, inv_rope, rope_dim;
   float rope_base;
   int tma_q, tma_kv, tma_tok;   // TMA tile loads for bf16 queries / dense entries / window rows
+  int n_split;                  // chunk-range splits per query token (partials merged afterwards)
 };
 
 // Chunk order: the window rows (source 2) come first, so that they start on a
@@ -100,6 +101,7 @@ struct AttnParams {
 struct RowSet {
   int n1, n2, n;            // rows from source 1, source 2, total
   int nc2, nchunks;         // window chunks, all chunks
+  int c0, c1;               // chunk range of this work item (split-KV)
   int64_t lo2;              // first window row
   const int32_t* idx;       // gather list (source 1)
 };
@@ -123,8 +125,8 @@ __device__ __forceinline__ int count_valid_warp(const int32_t* row, int k, int l
 }
 
 // Whole-warp call: every lane gets the same row set.
-__device__ __forceinline__ RowSet row_set_warp(const AttnParams& p, int b, int t, int lane) {
-  RowSet r{0, 0, 0, 0, 0, 0, nullptr};
+__device__ __forceinline__ RowSet row_set_warp(const AttnParams& p, int b, int t, int sp, int lane) {
+  RowSet r{0, 0, 0, 0, 0, 0, 0, 0, nullptr};
   const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
   if (p.src1 == SRC1_GATHER) {
     r.idx = p.idx + ((int64_t)b * p.T + t) * p.k;
@@ -143,6 +145,9 @@ __device__ __forceinline__ RowSet row_set_warp(const AttnParams& p, int b, int t
   r.n = r.n1 + r.n2;
   r.nc2 = (r.n2 + kRows - 1) / kRows;
   r.nchunks = r.nc2 + (r.n1 + kRows - 1) / kRows;
+  const int per = (r.nchunks + p.n_split - 1) / p.n_split;
+  r.c0 = min(r.nchunks, sp * per);
+  r.c1 = min(r.nchunks, r.c0 + per);
   return r;
 }
 
@@ -368,7 +373,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   volatile int* abort_flag = s_abort;
-  const int64_t n_items = (int64_t)p.n_seq * p.T;
+  const int64_t n_items = (int64_t)p.n_seq * p.T * p.n_split;
 
   if (warp >= 4 && warp < 8) {
     // ============================ loaders
@@ -376,9 +381,11 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
     uint32_t g = 0, qcount = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int b = (int)(item / p.T), t = (int)(item % p.T);
-      const RowSet rs = row_set_warp(p, b, t, lane);
-      if (rs.n == 0) continue;
+      const int64_t bt = item / p.n_split;
+      const int sp = (int)(item % p.n_split);
+      const int b = (int)(bt / p.T), t = (int)(bt % p.T);
+      const RowSet rs = row_set_warp(p, b, t, sp, lane);
+      if (rs.c1 <= rs.c0) continue;
       // ---- Q tile: 64 rows x NS slabs of 128 B
       if (!wait_bar(q_free, (qcount & 1) ^ 1, abort_flag)) { ok = false; break; }
       ++qcount;
@@ -429,7 +436,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
         mbar_arrive(q_full);
       }
       // ---- KV chunks
-      for (int c = 0; c < rs.nchunks && ok; ++c, ++g) {
+      for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
         const bool win = c < rs.nc2;                   // window chunk (source 2)
         const int cl = win ? c : c - rs.nc2;
         const int r = cl * kRows + lt;
@@ -472,6 +479,53 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
             }
           }
           continue;
+        }
+        if constexpr (KV == KV_FP8) {
+          if (!win) {
+            // e4m3 rows: the raw bytes of the row (nope part + bf16 RoPE part + scale)
+            // are fetched in two batches well ahead of use, then converted slab by slab
+            const int nope = D - p.rope_dim;            // rope_dim == 64
+            const uint4* srcn = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.kv) +
+                                                               ((int64_t)b * p.cap + row) * nope);
+            const uint4* srcr = reinterpret_cast<const uint4*>(p.kv_rope + ((int64_t)b * p.cap + row) * p.rope_dim);
+            const float sc = valid ? __ldg(p.kv_scale + (int64_t)b * p.cap + row) : 0.f;
+            constexpr int kNopeV = (D - 64) / 16;       // 16-byte vectors of e4m3 per row
+            constexpr int kHalf = (NS / 2) * 4;         // vectors of the first half of the slabs
+            uint4 raw[kNopeV];
+#pragma unroll
+            for (int i = 0; i < kHalf && i < kNopeV; ++i) raw[i] = valid ? __ldg(srcn + i) : make_uint4(0, 0, 0, 0);
+            uint4 rp[8];
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) {
+              if (!wait_bar(&pv_done[tt], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
+              if (tt == 0) {
+#pragma unroll
+                for (int i = kHalf; i < kNopeV; ++i) raw[i] = valid ? __ldg(srcn + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) rp[i] = valid ? __ldg(srcr + i) : make_uint4(0, 0, 0, 0);
+              }
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int sl = 2 * tt + h;
+                uint8_t* dst = sKV + sl * kKSlab;
+                if (64 * sl < nope) {
+#pragma unroll
+                  for (int q4 = 0; q4 < 4; ++q4) {
+                    float v[16];
+                    e4m3x16_to_float(raw[(4 * sl + q4) % kNopeV], sc, v);
+                    st_shared16(dst + swz128(lt, 2 * q4), to_bf16x8(v));
+                    st_shared16(dst + swz128(lt, 2 * q4 + 1), to_bf16x8(v + 8));
+                  }
+                } else {
+#pragma unroll
+                  for (int q = 0; q < 8; ++q) st_shared16(dst + swz128(lt, q), rp[q]);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&kv_full[sl]);
+              }
+            }
+            continue;
+          }
         }
         // every slab pair is issued as soon as the PV tile that read it retires;
         // completions are then retired in order (cp.async groups, one per slab)
@@ -518,14 +572,15 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
     uint32_t g = 0, qcount = 0, icount = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int b = (int)(item / p.T), t = (int)(item % p.T);
-      const RowSet rs = row_set_warp(p, b, t, lane);
-      if (rs.n == 0) continue;
+      const int64_t bt = item / p.n_split;
+      const int sp = (int)(item % p.n_split);
+      const int b = (int)(bt / p.T), t = (int)(bt % p.T);
+      const RowSet rs = row_set_warp(p, b, t, sp, lane);
+      if (rs.c1 <= rs.c0) continue;
       if (lane == 0) {
         if (!wait_bar(q_full, qcount & 1, abort_flag)) ok = false;
         ++qcount;
-        const int n_chunks = rs.nchunks;
-        for (int c = 0; c < n_chunks && ok; ++c, ++g) {
+        for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
 #pragma unroll 1
           for (int s = 0; s < NS; ++s) {
             if (!wait_bar(&kv_full[s], g & 1, abort_flag)) { ok = false; break; }
@@ -537,11 +592,11 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
           }
           if (!ok) break;
           mma_commit(s_done);
-          if (c == n_chunks - 1) mma_commit(q_free);
+          if (c == rs.c1 - 1) mma_commit(q_free);
           if (!wait_bar(p_full, g & 1, abort_flag)) { ok = false; break; }
-          if (c == 0 && !wait_bar(epi_done, (icount & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (c == rs.c0 && !wait_bar(epi_done, (icount & 1) ^ 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t acc0 = c > 0 ? 1u : 0u;
+          const uint32_t acc0 = c > rs.c0 ? 1u : 0u;
 #pragma unroll 1
           for (int tt = 0; tt < NT; ++tt) {
 #pragma unroll
@@ -564,8 +619,10 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
     uint32_t g = 0, icount = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int b = (int)(item / p.T), t = (int)(item % p.T);
-      const RowSet rs = row_set_warp(p, b, t, lane);
+      const int64_t bt = item / p.n_split;
+      const int sp = (int)(item % p.n_split);
+      const int b = (int)(bt / p.T), t = (int)(bt % p.T);
+      const RowSet rs = row_set_warp(p, b, t, sp, lane);
       const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
       float2* cs = s_cs + (icount & 1) * 32;
       if (EPI == EPI_COMBINE && p.inv_rope && tid < 32) {
@@ -578,8 +635,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
       }
       float m_own[2] = {-CUDART_INF_F, -CUDART_INF_F};   // running max of columns lane, 32 + lane
       float l_own[2] = {0.f, 0.f};
-      const int n_chunks = rs.nchunks;
-      for (int c = 0; c < n_chunks && ok; ++c, ++g) {
+      for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
         if (!wait_bar(s_done, g & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         float x[64];
@@ -620,7 +676,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
           float mx = fmaxf(fmaxf(red[col], red[64 + col]), fmaxf(red[128 + col], red[192 + col])) * p.scale_log2;
           float mn = (mx > m_own[h] + kTau) ? mx : m_own[h];
           alpha[h] = exp2f(m_own[h] - mn);             // 0 on the first chunk
-          if (mn != m_own[h] && c > 0) need_rescale = true;
+          if (mn != m_own[h] && c > rs.c0) need_rescale = true;
           m_own[h] = mn;
           bc_m[col] = mn;
           bc_m[64 + col] = alpha[h];
@@ -691,7 +747,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
         float cw, cp = 0.f;
         if (EPI == EPI_PARTIAL) {
           cw = lt > 0.f ? 1.f / lt : 0.f;
-          if (warp == 0 && col < p.H) p.lse_part[((int64_t)b * p.T + t) * p.H + col] = lse_w;
+          if (warp == 0 && col < p.H) p.lse_part[(bt * p.n_split + sp) * p.H + col] = lse_w;
         } else {
           const int64_t o = ((int64_t)b * p.T + t) * p.H + (col < p.H ? col : 0);
           const float lse_p = (p.O_in && col < p.H) ? p.lse_in[o] : -CUDART_INF_F;
@@ -707,13 +763,13 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
         bc_m[128 + col] = cp;
       }
       __syncwarp();
-      if (rs.n > 0) {
+      if (rs.c1 > rs.c0) {
         for (int tt = 0; tt < NT; ++tt)
           if (!wait_bar(&pv_done[tt], (g - 1) & 1, abort_flag)) { ok = false; break; }
         if (!ok) break;
         tc_fence_after();
       }
-      const int64_t obase = ((int64_t)b * p.T + t) * p.H;
+      const int64_t obase = (bt * p.n_split + sp) * p.H;   // n_split = 1: token row
       // Each 128-d tile is written in two halves of 32 heads.  Phase A: every
       // thread (one TMEM lane = one d) scales its accumulators and stages them
       // as fp32 [32 heads][128 d] in sP (free once the last PV retired).
@@ -726,7 +782,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
           float o[32];
-          if (rs.n > 0) {
+          if (rs.c1 > rs.c0) {
             tmem_ld16(tmem + lane_base + 64 + 64 * tt + 32 * hh, o);
             tmem_ld16(tmem + lane_base + 64 + 64 * tt + 32 * hh + 16, o + 16);
             tmem_wait_ld();
@@ -799,7 +855,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
           named_bar_sync(2, 128);   // staging buffer reused by the next half
         }
       }
-      if (rs.n > 0) {
+      if (rs.c1 > rs.c0) {
         tc_fence_before();
         mbar_arrive(epi_done);
         ++icount;
@@ -819,6 +875,84 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
   }
 }
 
+// Split-KV merge: each token's n_split partials (O normalised by its own sum,
+// lse) and the sink in one softmax, then the inverse RoPE of the output.
+// One CTA per token; 16-byte vector loads and stores along d.
+__global__ void __launch_bounds__(256)
+attn_merge_kernel(const float* __restrict__ Os, const float* __restrict__ Ls, const float* __restrict__ sink,
+                  const int64_t* __restrict__ q_pos, int T, int n_split, int H, int D, int inv_rope, int rope_dim,
+                  float rope_base, void* __restrict__ out, int out_bf16) {
+  constexpr int kHeads = 8;                       // heads per CTA (blockIdx.y selects the group)
+  __shared__ float s_coef[kHeads][16];
+  __shared__ float2 s_cs[32];
+  const int64_t bt = blockIdx.x;
+  const int h0 = blockIdx.y * kHeads;
+  const int b = (int)(bt / T), t = (int)(bt % T);
+  const int64_t pos = (q_pos ? q_pos[b] : 0) + t;
+  const int tid = threadIdx.x;
+  if (tid < kHeads && h0 + tid < H) {
+    const int h = h0 + tid;
+    float M = sink ? sink[h] : -CUDART_INF_F;
+    for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, Ls[(bt * n_split + sp) * H + h]);
+    if (M == -CUDART_INF_F) M = 0.f;
+    float den = sink ? __expf(sink[h] - M) : 0.f;
+    for (int sp = 0; sp < n_split; ++sp) den += __expf(Ls[(bt * n_split + sp) * H + h] - M);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int sp = 0; sp < n_split; ++sp) s_coef[tid][sp] = __expf(Ls[(bt * n_split + sp) * H + h] - M) * inv;
+  }
+  const int half = rope_dim / 2;
+  if (inv_rope && tid >= 32 && tid < 32 + half) {
+    const int j = tid - 32;
+    double inv_freq = exp(-2.0 * (double)j / (double)rope_dim * log((double)rope_base));
+    double ang = fmod((double)pos * inv_freq, 6.283185307179586476925286766559);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    s_cs[j] = make_float2((float)cd, (float)sd);
+  }
+  __syncthreads();
+  const int r0 = D - rope_dim;
+  const int per_row = D / 8;
+  const int nh = min(kHeads, H - h0);
+  for (int idx = tid; idx < nh * per_row; idx += blockDim.x) {
+    const int hl = idx / per_row, h = h0 + hl, d0 = (idx % per_row) * 8;
+    float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const bool rot = inv_rope && d0 >= r0;
+    const bool first = d0 < r0 + half;
+    const int pd = first ? d0 + half : d0 - half;
+    for (int sp = 0; sp < n_split; ++sp) {
+      const float c = s_coef[hl][sp];
+      const float* src = Os + ((bt * n_split + sp) * H + h) * (int64_t)D;
+      const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + d0));
+      const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + d0) + 1);
+      v[0] += c * a0.x; v[1] += c * a0.y; v[2] += c * a0.z; v[3] += c * a0.w;
+      v[4] += c * a1.x; v[5] += c * a1.y; v[6] += c * a1.z; v[7] += c * a1.w;
+      if (rot) {
+        const float4 b0 = __ldg(reinterpret_cast<const float4*>(src + pd));
+        const float4 b1 = __ldg(reinterpret_cast<const float4*>(src + pd) + 1);
+        w[0] += c * b0.x; w[1] += c * b0.y; w[2] += c * b0.z; w[3] += c * b0.w;
+        w[4] += c * b1.x; w[5] += c * b1.y; w[6] += c * b1.z; w[7] += c * b1.w;
+      }
+    }
+    if (rot) {
+      const int jj0 = d0 - r0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // inverse rotation by -pos: (a, b) -> (a cos + b sin, -a sin + b cos)
+        const float2 cs = s_cs[(jj0 + i) % half];
+        v[i] = first ? v[i] * cs.x + w[i] * cs.y : v[i] * cs.x - w[i] * cs.y;
+      }
+    }
+    const int64_t o = (bt * H + h) * (int64_t)D + d0;
+    if (out_bf16) {
+      *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + o) = to_bf16x8(v);
+    } else {
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + o);
+      dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+      dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+}
+
 struct AttnMaps {
   CUtensorMap q, kv, tok;
 };
@@ -831,7 +965,7 @@ csa_status_t launch_attn(const AttnParams& p, const AttnMaps& m, cudaStream_t st
   auto kern = attn_kernel<D, KV, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attention: cannot reserve %zu bytes of shared memory: %s", smem, cudaGetErrorString(e));
-  const int64_t items = (int64_t)p.n_seq * p.T;
+  const int64_t items = (int64_t)p.n_seq * p.T * p.n_split;
   if (items == 0) return CSA_OK;
   const int grid = (int)std::min<int64_t>(items, num_sms());
   kern<<<grid, kThreads, smem, st>>>(p, m.q, m.kv, m.tok);
@@ -867,6 +1001,7 @@ csa_status_t build_maps(AttnParams& p, AttnMaps& m, int D, csa_dtype_t q_dtype, 
 template <int EPI>
 csa_status_t dispatch(AttnParams& p, int D, csa_dtype_t q_dtype, csa_dtype_t kv_dtype, csa_dtype_t tok_dtype,
                       cudaStream_t st) {
+  if (p.n_split < 1) p.n_split = 1;
   AttnMaps m;
   csa_status_t s = build_maps(p, m, D, q_dtype, kv_dtype, tok_dtype);
   if (s != CSA_OK) return s;
@@ -991,4 +1126,55 @@ extern "C" csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, 
   p.sink = sink; p.out = out; p.out_bf16 = out_dtype == CSA_BF16;
   p.inv_rope = inv_rope; p.rope_dim = rope_dim; p.rope_base = rope_base;
   return dispatch<EPI_COMBINE>(p, D, q_dtype, kv_dtype, tok_dtype, stream);
+}
+
+extern "C" size_t csa_fused_attention_workspace(int n_seq, int T, int H, int D, int n_split) {
+  if (n_seq <= 0 || T <= 0 || H <= 0 || D <= 0 || n_split <= 0) return 0;
+  const size_t parts = (size_t)n_seq * T * n_split * H;
+  return ((parts * D * 4 + 255) / 256) * 256 + parts * 4;
+}
+
+extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q_dtype, const void* kv,
+                                                    csa_dtype_t kv_dtype, const void* kv_rope, const float* kv_scale,
+                                                    int64_t cap, const int32_t* idx, int k, int m, const void* kv_tok,
+                                                    csa_dtype_t tok_dtype, int64_t tok_cap, int W, int window_mode,
+                                                    const int64_t* q_pos, const float* sink, int n_seq, int T, int H,
+                                                    int D, int rope_dim, float rope_base, int inv_rope, float scale,
+                                                    int n_split, void* workspace, size_t ws_bytes, void* out,
+                                                    csa_dtype_t out_dtype, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(n_split >= 1 && n_split <= 16, "csa_fused_attention_splitkv: n_split must be in [1, 16]");
+  csa_status_t s = check_common("csa_fused_attention_splitkv", q, q_dtype, kv, kv_dtype, kv_rope, kv_scale, cap,
+                                n_seq, T, H, D, rope_dim);
+  if (s != CSA_OK) return s;
+  CSA_REQUIRE(q_pos && aligned16(q_pos), "csa_fused_attention_splitkv: q_pos required");
+  CSA_REQUIRE(idx ? (k >= 1 && aligned16(idx)) : m >= 1, "csa_fused_attention_splitkv: need idx with k >= 1, or m >= 1");
+  CSA_REQUIRE(kv_tok && aligned16(kv_tok) && tok_cap >= 1 && W >= 1, "csa_fused_attention_splitkv: kv_tok, tok_cap, W");
+  CSA_REQUIRE(tok_dtype == (kv_dtype == CSA_F32 ? CSA_F32 : CSA_BF16),
+              "csa_fused_attention_splitkv: window rows must be f32 with an f32 store and bf16 otherwise");
+  CSA_REQUIRE(window_mode == 0 || window_mode == 1, "csa_fused_attention_splitkv: window_mode must be 0 or 1");
+  CSA_REQUIRE(!inv_rope || rope_dim == 64, "csa_fused_attention_splitkv: inv_rope needs rope_dim 64");
+  CSA_REQUIRE(out && aligned16(out) && (out_dtype == CSA_F32 || out_dtype == CSA_BF16), "csa_fused_attention_splitkv: bad out");
+  const size_t need = csa_fused_attention_workspace(n_seq, T, H, D, n_split);
+  if (!workspace || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "csa_fused_attention_splitkv: workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  CSA_REQUIRE(aligned16(workspace), "csa_fused_attention_splitkv: workspace must be 16-byte aligned");
+  const size_t parts = (size_t)n_seq * T * n_split * H;
+  float* Os = static_cast<float*>(workspace);
+  float* Ls = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((parts * D * 4 + 255) / 256) * 256);
+  AttnParams p{};
+  p.q = q; p.q_f32 = q_dtype == CSA_F32; p.q_pos = q_pos;
+  p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale; p.cap = cap;
+  p.src1 = idx ? SRC1_GATHER : SRC1_DENSE; p.idx = idx; p.k = k; p.m = m;
+  p.kv2 = kv_tok; p.cap2 = tok_cap; p.src2 = window_mode == 0 ? SRC2_WINDOW : SRC2_CACHE; p.W = W;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.O_part = Os; p.lse_part = Ls; p.rope_dim = rope_dim; p.n_split = n_split;
+  s = dispatch<EPI_PARTIAL>(p, D, q_dtype, kv_dtype, tok_dtype, stream);
+  if (s != CSA_OK) return s;
+  const int64_t toks = (int64_t)n_seq * T;
+  if (toks == 0) return CSA_OK;
+  CSA_REQUIRE(toks <= 0x7fffffff, "csa_fused_attention_splitkv: too many tokens");
+  attn_merge_kernel<<<dim3((unsigned)toks, (unsigned)((H + 7) / 8)), 256, 0, stream>>>(
+      Os, Ls, sink, q_pos, T, n_split, H, D, inv_rope, rope_dim, rope_base, out, out_dtype == CSA_BF16);
+  return check_launch("csa_fused_attention_splitkv(merge)");
 }

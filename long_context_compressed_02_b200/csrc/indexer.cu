@@ -128,7 +128,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   const uint32_t tmem_cols = p.N <= 16 ? 32u : (p.N <= 32 ? 64u : (p.N <= 64 ? 128u : (p.N <= 128 ? 256u : 512u)));
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiThreads); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiThreads / 2); }
     mbar_init(qbar, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -176,7 +176,10 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     // ---------------- MMA issuer (lane 0)
     if (lane == 0) {
       const uint32_t idesc = make_idesc(128, p.N, 0, 0, 0, 0);
-      const uint32_t sB_addr = smem_u32(sB), sA_addr = smem_u32(sA);
+      // base descriptors once; each MMA only adds a start-address offset (>> 4)
+      const uint64_t dA = smem_desc(smem_u32(sA), 16, sbo, swz);
+      const uint64_t dB = smem_desc(smem_u32(sB), 16, sbo, swz);
+      const int nk = p.DI / 32;
       if (wait_bar(qbar, 0, abort_flag)) {
         for (int it = 0; it < n_tiles; ++it) {
           const int s = it % kStages;
@@ -186,10 +189,13 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
           if (!wait_bar(&full[s], ph, abort_flag)) break;
           if (!wait_bar(&tempty[acc], aph ^ 1, abort_flag)) break;
           tc_fence_after();
-          for (int kk = 0; kk < p.DI / 32; ++kk) {
-            uint64_t ad = smem_desc(sA_addr + s * a_bytes + kk * 32, 16, sbo, swz);
-            uint64_t bd = smem_desc(sB_addr + kk * 32, 16, sbo, swz);
-            mma_f8(tmem + acc * p.N, ad, bd, idesc, kk > 0);
+          const uint64_t dAs = dA + ((s * a_bytes) >> 4);
+          const uint32_t d = tmem + acc * p.N;
+          mma_f8(d, dAs, dB, idesc, 0);
+          if (nk > 1) mma_f8(d, dAs + 2, dB + 2, idesc, 1);
+          if (nk > 2) {
+            mma_f8(d, dAs + 4, dB + 4, idesc, 1);
+            mma_f8(d, dAs + 6, dB + 6, idesc, 1);
           }
           mma_commit(&empty[s]);
           mma_commit(&tfull[acc]);
@@ -197,15 +203,12 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       }
     }
   } else {
-    // ---------------- epilogue: 8 warps, two per TMEM sub-partition; each
-    // thread owns one key (TMEM lane) and half of the token columns (all of
-    // them when the block holds a single token).
+    // ---------------- epilogue: 8 warps in two groups of four; group h owns
+    // TMEM accumulator h and therefore every other tile, so two tiles'
+    // epilogues run at once.  Each thread owns one key (TMEM lane) of a tile.
     const int ew = warp - 2;
     const int sp = warp & 3;
-    const int half = ew >> 2;
-    const bool split = p.TQ >= 2 && p.N >= 64;
-    const int c_begin = split ? half * (p.N >> 1) : 0;
-    const int c_end = split ? c_begin + (p.N >> 1) : (half == 0 ? p.N : 0);
+    const int grp = ew >> 2;
     const int log2hi = __ffs(p.HI) - 1;
     const uint32_t w_addr = smem_u32(s_w);
     const int key_in_tile = sp * 32 + lane;
@@ -213,18 +216,18 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       const int64_t key = (int64_t)(tile0 + it) * 128 + key_in_tile;
       return (key < p.cap && it < n_tiles) ? (p.ks ? __ldg(p.ks + (int64_t)b * p.cap + key) : 1.f) : 0.f;
     };
-    float ksc_next = key_scale(0);
-    for (int it = 0; it < n_tiles; ++it) {
-      const int acc = it & 1;
+    float ksc_next = key_scale(grp);
+    for (int it = grp; it < n_tiles; it += 2) {
+      const int acc = grp;
       const uint32_t aph = (it >> 1) & 1;
       const int64_t key = (int64_t)(tile0 + it) * 128 + key_in_tile;
       const float ksc = ksc_next;
-      ksc_next = key_scale(it + 1);          // issued a tile ahead: off the critical path
+      ksc_next = key_scale(it + 2);          // issued a tile ahead: off the critical path
       if (!wait_bar(&tfull[acc], aph, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N;
       float run = 0.f;
-      for (int cc = c_begin; cc < c_end; cc += 32) {
+      for (int cc = 0; cc < p.N; cc += 32) {
         float v[32];
         tmem_ld32(tb + cc, v);
         tmem_wait_ld();
@@ -288,6 +291,7 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 struct SelectSmem {
   uint32_t whist[kTopkThreads / 32][256];
+  uint32_t wlo[kTopkThreads / 32], whi[kTopkThreads / 32];
   uint32_t hist[256];
   uint64_t warp_tot[kTopkThreads / 32];
   uint32_t digit, above;
@@ -319,16 +323,34 @@ __device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id
   int need_eq = 0;
   const bool all = n <= k;
   if (!all) {
-    uint32_t prefix = 0, mask = 0;
+    // Bits above the highest bit in which the row's keys differ are common to
+    // every key: the 8-bit digits start just below them, so the first histogram
+    // spreads over the data instead of piling onto one bin.
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int e = tid; e < n; e += kTopkThreads) { const uint32_t key = keys[e]; lo = min(lo, key); hi = max(hi, key); }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if ((tid & 31) == 0) { ss.wlo[tid >> 5] = lo; ss.whi[tid >> 5] = hi; }
+    __syncthreads();
+    lo = ss.wlo[0]; hi = ss.whi[0];
+    for (int w = 1; w < kTopkThreads / 32; ++w) { lo = min(lo, ss.wlo[w]); hi = max(hi, ss.whi[w]); }
+    const uint32_t diff = lo ^ hi;
+    const int top = diff ? 31 - __clz(diff) : -1;           // highest differing bit
+    uint32_t mask = top >= 31 ? 0u : ~((2u << top) - 1u);   // common high bits
+    uint32_t prefix = hi & mask;
     int remaining = k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int shift = top - 7; shift > -8; shift -= 8) {
+      const int sh = max(shift, 0);
+      const uint32_t dmask = shift >= 0 ? 255u : (255u >> (-shift));   // width of this digit
       for (int i = tid; i < 256 * (kTopkThreads / 32); i += kTopkThreads) (&ss.whist[0][0])[i] = 0;
       __syncthreads();
-      // per-warp private histograms: scores share their top bits, so a single
-      // histogram would serialise every warp on one bin
+      // per-warp private histograms
       for (int e = tid; e < n; e += kTopkThreads) {
         const uint32_t key = keys[e];
-        if ((key & mask) == prefix) atomicAdd(&ss.whist[tid >> 5][(key >> shift) & 255u], 1u);
+        if ((key & mask) == prefix) atomicAdd(&ss.whist[tid >> 5][(key >> sh) & dmask], 1u);
       }
       __syncthreads();
       for (int i = tid; i < 256; i += kTopkThreads) {
@@ -360,11 +382,12 @@ __device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id
         }
       }
       __syncthreads();
-      prefix |= ss.digit << shift;
-      mask |= 255u << shift;
+      prefix |= ss.digit << sh;
+      mask |= dmask << sh;
       remaining -= (int)ss.above;
       __syncthreads();
     }
+    if (top < 0) prefix = hi;                                // every key equal
     T = prefix;
     need_eq = remaining;
   }

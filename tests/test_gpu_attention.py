@@ -150,7 +150,8 @@ def _dequant(cache):
                            cache["kv_rope"].float().cpu().numpy()], axis=1)
 
 
-def test_fused_csa_decode_e4m3_caches():
+@pytest.mark.parametrize("n_split", [1, 3, 16])
+def test_fused_csa_decode_e4m3_caches(n_split):
     """Decode: top-k entries from an e4m3 + bf16-RoPE cache, the 128-row SWA
     cache and the sink in one softmax, inverse RoPE at the query position."""
     import long_context_compressed_02_b200 as csa
@@ -171,7 +172,7 @@ def test_fused_csa_decode_e4m3_caches():
         idx[b, 0, :n] = np.sort(rng.choice(nv, n, replace=False)) if nv else []
     out = csa.csa_fused_attention(cuda(q, torch.bfloat16), kv_nope, cuda(swa, torch.bfloat16), cuda(pos), W,
                                   cuda(sink), idx=cuda(idx), kv_rope=kv_rope, kv_scale=kv_scale, window_mode=1,
-                                  inv_rope=True, rope_dim=64, out_dtype=torch.float32)
+                                  inv_rope=True, rope_dim=64, out_dtype=torch.float32, n_split=n_split)
     csa.check_device_error()
     for b in range(n_seq):
         kv = _dequant(caches[b])
@@ -181,7 +182,8 @@ def test_fused_csa_decode_e4m3_caches():
         assert_close(host(out)[b], ref, what=f"fused CSA decode b={b}")
 
 
-def test_fused_hca_decode_e4m3_dense():
+@pytest.mark.parametrize("n_split", [1, 4])
+def test_fused_hca_decode_e4m3_dense(n_split):
     import long_context_compressed_02_b200 as csa
     rng = np.random.default_rng(22)
     gen = torch.Generator(device="cuda").manual_seed(22)
@@ -195,7 +197,7 @@ def test_fused_hca_decode_e4m3_dense():
     pos = np.array([128 * 700 - 1, 130, 128 * 333 + 17], np.int64)
     out = csa.csa_fused_attention(cuda(q, torch.bfloat16), kv_nope, cuda(swa, torch.bfloat16), cuda(pos), W,
                                   cuda(sink), m=m, kv_rope=kv_rope, kv_scale=kv_scale, window_mode=1,
-                                  inv_rope=True, rope_dim=64, out_dtype=torch.float32)
+                                  inv_rope=True, rope_dim=64, out_dtype=torch.float32, n_split=n_split)
     csa.check_device_error()
     for b in range(n_seq):
         kv = _dequant(caches[b])
@@ -219,3 +221,22 @@ def test_fused_equals_separate_calls():
     csa.check_device_error()
     # both paths are bf16-probability approximations of the same softmax: the benchmark spec tolerance
     assert_close(host(fus), host(sep), what="fused vs separate")
+
+
+def test_split_kv_prefill_matches_oracle():
+    """Split-KV over bf16 prefill rows (window first, then gathered entries)."""
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(24)
+    S, ne, H, D, k, W = 300, 200, 64, 512, 160, 128
+    q = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((S, H, D))))
+    kv = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((ne, D))))
+    kt = synth.to_bf16_values(O.rmsnorm(rng.standard_normal((S, D))))
+    idx = _rand_idx(rng, S, k, ne, [160, 0, 1, 129, 70])
+    sink = rng.standard_normal(H).astype(np.float32)
+    out = csa.csa_fused_attention(cuda(q, torch.bfloat16)[None], cuda(kv, torch.bfloat16)[None],
+                                  cuda(kt, torch.bfloat16)[None], cuda(np.array([0], np.int64)), W, cuda(sink),
+                                  idx=cuda(idx)[None], inv_rope=True, rope_dim=64, out_dtype=torch.float32, n_split=3)
+    csa.check_device_error()
+    Op, Lp = O.sparse_attention_partial(q, kv, idx)
+    ref = O.window_sink_combine(q, kt, np.arange(S), W, sink, Op, Lp, inv_rope=True)
+    assert_close(host(out)[0], ref, what="split-KV prefill")
