@@ -207,6 +207,126 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None):
                          "frac": ach_idx / hbm, "traffic": None, "peak_source": f"{src} copy bandwidth"}}
 
 
+def mixed_decode_leg(dev, steps, warmup, csa, synth, torch, seed=0):
+    """The 4-layer decode stack (CSA, HCA, CSA, HCA), batch 32, per-sequence
+    contexts U[64K, 1M]: one new token per sequence through all four layers."""
+    layers, q_pos, cfg = synth.mixed_decode_inputs_device(dev, seed=seed)
+    Bn, k, W, H, D, HI, DI = (cfg[x] for x in ("batch", "k", "W", "H", "D", "HI", "DI"))
+    L = cfg["lengths"]
+    sms = csa.num_sms()
+    split = {"csa": max(1, min(9, sms // Bn)), "hca": 16}
+    bufs = []
+    for lay in layers:
+        b = {"out": torch.empty(Bn, 1, H, D, dtype=torch.bfloat16, device=dev)}
+        cap = lay["kv_nope"].shape[1]
+        ns = split[lay["kind"]]
+        b["aws"] = torch.empty(csa.csa_fused_attention_workspace(Bn, 1, H, D, ns), dtype=torch.uint8, device=dev)
+        if lay["kind"] == "csa":
+            b["idx"] = torch.empty(Bn, 1, k, dtype=torch.int32, device=dev)
+            b["iws"] = torch.empty(csa.csa_index_topk_workspace(Bn, 1, cap, k), dtype=torch.uint8, device=dev)
+        bufs.append(b)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        for i, (lay, b) in enumerate(zip(layers, bufs)):
+            if ev is not None:
+                ev[i].record(stream)
+            if lay["kind"] == "csa":
+                csa.csa_layer_decode(lay, q_pos, k=k, n_split=split["csa"], idx=b["idx"], out=b["out"],
+                                     index_workspace=b["iws"], attn_workspace=b["aws"])
+            else:
+                csa.hca_layer_decode(lay, q_pos, n_split=split["hca"], out=b["out"], attn_workspace=b["aws"])
+        if ev is not None:
+            ev[len(layers)].record(stream)
+
+    for _ in range(max(3, warmup)):
+        step()
+    csa.check_device_error()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(layers) + 1)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    per_layer = [float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs])) for i in range(len(layers))]
+    ms = float(np.mean([e[0].elapsed_time(e[len(layers)]) for e in evs]))
+    # algorithmic bytes per step: CSA = every visible indexer key + scale, the
+    # selected e4m3 rows (448 + 128 + 4 bytes); HCA = every complete entry;
+    # both = the SWA rows and the query side
+    row = D - 64 + 128 + 4
+    qside = H * D * 2
+    algo = 0
+    for lay in layers:
+        if lay["kind"] == "csa":
+            nv = (L // 4)
+            algo += int((nv * (DI + 4)).sum() + (np.minimum(k, nv) * row).sum()) + Bn * (HI * DI + HI * 8)
+        else:
+            algo += int(((L // 128) * row).sum())
+        algo += Bn * (W * D * 2 + qside)
+    hbm, _, _, src = _peaks()
+    return {"workload": "mixed_decode", "layers": [l["kind"] for l in layers], "batch": Bn,
+            "context_min": int(L.min()), "context_max": int(L.max()), "top_k": k,
+            "attention_splits": split, "tokens_per_s": Bn / (ms * 1e-3), "ms_per_step": ms,
+            "layers_ms": per_layer, "algorithmic_bytes_per_step": algo,
+            "hbm_frac_step": algo / (ms * 1e-3) / 1e9 / hbm, "peak_source": f"{src} copy bandwidth"}
+
+
+def hca_prefill_leg(dev, steps, warmup, csa, synth, torch, seed=0):
+    """HCA layer prefill, S 131072, 64 x 512 bf16, m' 128 (1024 entries):
+    Q and window-row RMSNorm + RoPE, compressor (+ K norm / RoPE), and the fused
+    dense attention over complete entries + 128-token window + sink."""
+    inp, cfg = synth.prefill_inputs_device("hca_prefill", dev, seed=seed)
+    S, H, D, m, W = (cfg[x] for x in ("S", "H", "D", "m", "W"))
+    ne = S // m
+    bf = torch.bfloat16
+    pos = torch.zeros(1, dtype=torch.int64, device=dev)
+    qn = torch.empty(S, H, D, dtype=bf, device=dev)
+    kt = torch.empty(S, D, dtype=bf, device=dev)
+    kv = torch.empty(ne, D, dtype=bf, device=dev)
+    out = torch.empty(1, S, H, D, dtype=bf, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ["q_norm_rope", "kv_tok_norm_rope", "compress", "fused_attention"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        csa.csa_rmsnorm_rope(inp["q"], rows_per_pos=H, out=qn)
+        mark(1)
+        csa.csa_rmsnorm_rope(inp["C"], rows_per_pos=1, out=kt)
+        mark(2)
+        csa.csa_compress(inp["C"], inp["Z"], inp["B"], m, False, norm=True, rope_dim=64, out=kv)
+        mark(3)
+        csa.csa_fused_attention(qn[None], kv[None], kt[None], pos, W, inp["sink"], m=m, inv_rope=True,
+                                rope_dim=64, out=out)
+        mark(4)
+
+    for _ in range(max(3, warmup)):
+        step()
+    csa.check_device_error()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    per = {n: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in evs])) for j, n in enumerate(names)}
+    ms = float(np.mean([e[0].elapsed_time(e[len(names)]) for e in evs]))
+    t = np.arange(S, dtype=np.int64)
+    fl_dense = 4 * D * H * int(((t + 1) // m).sum())
+    fl_window = 4 * D * H * int(np.minimum(W, t + 1).sum())
+    _, _, bf16_sus, src = _peaks()
+    ach = (fl_dense + fl_window) / (per["fused_attention"] * 1e-3) / 1e12
+    return {"workload": "hca_prefill", "S": S, "H": H, "D": D, "m": m, "entries": ne, "window": W,
+            "tflops": (fl_dense + fl_window) / (ms * 1e-3) / 1e12, "ms_per_step": ms,
+            "prefill_tokens_per_s": S / (ms * 1e-3), "kernels_ms": per,
+            "flops_per_step": {"hca_dense": fl_dense, "swa_window": fl_window},
+            "roofline": {"kernel": "fused_attention", "bound": "tensor", "achieved": ach, "peak": bf16_sus,
+                         "unit": "TFLOP/s", "frac": ach / bf16_sus, "traffic": None,
+                         "peak_source": f"{src} bf16 sustained"}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -219,6 +339,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the 1M-context decode leg")
     ap.add_argument("--decode-batch", type=int, default=None, help="fewer decode sequences (profiling cases only)")
     ap.add_argument("--no-prefill", action="store_true", help="run only the decode leg (profiling cases only)")
+    ap.add_argument("--no-hca", action="store_true", help="skip the HCA prefill leg (S 131072)")
+    ap.add_argument("--no-mixed", action="store_true", help="skip the 4-layer mixed decode leg")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -357,7 +479,6 @@ def main():
     decode = None
     if not args.no_decode and args.S is None:
         decode = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch)
-
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = host_inputs(inp)
@@ -372,6 +493,17 @@ def main():
                "sample": f"{n_rows} evenly spaced query rows of the same S=16384 layer (float64 numpy oracle, "
                          f"{dt:.1f} s including its full-sequence compressor and window-row passes)"}
 
+    hca = mixed = None
+    if args.S is None:
+        del inp, qn, kt, kv, idx, ws, out
+        torch.cuda.empty_cache()
+        if not args.no_hca:
+            hca = hca_prefill_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=rank)
+            torch.cuda.empty_cache()
+        if not args.no_mixed:
+            mixed = mixed_decode_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=rank)
+            torch.cuda.empty_cache()
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -384,6 +516,7 @@ def main():
                                               "indexer_fp8": fl_index}},
                 "prefill_tokens_per_s": world * S / (ms * 1e-3),
                 "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode,
+                "hca_prefill": hca, "decode_mixed": mixed,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:

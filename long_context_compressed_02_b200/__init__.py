@@ -306,3 +306,29 @@ def hca_layer_prefill(q, C, Z, B, sink, *, m=128, W=128, norm_rope=False, inv_ro
         out = swa_sink_combine(qn[None], kt[None], pos, W, sink, Op, Lp, window_mode=0, inv_rope=inv_rope,
                                rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
     return out[0]
+
+
+def csa_layer_decode(lay, q_pos, *, k, m=4, W=128, n_split=1, idx=None, out=None, index_workspace=None,
+                     attn_workspace=None, stream=None):
+    """One CSA layer, one decode step per sequence over its caches: lightning
+    indexer + top-k over the e4m3 key cache, then the selected e4m3 entries,
+    the SWA cache and the sink in one softmax, inverse RoPE at q_pos.
+    `lay` holds q, qI, qI_scale, w, kI, kI_scale, kv_nope, kv_rope, kv_scale,
+    swa, sink (the layout of synth's decode inputs).  Returns (out, idx)."""
+    idx = csa_index_topk(lay["qI"], lay["w"], lay["kI"], q_pos, m, k, qI_scale=lay["qI_scale"],
+                         kI_scale=lay["kI_scale"], workspace=index_workspace, idx=idx, stream=stream)
+    out = csa_fused_attention(lay["q"], lay["kv_nope"], lay["swa"], q_pos, W, lay["sink"], idx=idx,
+                              kv_rope=lay["kv_rope"], kv_scale=lay["kv_scale"], window_mode=1, inv_rope=True,
+                              rope_dim=lay["kv_rope"].shape[-1], out=out, n_split=n_split,
+                              workspace=attn_workspace, stream=stream)
+    return out, idx
+
+
+def hca_layer_decode(lay, q_pos, *, m=128, W=128, n_split=1, out=None, attn_workspace=None, stream=None):
+    """One HCA layer, one decode step per sequence: dense attention over every
+    complete m'-entry of the e4m3 cache, the SWA cache and the sink in one
+    softmax, inverse RoPE at q_pos."""
+    return csa_fused_attention(lay["q"], lay["kv_nope"], lay["swa"], q_pos, W, lay["sink"], m=m,
+                               kv_rope=lay["kv_rope"], kv_scale=lay["kv_scale"], window_mode=1, inv_rope=True,
+                               rope_dim=lay["kv_rope"].shape[-1], out=out, n_split=n_split,
+                               workspace=attn_workspace, stream=stream)

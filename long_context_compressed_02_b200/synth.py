@@ -180,6 +180,42 @@ def prefill_inputs_device(name: str, device, seed: int = 0, S: int | None = None
     return out, dict(cfg, S=S)
 
 
+def _decode_layer(g, B, ne, H, D, HI, DI, W, r, grid, indexer):
+    """One layer's batched decode caches and query side, drawn from generator g.
+    Row scales are powers of two 2^U{-2..2} and codes hold N(0,1)/scale."""
+    device = g.device
+
+    def pow2(*shape):
+        return torch.pow(2.0, torch.randint(-2, 3, shape, generator=g, device=device).float())
+
+    out = {}
+    sc = pow2(B, ne)
+    out["kv_nope"] = (torch.randn(B, ne, D - r, generator=g, device=device) / sc[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    out["kv_rope"] = torch.randn(B, ne, r, generator=g, device=device).to(torch.bfloat16)
+    out["kv_scale"] = sc
+    if indexer:
+        ks = pow2(B, ne)
+        y = torch.randn(B, ne, DI, generator=g, device=device)
+        qs = pow2(B, 1, HI)
+        x = torch.randn(B, 1, HI, DI, generator=g, device=device)
+        if grid:
+            y, x = torch.round(y * 8) / 8, torch.round(x * 8) / 8
+            ks, qs = torch.ones_like(ks), torch.ones_like(qs)
+            w = torch.floor(torch.rand(B, 1, HI, generator=g, device=device) * 16) / 16
+        else:
+            y, x = y / ks[..., None], x / qs[..., None]
+            w = torch.rand(B, 1, HI, generator=g, device=device)
+        out["kI"] = y.to(torch.float8_e4m3fn).view(torch.uint8)
+        out["kI_scale"] = ks
+        out["qI"] = x.to(torch.float8_e4m3fn).view(torch.uint8)
+        out["qI_scale"] = qs
+        out["w"] = w.contiguous()
+    out["q"] = torch.randn(B, 1, H, D, generator=g, device=device).to(torch.bfloat16)
+    out["swa"] = torch.randn(B, W, D, generator=g, device=device).to(torch.bfloat16)
+    out["sink"] = torch.randn(H, generator=g, device=device)
+    return out
+
+
 def decode_inputs_device(name: str, device, seed: int = 0, grid: bool = False, batch: int | None = None,
                          ctx: int | None = None):
     """Batched decode-step inputs for `csa_decode_1m` on `device` (torch's seeded
@@ -196,33 +232,31 @@ def decode_inputs_device(name: str, device, seed: int = 0, grid: bool = False, b
     m = cfg["m"]
     ne = L // m
     g = torch.Generator(device=device).manual_seed(seed)
-
-    def pow2(*shape):
-        return torch.pow(2.0, torch.randint(-2, 3, shape, generator=g, device=device).float())
-
-    out = {}
-    sc = pow2(B, ne)
-    out["kv_nope"] = (torch.randn(B, ne, D - r, generator=g, device=device) / sc[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
-    out["kv_rope"] = torch.randn(B, ne, r, generator=g, device=device).to(torch.bfloat16)
-    out["kv_scale"] = sc
-    ks = pow2(B, ne)
-    y = torch.randn(B, ne, DI, generator=g, device=device)
-    qs = pow2(B, 1, HI)
-    x = torch.randn(B, 1, HI, DI, generator=g, device=device)
-    if grid:
-        y, x = torch.round(y * 8) / 8, torch.round(x * 8) / 8
-        ks, qs = torch.ones_like(ks), torch.ones_like(qs)
-        w = torch.floor(torch.rand(B, 1, HI, generator=g, device=device) * 16) / 16
-    else:
-        y, x = y / ks[..., None], x / qs[..., None]
-        w = torch.rand(B, 1, HI, generator=g, device=device)
-    out["kI"] = y.to(torch.float8_e4m3fn).view(torch.uint8)
-    out["kI_scale"] = ks
-    out["qI"] = x.to(torch.float8_e4m3fn).view(torch.uint8)
-    out["qI_scale"] = qs
-    out["w"] = w.contiguous()
-    out["q"] = torch.randn(B, 1, H, D, generator=g, device=device).to(torch.bfloat16)
-    out["swa"] = torch.randn(B, W, D, generator=g, device=device).to(torch.bfloat16)
-    out["sink"] = torch.randn(H, generator=g, device=device)
+    out = _decode_layer(g, B, ne, H, D, HI, DI, W, r, grid, True)
     out["q_pos"] = torch.full((B,), L - 1, dtype=torch.int64, device=device)
     return out, dict(cfg, batch=B, ctx=L, n_e=ne)
+
+
+def mixed_decode_inputs_device(device, seed: int = 0, grid: bool = False, batch: int | None = None,
+                               lengths=None):
+    """Inputs of one decode step of the 4-layer stack `mixed_decode` (CSA, HCA,
+    CSA, HCA), each layer with its own independently drawn caches and query:
+    per-sequence contexts L_b (decode_lengths, or `lengths`), caches padded to
+    the longest sequence (CSA: max L / 4 entries, HCA: max L / 128), new token
+    at position L_b - 1.  Returns (layers, q_pos [B] int64, cfg); each layer is a
+    dict like decode_inputs_device's plus "kind" and "m"."""
+    cfg = dict(WORKLOADS["mixed_decode"])
+    L = decode_lengths("mixed_decode", seed) if lengths is None else np.asarray(lengths, np.int64)
+    if batch is not None:
+        L = L[:batch]
+    B = len(L)
+    H, D, HI, DI, W, r = cfg["H"], cfg["D"], cfg["HI"], cfg["DI"], cfg["W"], cfg["rope_dim"]
+    g = torch.Generator(device=device).manual_seed(seed)
+    layers = []
+    for kind in cfg["layers"]:
+        m = 4 if kind == "csa" else 128
+        lay = _decode_layer(g, B, int(L.max()) // m, H, D, HI, DI, W, r, grid, kind == "csa")
+        lay["kind"], lay["m"] = kind, m
+        layers.append(lay)
+    q_pos = torch.as_tensor(L - 1, dtype=torch.int64).to(device)
+    return layers, q_pos, dict(cfg, batch=B, lengths=L)
