@@ -338,7 +338,7 @@ def main():
     ap.add_argument("--S", type=int, default=None, help="shorter sequence (profiling cases only)")
     ap.add_argument("--no-decode", action="store_true", help="skip the 1M-context decode leg")
     ap.add_argument("--decode-batch", type=int, default=None, help="fewer decode sequences (profiling cases only)")
-    ap.add_argument("--no-prefill", action="store_true", help="run only the decode leg (profiling cases only)")
+    ap.add_argument("--no-prefill", action="store_true", help="run only the decode legs (profiling cases only)")
     ap.add_argument("--no-hca", action="store_true", help="skip the HCA prefill leg (S 131072)")
     ap.add_argument("--no-mixed", action="store_true", help="skip the 4-layer mixed decode leg")
     args = ap.parse_args()
@@ -364,9 +364,13 @@ def main():
     csa.lib()
 
     if args.no_prefill:
-        d = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch)
+        out = {}
+        if not args.no_decode:
+            out["decode_1m"] = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch)
+        if not args.no_mixed:
+            out["decode_mixed"] = mixed_decode_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=rank)
         if rank == 0:
-            print(json.dumps({"decode_1m": d}), flush=True)
+            print(json.dumps(out), flush=True)
         return
     inp, cfg = synth.prefill_inputs_device(WORKLOAD, dev, seed=rank, S=args.S)
     S, H, D, m, k, W, HI, DI = (cfg[x] for x in ("S", "H", "D", "m", "k", "W", "HI", "DI"))

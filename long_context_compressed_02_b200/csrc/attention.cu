@@ -12,23 +12,26 @@
 // inverse RoPE applied on the output side.
 //
 // Design (one query token = 64 query rows: its heads, zero-padded):
-//   S^T[row, head] = KV_chunk[128 rows, D] . Q[64, D]^T     M=128, N=64, K=D
-//   O^T[d, head]  += KV_chunk^T[d, 128 rows] . P^T[rows, 64]  M=128 per 128-d tile
-// Both products are BF16 kind::f16 MMAs with fp32 accumulators in TMEM, so
-// every MMA has M = 128 (the full tensor-core height) while a token's 64 heads
-// sit on N.  K = V: the SAME shared-memory chunk is the K-major A operand of
-// the first product and, read through an MN-major descriptor, the A operand
-// of the second; nothing is transposed or copied.  Softmax runs over TMEM
-// lanes (rows) per column (head): column maxima and sums use warp
-// transpose-reductions plus a 4-warp exchange; the running max is only raised
-// when it grows by more than 2^8, so O^T is rarely rescaled.
+//   S^T[row, head] = KV_half[64 rows, D] . Q[64, D]^T       M=64,  N=64, K=D
+//   O^T[d, head]  += KV_half^T[d, 64 rows] . P^T[rows, 64]    M=128 per 128-d tile, K=64
+// Both products are BF16 kind::f16 MMAs with fp32 accumulators in TMEM; a
+// token's 64 heads sit on N.  K = V: the SAME shared-memory rows are the
+// K-major A operand of the first product and, read through an MN-major
+// descriptor, the A operand of the second; nothing is transposed or copied.
+// Rows stream through a ring of two 64-row slots (half chunks), so the loads
+// of half chunk h+1 overlap the S, softmax and PV work of half chunk h, and
+// S(h+1) is issued ahead of PV(h) so the softmax of h+1 overlaps PV(h).
+// Softmax runs per column (head) over TMEM lanes (rows): the M=64 S^T is
+// read with the 16x256b TMEM shape (all 32 threads of a warp hold data),
+// column maxima and sums use a 3-level butterfly plus a 4-warp exchange; the
+// running max is only raised when it grows by more than 2^8, so O^T is
+// rarely rescaled.
 //
-// Roles (288 threads): warps 0-3 softmax + epilogue (one TMEM lane each),
-// warps 4-7 loaders (one chunk row each: gather through cp.async, or
-// load-convert for fp32 / e4m3 stores), warp 8 TMEM allocation + MMA issue.
-// The chunk buffer is loaded slab by slab (64 columns = 128 bytes, 128-byte
-// swizzle) and a slab pair is refilled as soon as the PV MMA of its 128-column
-// tile retires, so loads overlap the tail of the previous chunk's MMAs.
+// Roles (288 threads): warps 0-3 softmax + epilogue, warps 4-7 loaders
+// (gathers through cp.async tracked on mbarriers, TMA boxes for contiguous
+// rows, or load-convert for fp32 / e4m3 stores), warp 8 TMEM allocation +
+// MMA issue.  Each slot is refilled slab pair by slab pair as the PV tile
+// that read it retires, and S MMAs start on a slab pair as soon as it lands.
 #include <algorithm>
 #include <cstring>
 #include <cuda_bf16.h>
@@ -53,7 +56,7 @@ namespace {
 
 constexpr int kThreads = 288;
 constexpr int kNQ = 64;            // query rows (heads) per tile = MMA N
-constexpr int kRows = 128;         // KV rows per chunk = MMA M
+constexpr int kRows = 64;          // KV rows per ring slot (a half chunk) = M of the S MMA
 constexpr float kTau = 8.0f;       // lazy-rescale threshold (log2 units)
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -92,16 +95,17 @@ struct AttnParams {
   int out_bf16, inv_rope, rope_dim;
   float rope_base;
   int tma_q, tma_kv, tma_tok;   // TMA tile loads for bf16 queries / dense entries / window rows
-  int n_split;                  // chunk-range splits per query token (partials merged afterwards)
+  int n_split;                  // ranges of half chunks per query token (partials merged afterwards)
 };
 
-// Chunk order: the window rows (source 2) come first, so that they start on a
-// 128-row chunk boundary and load as one TMA box per slab; the compressed
-// rows (source 1) follow from the next chunk boundary.
+// Rows are consumed in half chunks of 64 (one ring slot each).  The window
+// rows (source 2) come first, so that they start on a half-chunk boundary and
+// load as one TMA box per slab; the compressed rows (source 1) follow from
+// the next boundary.  Every half chunk holds rows of one source only.
 struct RowSet {
   int n1, n2, n;            // rows from source 1, source 2, total
-  int nc2, nchunks;         // window chunks, all chunks
-  int c0, c1;               // chunk range of this work item (split-KV)
+  int nh2, nh;              // window half chunks, all half chunks
+  int c0, c1;               // half-chunk range of this work item (split-KV)
   int64_t lo2;              // first window row
   const int32_t* idx;       // gather list (source 1)
 };
@@ -143,21 +147,21 @@ __device__ __forceinline__ RowSet row_set_warp(const AttnParams& p, int b, int t
     r.n2 = (int)min(min((int64_t)p.W, p.cap2), pos + 1);
   }
   r.n = r.n1 + r.n2;
-  r.nc2 = (r.n2 + kRows - 1) / kRows;
-  r.nchunks = r.nc2 + (r.n1 + kRows - 1) / kRows;
-  const int per = (r.nchunks + p.n_split - 1) / p.n_split;
-  r.c0 = min(r.nchunks, sp * per);
-  r.c1 = min(r.nchunks, r.c0 + per);
+  r.nh2 = (r.n2 + kRows - 1) / kRows;
+  r.nh = r.nh2 + (r.n1 + kRows - 1) / kRows;
+  const int per = (r.nh + p.n_split - 1) / p.n_split;
+  r.c0 = min(r.nh, sp * per);
+  r.c1 = min(r.nh, r.c0 + per);
   return r;
 }
 
+// mbarrier.try_wait suspends the thread in hardware until the phase completes
+// (or a short system time limit passes), so the loop needs no sleep of its own;
+// the wall clock and the CTA's abort flag are checked every 64 polls.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  // a few tight polls, then back off with nanosleep so that waiting warps do not
-  // flood the shared-memory pipe that the loads and stores of other warps use
   uint64_t start = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (i > 8) __nanosleep(i < 64 ? 32 : 128);
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
       const uint64_t now = global_ns();
@@ -188,22 +192,11 @@ __device__ __forceinline__ uint4 to_bf16x8(const float* v) {
   return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
 }
 
-// cp.async.wait_group needs an immediate: dispatch the (unrolled) count.
-__device__ __forceinline__ void cp_async_wait_pending(int n) {
-  switch (n) {
-    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-    case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
-    case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
-    case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
-    default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
-  }
-}
-
 __device__ __forceinline__ void st_shared16(uint8_t* dst, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" :: "r"(smem_u32(dst)), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void st_shared4(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" :: "r"(addr), "r"(v) : "memory");
 }
 
 // e4m3 x 16 -> 16 floats (hardware conversion through f16x2)
@@ -219,111 +212,50 @@ __device__ __forceinline__ void e4m3x16_to_float(uint4 raw, float scale, float* 
   }
 }
 
-// Loads the 64-column slab `s` of KV row `row` (or zeros) into row `r` of a
-// 128-byte-swizzled slab buffer.  BF16 rows use cp.async (caller commits).
-template <int D, int KV>
-__device__ __forceinline__ void load_kv_slab(const AttnParams& p, int b, int64_t row, bool valid, int s,
-                                             uint8_t* slab_base, int r) {
-  if constexpr (KV == KV_BF16) {
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kv) +
-                         ((((int64_t)b * p.cap + (valid ? row : 0)) * D + 64 * s) * 2);
+// 64 fp32 values (one 128-byte slab of a row, after conversion) -> row r of a
+// 128-byte-swizzled bf16 slab.
+__device__ __forceinline__ void store_row_slab_f32(uint8_t* slab_base, int r, const float* v) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) cp_async16(slab_base + swz128(r, q), src + 16 * q, valid ? 16u : 0u);
-  } else if constexpr (KV == KV_F32) {
-    const float* src = reinterpret_cast<const float*>(p.kv) + ((int64_t)b * p.cap + (valid ? row : 0)) * D + 64 * s;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      float v[8];
-      if (valid) {
-        float4 a = __ldg(reinterpret_cast<const float4*>(src + 8 * q));
-        float4 c = __ldg(reinterpret_cast<const float4*>(src + 8 * q) + 1);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.f;
-      }
-      st_shared16(slab_base + swz128(r, q), to_bf16x8(v));
-    }
-  } else {
-    const int nope = D - p.rope_dim;           // rope_dim == 64: last slab is the bf16 RoPE part
-    if (64 * s < nope) {
-      float v[64];
-      if (valid) {
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kv) + ((int64_t)b * p.cap + row) * nope + 64 * s;
-        const float sc = p.kv_scale[(int64_t)b * p.cap + row];
-        uint4 raw[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) raw[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) e4m3x16_to_float(raw[i], sc, v + 16 * i);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) v[i] = 0.f;
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) st_shared16(slab_base + swz128(r, q), to_bf16x8(v + 8 * q));
-    } else {
-      const uint4* src = reinterpret_cast<const uint4*>(p.kv_rope + ((int64_t)b * p.cap + (valid ? row : 0)) * p.rope_dim);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) st_shared16(slab_base + swz128(r, q), valid ? __ldg(src + q) : make_uint4(0, 0, 0, 0));
-    }
-  }
+  for (int q = 0; q < 8; ++q) st_shared16(slab_base + swz128(r, q), to_bf16x8(v + 8 * q));
 }
 
-// Source-2 (window) rows: bf16 or f32 [n_seq, cap2, D].  ASYNC selects
-// cp.async (bf16 only, caller commits) or a synchronous load + store.
-template <int D, int KV2, bool ASYNC>
-__device__ __forceinline__ void load_tok_slab(const AttnParams& p, int b, int64_t row, bool valid, int s,
-                                              uint8_t* slab_base, int r) {
-  if constexpr (KV2 == KV_BF16) {
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kv2) +
-                         ((((int64_t)b * p.cap2 + (valid ? row : 0)) * D + 64 * s) * 2);
-    if constexpr (ASYNC) {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) cp_async16(slab_base + swz128(r, q), src + 16 * q, valid ? 16u : 0u);
-    } else {
-      uint4 v[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = valid ? __ldg(reinterpret_cast<const uint4*>(src) + q) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) st_shared16(slab_base + swz128(r, q), v[q]);
-    }
-  } else {
-    const float* src = reinterpret_cast<const float*>(p.kv2) + ((int64_t)b * p.cap2 + (valid ? row : 0)) * D + 64 * s;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      float v[8];
-      if (valid) {
-        float4 a = __ldg(reinterpret_cast<const float4*>(src + 8 * q));
-        float4 c = __ldg(reinterpret_cast<const float4*>(src + 8 * q) + 1);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.f;
-      }
-      st_shared16(slab_base + swz128(r, q), to_bf16x8(v));
-    }
-  }
-}
-
-// BF16 stores, cp.async: one 128-byte slab of 32 chunk rows per loader warp.
-// Lane l moves 16 bytes of row 4j + l/8 (j = 0..7), so each warp instruction
-// reads 4 whole 128-byte row segments (full L2 sectors) instead of 32 scattered
-// 16-byte pieces.  row / valid / win are the caller's own chunk row (lane).
-template <int D>
-__device__ __forceinline__ void gather_slab_bf16(const AttnParams& p, int b, int64_t row, bool valid, bool win,
-                                                 int sl, uint8_t* slab_base, int warp_row0, int lane) {
+// One loader warp's 16 rows of one 128-byte slab, bf16, cp.async: lane l holds
+// the row pointer of row l & 15; each instruction moves 4 whole 128-byte row
+// segments (lane l: 16 bytes of row 4j + l/8), so every request is a full L2
+// line.  Rows marked invalid are zero-filled.
+__device__ __forceinline__ void gather16_bf16(const uint8_t* rp, bool valid, int sl, uint8_t* slab_base,
+                                              int row0, int lane) {
   const int q = lane & 7;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < 4; ++j) {
     const int rl = 4 * j + (lane >> 3);
-    const int64_t rr = __shfl_sync(0xffffffffu, row, rl);
-    const bool rv = __shfl_sync(0xffffffffu, valid, rl);
-    const bool rw = __shfl_sync(0xffffffffu, win, rl);
-    const uint8_t* base = rw ? reinterpret_cast<const uint8_t*>(p.kv2) + ((int64_t)b * p.cap2 + (rv ? rr : 0)) * D * 2
-                             : reinterpret_cast<const uint8_t*>(p.kv) + ((int64_t)b * p.cap + (rv ? rr : 0)) * D * 2;
-    cp_async16(slab_base + swz128(warp_row0 + rl, q), base + 128 * sl + 16 * q, rv ? 16u : 0u);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(rp), rl));
+    const bool v = __shfl_sync(0xffffffffu, valid, rl);
+    cp_async16(slab_base + swz128(row0 + rl, q), src + 128 * sl + 16 * q, v ? 16u : 0u);
   }
+}
+
+// Column reduction over a warp's 16 accumulator rows, laid out as returned by
+// tmem_ld16x256b_x8: v[2c + j] (c = 0..7, j = 0..1) is this thread's value of
+// column 8c + 2(lane % 4) + j, already combined over its two rows.  Three
+// butterfly levels over lane bits 4, 3, 2 halve the list each time, so that
+// lane l ends with columns 2l and 2l + 1 reduced over all 16 rows.
+template <bool MAX>
+__device__ __forceinline__ float2 col_reduce16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int lv = 0; lv < 3; ++lv) {
+    const int off = 16 >> lv, n = 8 >> lv;
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+      const float keep = up ? v[i + n] : v[i];
+      const float send = up ? v[i] : v[i + n];
+      const float got = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return make_float2(v[0], v[1]);
 }
 
 template <int D, int KV, int EPI>
@@ -331,39 +263,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap map_q,
             const __grid_constant__ CUtensorMap map_kv, const __grid_constant__ CUtensorMap map_tok) {
   constexpr int NS = D / 64;                 // 128-byte slabs per row
-  constexpr int NT = D / 128;                // O^T tiles
+  constexpr int NT = D / 128;                // O^T tiles (two slabs each)
   constexpr uint32_t kQSlab = kNQ * 128;     // 8 KB
-  constexpr uint32_t kKSlab = kRows * 128;   // 16 KB
-  constexpr uint32_t kTmemCols = (64 + 64 * NT) <= 128 ? 128 : ((64 + 64 * NT) <= 256 ? 256 : 512);
+  constexpr uint32_t kSlab = kRows * 128;    // 8 KB: one slab of a slot
+  constexpr uint32_t kSlot = NS * kSlab;     // one half chunk
+  constexpr uint32_t kPBuf = kRows * 128;    // P^T of one half chunk (64 rows x 64 heads bf16)
+  // TMEM: S^T of the two slots in two accumulators each (columns 0..255), O^T tiles from 256
+  constexpr uint32_t kTmemCols = 512;
+  constexpr uint32_t kOCol = 256;
   constexpr int KV2 = (KV == KV_F32) ? KV_F32 : KV_BF16;   // window rows: bf16 unless the store is fp32
-  constexpr bool kAsync = (KV == KV_BF16);                  // cp.async for every row of a bf16 store
 
   extern __shared__ uint8_t smem_raw[];
   // aligned by offsetting the shared array itself, so accesses stay in the shared window
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + NS * kQSlab;
-  uint8_t* sP = sKV + NS * kKSlab;
-  float* s_red = reinterpret_cast<float*>(sP + kRows * 128);   // [2][4][64] column partials
+  uint8_t* sKV = sQ + NS * kQSlab;                               // [2 slots][NS slabs][64 rows][128 B]
+  uint8_t* sP = sKV + 2 * kSlot;                                 // [2][64 rows][128 B]; epilogue staging
+  float* s_red = reinterpret_cast<float*>(sP + 2 * kPBuf);       // [2][4][64] column partials
   float* s_bc = s_red + 2 * 4 * 64;                              // [4 warps][3][64] broadcasts
   float2* s_cs = reinterpret_cast<float2*>(s_bc + 4 * 3 * 64);  // [2][32] inverse-RoPE cos/sin
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_cs + 64);
   uint64_t* q_full = bars + 0;
   uint64_t* q_free = bars + 1;
-  uint64_t* s_done = bars + 2;
-  uint64_t* p_full = bars + 3;
-  uint64_t* epi_done = bars + 4;
-  uint64_t* kv_full = bars + 5;              // [NS]
-  uint64_t* pv_done = kv_full + NS;          // [NT]
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(pv_done + NT);
+  uint64_t* epi_done = bars + 2;
+  uint64_t* s_full = bars + 3;               // [2]   S^T of a half chunk in TMEM
+  uint64_t* s_free = bars + 5;               // [2]   ... read by the softmax warps
+  uint64_t* p_full = bars + 7;               // [2]   P^T in shared memory (and O^T rescaled)
+  uint64_t* kv_full = bars + 9;              // [2][NT] slab pair of a slot loaded
+  uint64_t* pv_done = kv_full + 2 * NT;      // [2][NT] PV tile of a slot retired
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(pv_done + 2 * NT);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(q_full, 128); mbar_init(q_free, 1); mbar_init(s_done, 1);
-    mbar_init(p_full, 128); mbar_init(epi_done, 128);
-    for (int s = 0; s < NS; ++s) mbar_init(&kv_full[s], 128);
-    for (int t = 0; t < NT; ++t) mbar_init(&pv_done[t], 1);
+    mbar_init(q_full, 128); mbar_init(q_free, 1); mbar_init(epi_done, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128); mbar_init(&p_full[i], 128);
+      for (int t = 0; t < NT; ++t) { mbar_init(&kv_full[i * NT + t], 128); mbar_init(&pv_done[i * NT + t], 1); }
+    }
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -377,7 +314,9 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
 
   if (warp >= 4 && warp < 8) {
     // ============================ loaders
-    const int lt = tid - 128;
+    const int lt = tid - 128;                 // 0..127
+    const int lw = lt >> 5;                   // loader warp: rows 16 lw .. 16 lw + 15 of a slot (gathers)
+    const int my_r = lt & 63, part = lt >> 6; // converting loads: one row, slabs part, part + 2, ...
     uint32_t g = 0, qcount = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -397,50 +336,114 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
 #pragma unroll 1
           for (int s = 0; s < NS; ++s)
             tma_load_2d(sQ + s * kQSlab, &map_q, 64 * s, (int32_t)(((int64_t)b * p.T + t) * p.H), q_full);
-        }
-      } else if (p.q_f32) {
-        for (int u = lt; u < kNQ * NS; u += 128) {
-          const int r = u % kNQ, s = u / kNQ;
-          uint8_t* dst = sQ + s * kQSlab;
-          const bool v = r < p.H;
-          const int64_t qrow = ((int64_t)b * p.T + t) * p.H + (v ? r : 0);
-          const float* src = reinterpret_cast<const float*>(p.q) + qrow * D + 64 * s;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float x[8];
-            if (v) {
-              float4 a = __ldg(reinterpret_cast<const float4*>(src + 8 * q));
-              float4 c = __ldg(reinterpret_cast<const float4*>(src + 8 * q) + 1);
-              x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) x[i] = 0.f;
-            }
-            st_shared16(dst + swz128(r, q), to_bf16x8(x));
-          }
+        } else {
+          mbar_arrive(q_full);
         }
       } else {
-        // consecutive lanes take consecutive 16-byte pieces of one query row
-        constexpr int kPieces = D / 8;                       // 16-byte pieces per row
-        const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q) + ((int64_t)b * p.T + t) * p.H * D * 2;
-        for (int u = lt; u < kNQ * kPieces; u += 128) {
-          const int r = u / kPieces, c = u % kPieces;
-          const bool v = r < p.H;
-          cp_async16(sQ + (c >> 3) * kQSlab + swz128(r, c & 7), qb + ((int64_t)(v ? r : 0) * D) * 2 + 16 * c,
-                     v ? 16u : 0u);
+        if (p.q_f32) {
+          for (int u = lt; u < kNQ * NS; u += 128) {
+            const int r = u % kNQ, s = u / kNQ;
+            const bool v = r < p.H;
+            const int64_t qrow = ((int64_t)b * p.T + t) * p.H + (v ? r : 0);
+            const float* src = reinterpret_cast<const float*>(p.q) + qrow * D + 64 * s;
+            float x[64];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float4 a = v ? __ldg(reinterpret_cast<const float4*>(src) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+              x[4 * i] = a.x; x[4 * i + 1] = a.y; x[4 * i + 2] = a.z; x[4 * i + 3] = a.w;
+            }
+            store_row_slab_f32(sQ + s * kQSlab, r, x);
+          }
+        } else {
+          // consecutive lanes take consecutive 16-byte pieces of one query row
+          constexpr int kPieces = D / 8;                       // 16-byte pieces per row
+          const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q) + ((int64_t)b * p.T + t) * p.H * D * 2;
+          for (int u = lt; u < kNQ * kPieces; u += 128) {
+            const int r = u / kPieces, c = u % kPieces;
+            const bool v = r < p.H;
+            cp_async16(sQ + (c >> 3) * kQSlab + swz128(r, c & 7), qb + ((int64_t)(v ? r : 0) * D) * 2 + 16 * c,
+                       v ? 16u : 0u);
+          }
+          asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
         }
-      }
-      if (!p.tma_q || lt != 0) {
-        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
         fence_proxy_async_smem();
         mbar_arrive(q_full);
       }
-      // ---- KV chunks
+      // ---- KV half chunks into the two-slot ring
       for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
-        const bool win = c < rs.nc2;                   // window chunk (source 2)
-        const int cl = win ? c : c - rs.nc2;
-        const int r = cl * kRows + lt;
-        bool valid = r < (win ? rs.n2 : rs.n1);
+        const int slot = g & 1;
+        const uint32_t fpar = ((g >> 1) & 1) ^ 1;     // completion of PV(g - 2), which read this slot
+        uint8_t* sl_base = sKV + slot * kSlot;
+        uint64_t* full = kv_full + slot * NT;
+        uint64_t* done = pv_done + slot * NT;
+        const bool win = c < rs.nh2;                   // window rows (source 2)
+        const int cl = win ? c : c - rs.nh2;
+        const int nset = win ? rs.n2 : rs.n1;
+        // TMA boxes load whole 64-row blocks: used when every row of the box is
+        // either in the set or a real row of the same tensor (prefill window rows
+        // past the query are later tokens; masked rows then hold finite data).
+        // Partial blocks of caches, whose tail rows may be unwritten, take the
+        // zero-filling path instead.
+        const bool fullh = (cl + 1) * kRows <= nset;
+        const bool tma = win ? (p.tma_tok != 0 && (p.src2 == SRC2_WINDOW || fullh))
+                             : (rs.idx == nullptr && p.tma_kv != 0 && fullh);
+        if (tma) {
+          const int32_t y0 = win ? (int32_t)((int64_t)b * p.cap2 + rs.lo2 + (int64_t)cl * kRows)
+                                 : (int32_t)((int64_t)b * p.cap + (int64_t)cl * kRows);
+          for (int tt = 0; tt < NT; ++tt) {
+            if (!wait_bar(&done[tt], fpar, abort_flag)) { ok = false; break; }
+            if (lt == 0) {
+              mbar_expect_tx(&full[tt], 2 * kSlab);
+              tma_load_2d(sl_base + (2 * tt) * kSlab, win ? &map_tok : &map_kv, 128 * tt, y0, &full[tt]);
+              tma_load_2d(sl_base + (2 * tt + 1) * kSlab, win ? &map_tok : &map_kv, 128 * tt + 64, y0, &full[tt]);
+            } else {
+              mbar_arrive(&full[tt]);
+            }
+          }
+          continue;
+        }
+        const bool bf16_rows = win ? (KV2 == KV_BF16) : (KV == KV_BF16);
+        if (bf16_rows) {
+          // gather: this warp's 16 rows, one cp.async batch per slab pair, completion
+          // tracked on the slab pair's barrier (no wait in the loader)
+          const int r = cl * kRows + 16 * lw + (lane & 15);
+          bool valid = r < nset;
+          int64_t row = 0;
+          if (valid) {
+            if (win) {
+              row = rs.lo2 + r;
+            } else if (rs.idx) {
+              row = rs.idx[r];
+              if (row < 0 || row >= p.cap) { atomicOr(&g_err_attn, DEV_ERR_BAD_INDEX); valid = false; row = 0; }
+            } else {
+              row = r;
+            }
+          }
+          const uint8_t* rp = win ? reinterpret_cast<const uint8_t*>(p.kv2) + ((int64_t)b * p.cap2 + row) * D * 2
+                                  : reinterpret_cast<const uint8_t*>(p.kv) + ((int64_t)b * p.cap + row) * D * 2;
+          // Slab pair tt is signalled once this thread's copies of it have landed
+          // (cp.async group tt), fenced to the async proxy here, on the producer
+          // side, so the MMA issuer needs no proxy fence of its own.
+          for (int tt = 0; tt < NT; ++tt) {
+            if (!wait_bar(&done[tt], fpar, abort_flag)) { ok = false; break; }
+            gather16_bf16(rp, valid, 2 * tt, sl_base + (2 * tt) * kSlab, 16 * lw, lane);
+            gather16_bf16(rp, valid, 2 * tt + 1, sl_base + (2 * tt + 1) * kSlab, 16 * lw, lane);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            if (tt > 0) {
+              asm volatile("cp.async.wait_group 1;" ::: "memory");
+              fence_proxy_async_smem();
+              mbar_arrive(&full[tt - 1]);
+            }
+          }
+          if (!ok) break;
+          asm volatile("cp.async.wait_group 0;" ::: "memory");
+          fence_proxy_async_smem();
+          mbar_arrive(&full[NT - 1]);
+          continue;
+        }
+        // converting loads: thread (my_r, part) converts slabs 2 tt + part of row my_r
+        const int r = cl * kRows + my_r;
+        bool valid = r < nset;
         int64_t row = 0;
         if (valid) {
           if (win) {
@@ -452,125 +455,111 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
             row = r;
           }
         }
-        // TMA boxes load whole 128-row blocks: used when every row of the box is
-        // either in the set or a real row of the same tensor (prefill window rows
-        // past the query are later tokens; masked rows then hold finite data).
-        // Partial chunks of caches, whose tail rows may be unwritten, take the
-        // zero-filling path instead.
-        const int nset = win ? rs.n2 : rs.n1;
-        const bool full = (cl + 1) * kRows <= nset;
-        const bool tma = win ? (p.tma_tok != 0 && (p.src2 == SRC2_WINDOW || full))
-                             : (rs.idx == nullptr && p.tma_kv != 0 && full);
-        if (tma) {
-          // one box of 128 rows x 64 columns per slab; rows past the set are masked later
-          const int32_t y0 = win ? (int32_t)((int64_t)b * p.cap2 + rs.lo2 + (int64_t)cl * kRows)
-                                 : (int32_t)((int64_t)b * p.cap + (int64_t)cl * kRows);
-          for (int tt = 0; tt < NT; ++tt) {
-            if (!wait_bar(&pv_done[tt], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (KV == KV_FP8 && !win) {
+          // e4m3 row: nope part (D - 64 bytes) + bf16 RoPE part + scale.  The raw
+          // bytes of this thread's slabs are fetched before the slot is free.
+          constexpr int kNope = D - 64;
+          const uint8_t* srcn = reinterpret_cast<const uint8_t*>(p.kv) + ((int64_t)b * p.cap + row) * kNope;
+          const uint4* srcr = reinterpret_cast<const uint4*>(p.kv_rope + ((int64_t)b * p.cap + row) * 64);
+          const float sc = valid ? __ldg(p.kv_scale + (int64_t)b * p.cap + row) : 0.f;
+          uint4 raw[NT][4];
+          uint4 rp8[8];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int sl = 2 * tt + h;
-              if (lt == 0) {
-                mbar_expect_tx(&kv_full[sl], kKSlab);
-                tma_load_2d(sKV + sl * kKSlab, win ? &map_tok : &map_kv, 64 * sl, y0, &kv_full[sl]);
-              } else {
-                mbar_arrive(&kv_full[sl]);
+          for (int tt = 0; tt < NT; ++tt) {
+            const int s = 2 * tt + part;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              raw[tt][i] = (valid && s < NS - 1) ? __ldg(reinterpret_cast<const uint4*>(srcn + 64 * s) + i)
+                                                  : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) rp8[i] = (valid && part == 1) ? __ldg(srcr + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int tt = 0; tt < NT; ++tt) {
+            if (!wait_bar(&done[tt], fpar, abort_flag)) { ok = false; break; }
+            const int s = 2 * tt + part;
+            uint8_t* dst = sl_base + s * kSlab;
+            if (s < NS - 1) {
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                float v[16];
+                e4m3x16_to_float(raw[tt][q4], sc, v);
+                st_shared16(dst + swz128(my_r, 2 * q4), to_bf16x8(v));
+                st_shared16(dst + swz128(my_r, 2 * q4 + 1), to_bf16x8(v + 8));
               }
+            } else {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) st_shared16(dst + swz128(my_r, q), rp8[q]);
             }
+            fence_proxy_async_smem();
+            mbar_arrive(&full[tt]);
           }
           continue;
         }
-        if constexpr (KV == KV_FP8) {
-          if (!win) {
-            // e4m3 rows: the raw bytes of the row (nope part + bf16 RoPE part + scale)
-            // are fetched in two batches well ahead of use, then converted slab by slab
-            const int nope = D - p.rope_dim;            // rope_dim == 64
-            const uint4* srcn = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.kv) +
-                                                               ((int64_t)b * p.cap + row) * nope);
-            const uint4* srcr = reinterpret_cast<const uint4*>(p.kv_rope + ((int64_t)b * p.cap + row) * p.rope_dim);
-            const float sc = valid ? __ldg(p.kv_scale + (int64_t)b * p.cap + row) : 0.f;
-            constexpr int kNopeV = (D - 64) / 16;       // 16-byte vectors of e4m3 per row
-            constexpr int kHalf = (NS / 2) * 4;         // vectors of the first half of the slabs
-            uint4 raw[kNopeV];
-#pragma unroll
-            for (int i = 0; i < kHalf && i < kNopeV; ++i) raw[i] = valid ? __ldg(srcn + i) : make_uint4(0, 0, 0, 0);
-            uint4 rp[8];
-#pragma unroll
-            for (int tt = 0; tt < NT; ++tt) {
-              if (!wait_bar(&pv_done[tt], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
-              if (tt == 0) {
-#pragma unroll
-                for (int i = kHalf; i < kNopeV; ++i) raw[i] = valid ? __ldg(srcn + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) rp[i] = valid ? __ldg(srcr + i) : make_uint4(0, 0, 0, 0);
-              }
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int sl = 2 * tt + h;
-                uint8_t* dst = sKV + sl * kKSlab;
-                if (64 * sl < nope) {
-#pragma unroll
-                  for (int q4 = 0; q4 < 4; ++q4) {
-                    float v[16];
-                    e4m3x16_to_float(raw[(4 * sl + q4) % kNopeV], sc, v);
-                    st_shared16(dst + swz128(lt, 2 * q4), to_bf16x8(v));
-                    st_shared16(dst + swz128(lt, 2 * q4 + 1), to_bf16x8(v + 8));
-                  }
-                } else {
-#pragma unroll
-                  for (int q = 0; q < 8; ++q) st_shared16(dst + swz128(lt, q), rp[q]);
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&kv_full[sl]);
-              }
-            }
-            continue;
-          }
-        }
-        // every slab pair is issued as soon as the PV tile that read it retires;
-        // completions are then retired in order (cp.async groups, one per slab)
+        // fp32 rows (an fp32 store and its window rows)
+        const float* src = win ? reinterpret_cast<const float*>(p.kv2) + ((int64_t)b * p.cap2 + row) * D
+                               : reinterpret_cast<const float*>(p.kv) + ((int64_t)b * p.cap + row) * D;
         for (int tt = 0; tt < NT; ++tt) {
-          if (!wait_bar(&pv_done[tt], (g & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int s = 2 * tt + part;
+          float v[64];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int sl = 2 * tt + h;
-            if constexpr (kAsync) gather_slab_bf16<D>(p, b, row, valid, win, sl, sKV + sl * kKSlab, lt & ~31, lane);
-            else if (win) load_tok_slab<D, KV2, kAsync>(p, b, row, valid, sl, sKV + sl * kKSlab, lt);
-            else     load_kv_slab<D, KV>(p, b, row, valid, sl, sKV + sl * kKSlab, lt);
-            if constexpr (kAsync) {
-              asm volatile("cp.async.commit_group;" ::: "memory");
-            } else {
-              fence_proxy_async_smem();
-              mbar_arrive(&kv_full[sl]);
-            }
+          for (int i = 0; i < 16; ++i) {
+            const float4 a = valid ? __ldg(reinterpret_cast<const float4*>(src + 64 * s) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
           }
-        }
-        if constexpr (kAsync) {
-          if (ok) {
-            // NS groups outstanding, oldest first: retire them one by one
-#pragma unroll
-            for (int sl = 0; sl < NS; ++sl) {
-              cp_async_wait_pending(NS - 1 - sl);
-              fence_proxy_async_smem();
-              mbar_arrive(&kv_full[sl]);
-            }
-          }
+          if (!wait_bar(&done[tt], fpar, abort_flag)) { ok = false; break; }
+          store_row_slab_f32(sl_base + s * kSlab, my_r, v);
+          fence_proxy_async_smem();
+          mbar_arrive(&full[tt]);
         }
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 8) {
     // ============================ MMA issuer (lane 0; the warp computes row sets)
-    const uint32_t idesc_s = make_idesc(128, kNQ, 1, 1, 0, 0);
+    // S^T(h) = KV_h[64 rows, D] . Q^T        M 64, N 64, into TMEM columns 64 (h % 2)
+    // O^T   += KV_h^T[128 d, 64 rows] . P_h^T  M 128, N 64, per 128-d tile
+    // S(h + 1) is issued before PV(h), so the softmax of half chunk h overlaps
+    // the S products of the next one.
+    const uint32_t idesc_s = make_idesc(64, kNQ, 1, 1, 0, 0);
     const uint32_t idesc_o = make_idesc(128, kNQ, 1, 1, 1, 1);
     // Descriptors differ only in the start-address field (bits 0..13, address >> 4):
-    // build each base once and add compile-time offsets, so an MMA costs one add.
-    const uint64_t dS_A = smem_desc(smem_u32(sKV), 16, 1024, SWZ_128B);       // KV chunk, K-major
+    // build each base once and add offsets, so an MMA costs one add.
+    const uint64_t dS_A = smem_desc(smem_u32(sKV), 16, 1024, SWZ_128B);       // KV half chunk, K-major
     const uint64_t dS_B = smem_desc(smem_u32(sQ), 16, 1024, SWZ_128B);        // Q tile, K-major
-    const uint64_t dO_A = smem_desc(smem_u32(sKV), kKSlab, 1024, SWZ_128B);   // KV chunk as V^T, MN-major
+    const uint64_t dO_A = smem_desc(smem_u32(sKV), kSlab, 1024, SWZ_128B);    // KV half chunk as V^T, MN-major
     const uint64_t dO_B = smem_desc(smem_u32(sP), 16, 1024, SWZ_128B);        // P^T, MN-major
-    uint32_t g = 0, qcount = 0, icount = 0;
+    uint32_t g = 0, qcount = 0, pv_items = 0;
     bool ok = true;
+    // PV(h): the 4 K-steps of a tile pair alternate between the pair's two
+    // accumulators (an MMA into the accumulator of the previous one waits for
+    // it); each pair commits its two tiles' barriers, which free their slabs.
+    auto issue_pv = [&](uint32_t h, bool first) -> bool {
+      if (!wait_bar(&p_full[h & 1], (h >> 1) & 1, abort_flag)) return false;
+      if (first) {
+        // O^T is overwritten: the previous item's epilogue must have read it
+        if (!wait_bar(epi_done, (pv_items & 1) ^ 1, abort_flag)) return false;
+        ++pv_items;
+      }
+      tc_fence_after();
+      const uint32_t slot = h & 1;
+#pragma unroll 1
+      for (int t0 = 0; t0 < NT; t0 += 2) {
+        const int np = NT - t0 >= 2 ? 2 : 1;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (j < np) {
+              const int tt = t0 + j;
+              mma_bf16(tmem + kOCol + 64 * tt, dO_A + ((slot * kSlot + 2 * tt * kSlab + kk * 2048) >> 4),
+                       dO_B + ((slot * kPBuf + kk * 2048) >> 4), idesc_o, (kk > 0 || !first) ? 1u : 0u);
+            }
+          }
+        }
+        for (int j = 0; j < np; ++j) mma_commit(&pv_done[slot * NT + t0 + j]);
+      }
+      return true;
+    };
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const int64_t bt = item / p.n_split;
       const int sp = (int)(item % p.n_split);
@@ -580,42 +569,59 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
       if (lane == 0) {
         if (!wait_bar(q_full, qcount & 1, abort_flag)) ok = false;
         ++qcount;
+        // Order: S(h), then PV(h - 1) (its softmax overlapped S(h)); the item's
+        // last PV follows its S at once, so the epilogue does not wait for the
+        // next item's loads.
+        bool pend = false;
+        uint32_t pend_g = 0;
+        bool pend_first = false;
         for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
-#pragma unroll 1
-          for (int s = 0; s < NS; ++s) {
-            if (!wait_bar(&kv_full[s], g & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tmem, dS_A + ((s * kKSlab + kk * 32) >> 4), dS_B + ((s * kQSlab + kk * 32) >> 4), idesc_s,
-                       (s | kk) != 0);
-          }
-          if (!ok) break;
-          mma_commit(s_done);
-          if (c == rs.c1 - 1) mma_commit(q_free);
-          if (!wait_bar(p_full, g & 1, abort_flag)) { ok = false; break; }
-          if (c == rs.c0 && !wait_bar(epi_done, (icount & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const uint32_t slot = g & 1;
+          if (!wait_bar(&s_free[slot], ((g >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t acc0 = c > rs.c0 ? 1u : 0u;
+          // S^T(g): even slabs into accumulator a (columns 64 slot), odd slabs into
+          // accumulator b (columns 128 + 64 slot), alternating MMA by MMA
 #pragma unroll 1
           for (int tt = 0; tt < NT; ++tt) {
+            if (!wait_bar(&kv_full[slot * NT + tt], (g >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16(tmem + 64 + 64 * tt, dO_A + ((2 * tt * kKSlab + kk * 2048) >> 4), dO_B + ((kk * 2048) >> 4),
-                       idesc_o, kk > 0 ? 1u : acc0);
-            mma_commit(&pv_done[tt]);
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const int s = 2 * tt + hh;
+                mma_bf16(tmem + 64 * slot + 128 * hh, dS_A + ((slot * kSlot + s * kSlab + kk * 32) >> 4),
+                         dS_B + ((s * kQSlab + kk * 32) >> 4), idesc_s, (tt | kk) != 0);
+              }
+            }
+          }
+          if (!ok) break;
+          mma_commit(&s_full[slot]);
+          const bool last = c == rs.c1 - 1;
+          if (last) mma_commit(q_free);
+          if (pend && !issue_pv(pend_g, pend_first)) { ok = false; break; }
+          pend = true; pend_g = g; pend_first = (c == rs.c0);
+          if (last) {
+            if (!issue_pv(pend_g, pend_first)) { ok = false; break; }
+            pend = false;
           }
         }
-        ++icount;
       }
       __syncwarp();
       ok = __shfl_sync(0xffffffffu, ok, 0);
+      g = __shfl_sync(0xffffffffu, g, 0);
     }
+    __syncwarp();
   } else {
     // ============================ softmax + epilogue (warps 0-3)
-    const int e = tid;                        // TMEM lane = chunk row = O^T d-row
+    // A half chunk's S^T (M = 64) sits in TMEM lanes 32w .. 32w + 15 of warp w:
+    // rows 16w .. 16w + 15.  tcgen05.ld 16x256b gives thread l rows
+    // 16w + l/4 and 16w + l/4 + 8 of columns 8c + 2(l%4) + {0, 1}; column
+    // statistics end up owned by lane l for columns 2l, 2l + 1.
+    const int e = tid;                        // TMEM lane of the O^T tiles = d-row
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     float* bc_m = s_bc + warp * 192;          // per-warp broadcast: [0,64) max, [64,128) alpha / coef_w, [128,192) coef_p
+    const int rA = 16 * warp + (lane >> 2), rB = rA + 8;
     uint32_t g = 0, icount = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
@@ -633,92 +639,100 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
         sincos(ang, &sd, &cd);
         cs[j] = make_float2((float)cd, (float)sd);
       }
-      float m_own[2] = {-CUDART_INF_F, -CUDART_INF_F};   // running max of columns lane, 32 + lane
-      float l_own[2] = {0.f, 0.f};
+      float m_own[2] = {-CUDART_INF_F, -CUDART_INF_F};   // running max of columns 2 lane, 2 lane + 1
+      float l_own[2] = {0.f, 0.f};                       // this warp's rows' sums of the same columns
       for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
-        if (!wait_bar(s_done, g & 1, abort_flag)) { ok = false; break; }
+        const uint32_t sb = g & 1;
+        if (!wait_bar(&s_full[sb], (g >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float x[64];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld16(tmem + lane_base + 16 * q, x + 16 * q);
+        float x[32], xb[32];
+        tmem_ld16x256b_x8(tmem + lane_base + 64 * sb, x);
+        tmem_ld16x256b_x8(tmem + lane_base + 128 + 64 * sb, xb);
         tmem_wait_ld();
-        const bool valid = c < rs.nc2 ? c * kRows + e < rs.n2 : (c - rs.nc2) * kRows + e < rs.n1;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) x[j] = valid ? x[j] : -CUDART_INF_F;   // raw logits; scale folded below
-        // column maxima over this warp's 32 rows: lane ends with columns lane, 32 + lane
-        float cm[2];
+        for (int i = 0; i < 32; ++i) x[i] += xb[i];
+        tc_fence_before();
+        mbar_arrive(&s_free[sb]);
+        const bool win = c < rs.nh2;
+        const int h0 = (win ? c : c - rs.nh2) * kRows;
+        const int nset = win ? rs.n2 : rs.n1;
+        const bool vA = h0 + rA < nset, vB = h0 + rB < nset;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = x[32 * h + i];
-#pragma unroll
-          for (int off = 16, n = 32; off >= 1; off >>= 1, n >>= 1) {
-            const bool up = (lane & off) != 0;
-#pragma unroll
-            for (int i = 0; i < n / 2; ++i) {
-              float keep = up ? v[i + n / 2] : v[i];
-              float send = up ? v[i] : v[i + n / 2];
-              v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
-            }
-          }
-          cm[h] = v[0];
+        for (int cc = 0; cc < 8; ++cc) {                   // raw logits; scale folded below
+          if (!vA) { x[4 * cc] = -CUDART_INF_F; x[4 * cc + 1] = -CUDART_INF_F; }
+          if (!vB) { x[4 * cc + 2] = -CUDART_INF_F; x[4 * cc + 3] = -CUDART_INF_F; }
         }
+        float v16[16];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          v16[2 * cc] = fmaxf(x[4 * cc], x[4 * cc + 2]);
+          v16[2 * cc + 1] = fmaxf(x[4 * cc + 1], x[4 * cc + 3]);
+        }
+        const float2 cm = col_reduce16<true>(v16, lane);
         float* red = s_red + (g & 1) * 256;
-        red[warp * 64 + lane] = cm[0];
-        red[warp * 64 + 32 + lane] = cm[1];
+        *reinterpret_cast<float2*>(red + warp * 64 + 2 * lane) = cm;
         named_bar_sync(1, 128);
         bool need_rescale = false;
         float alpha[2];
+        {
+          const float2 r0 = *reinterpret_cast<const float2*>(red + 2 * lane);
+          const float2 r1 = *reinterpret_cast<const float2*>(red + 64 + 2 * lane);
+          const float2 r2 = *reinterpret_cast<const float2*>(red + 128 + 2 * lane);
+          const float2 r3 = *reinterpret_cast<const float2*>(red + 192 + 2 * lane);
+          const float mx[2] = {fmaxf(fmaxf(r0.x, r1.x), fmaxf(r2.x, r3.x)) * p.scale_log2,
+                               fmaxf(fmaxf(r0.y, r1.y), fmaxf(r2.y, r3.y)) * p.scale_log2};
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int col = 32 * h + lane;
-          float mx = fmaxf(fmaxf(red[col], red[64 + col]), fmaxf(red[128 + col], red[192 + col])) * p.scale_log2;
-          float mn = (mx > m_own[h] + kTau) ? mx : m_own[h];
-          alpha[h] = exp2f(m_own[h] - mn);             // 0 on the first chunk
-          if (mn != m_own[h] && c > rs.c0) need_rescale = true;
-          m_own[h] = mn;
-          bc_m[col] = mn;
-          bc_m[64 + col] = alpha[h];
+          for (int j = 0; j < 2; ++j) {
+            const float mn = (mx[j] > m_own[j] + kTau) ? mx[j] : m_own[j];
+            alpha[j] = exp2f(m_own[j] - mn);             // 0 on the first half chunk
+            if (mn != m_own[j] && c > rs.c0) need_rescale = true;
+            m_own[j] = mn;
+          }
+          __syncwarp();
+          *reinterpret_cast<float2*>(bc_m + 2 * lane) = make_float2(m_own[0], m_own[1]);
+          *reinterpret_cast<float2*>(bc_m + 64 + 2 * lane) = make_float2(alpha[0], alpha[1]);
         }
         need_rescale = __any_sync(0xffffffffu, need_rescale);
         __syncwarp();
-        float p_[64];
         const float sl2 = p.scale_log2;
+        float pr[32];
 #pragma unroll
-        for (int j = 0; j < 64; j += 4) {
-          float4 mm = *reinterpret_cast<const float4*>(bc_m + j);
-          p_[j] = fast_exp2(fmaf(x[j], sl2, -mm.x)); p_[j + 1] = fast_exp2(fmaf(x[j + 1], sl2, -mm.y));
-          p_[j + 2] = fast_exp2(fmaf(x[j + 2], sl2, -mm.z)); p_[j + 3] = fast_exp2(fmaf(x[j + 3], sl2, -mm.w));
+        for (int cc = 0; cc < 8; ++cc) {
+          const float2 mm = *reinterpret_cast<const float2*>(bc_m + 8 * cc + 2 * (lane & 3));
+          pr[4 * cc + 0] = fast_exp2(fmaf(x[4 * cc + 0], sl2, -mm.x));
+          pr[4 * cc + 1] = fast_exp2(fmaf(x[4 * cc + 1], sl2, -mm.y));
+          pr[4 * cc + 2] = fast_exp2(fmaf(x[4 * cc + 2], sl2, -mm.x));
+          pr[4 * cc + 3] = fast_exp2(fmaf(x[4 * cc + 3], sl2, -mm.y));
         }
-        // P^T row e -> shared memory (MN-major B operand of the PV MMA)
+        // P^T rows rA, rB -> this half chunk's buffer (MN-major B operand of PV),
+        // free once PV(g - 2) has retired
+        if (!wait_bar(&pv_done[sb * NT + NT - 1], ((g >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        const uint32_t pb = smem_u32(sP + sb * kPBuf) + 4 * (lane & 3);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) st_shared16(sP + swz128(e, q), to_bf16x8(p_ + 8 * q));
-        // column sums of this chunk (per-lane ownership, like the maxima)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = p_[32 * h + i];
-#pragma unroll
-          for (int off = 16, n = 32; off >= 1; off >>= 1, n >>= 1) {
-            const bool up = (lane & off) != 0;
-#pragma unroll
-            for (int i = 0; i < n / 2; ++i) {
-              float keep = up ? v[i + n / 2] : v[i];
-              float send = up ? v[i] : v[i + n / 2];
-              v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-            }
-          }
-          l_own[h] = l_own[h] * alpha[h] + v[0];
+        for (int cc = 0; cc < 8; ++cc) {
+          st_shared4(pb + swz128(rA, cc), pack_bf16(pr[4 * cc], pr[4 * cc + 1]));
+          st_shared4(pb + swz128(rB, cc), pack_bf16(pr[4 * cc + 2], pr[4 * cc + 3]));
         }
+        // column sums of this half chunk (same ownership as the maxima)
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          v16[2 * cc] = pr[4 * cc] + pr[4 * cc + 2];
+          v16[2 * cc + 1] = pr[4 * cc + 1] + pr[4 * cc + 3];
+        }
+        const float2 csum = col_reduce16<false>(v16, lane);
+        l_own[0] = l_own[0] * alpha[0] + csum.x;
+        l_own[1] = l_own[1] * alpha[1] + csum.y;
         if (need_rescale) {
-          // O^T columns scale by alpha (this thread is TMEM lane e of every tile)
+          // O^T columns scale by alpha once PV(g - 1) has retired (this thread is
+          // TMEM lane e of every tile)
+          const uint32_t gp = g - 1;
+          if (!wait_bar(&pv_done[(gp & 1) * NT + NT - 1], (gp >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
           for (int tt = 0; tt < NT; ++tt) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               float o[16];
-              const uint32_t ta = tmem + lane_base + 64 + 64 * tt + 16 * q;
+              const uint32_t ta = tmem + lane_base + kOCol + 64 * tt + 16 * q;
               tmem_ld16(ta, o);
               tmem_wait_ld();
 #pragma unroll
@@ -730,20 +744,20 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
         }
         tc_fence_before();
         fence_proxy_async_smem();
-        mbar_arrive(p_full);
+        mbar_arrive(&p_full[sb]);
       }
       if (!ok) break;
       // ---------------- epilogue
       // column sums over the 4 warps
       float* red = s_red + (g & 1) * 256;
-      red[warp * 64 + lane] = l_own[0];
-      red[warp * 64 + 32 + lane] = l_own[1];
+      *reinterpret_cast<float2*>(red + warp * 64 + 2 * lane) = make_float2(l_own[0], l_own[1]);
       named_bar_sync(1, 128);
+      __syncwarp();
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int col = 32 * h + lane;
+      for (int j = 0; j < 2; ++j) {
+        const int col = 2 * lane + j;
         const float lt = red[col] + red[64 + col] + red[128 + col] + red[192 + col];
-        const float lse_w = (lt > 0.f) ? (m_own[h] + log2f(lt)) * kLn2 : -CUDART_INF_F;
+        const float lse_w = (lt > 0.f) ? (m_own[j] + log2f(lt)) * kLn2 : -CUDART_INF_F;
         float cw, cp = 0.f;
         if (EPI == EPI_PARTIAL) {
           cw = lt > 0.f ? 1.f / lt : 0.f;
@@ -763,107 +777,79 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
         bc_m[128 + col] = cp;
       }
       __syncwarp();
-      if (rs.c1 > rs.c0) {
-        for (int tt = 0; tt < NT; ++tt)
-          if (!wait_bar(&pv_done[tt], (g - 1) & 1, abort_flag)) { ok = false; break; }
-        if (!ok) break;
+      const bool any = rs.c1 > rs.c0;
+      if (any) {
+        const uint32_t gl = g - 1;               // last half chunk of this item
+        if (!wait_bar(&pv_done[(gl & 1) * NT + NT - 1], (gl >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
       }
+      // Each thread is TMEM lane e of every O^T tile, i.e. output dim d = 128 tt + e
+      // of all heads: it scales its 64 accumulators by the column coefficients and
+      // writes them straight out (a warp covers 32 consecutive d of one head per
+      // store).  The RoPE dims pair d with d +- 32, held by the other warp of the
+      // last tile's upper half: those 64 threads exchange through shared memory.
       const int64_t obase = (bt * p.n_split + sp) * p.H;   // n_split = 1: token row
-      // Each 128-d tile is written in two halves of 32 heads.  Phase A: every
-      // thread (one TMEM lane = one d) scales its accumulators and stages them
-      // as fp32 [32 heads][128 d] in sP (free once the last PV retired).
-      // Phase B: the 128 threads walk the staged rows in order, add the
-      // compressed-branch partial, apply the inverse RoPE, and store 16-byte
-      // vectors, so every global write is a full, coalesced row segment.
-      float* stage = reinterpret_cast<float*>(sP);
-      const int r0 = D - p.rope_dim;
+      float* xs = reinterpret_cast<float*>(sP);            // [64 heads][64 lanes] exchange
       for (int tt = 0; tt < NT; ++tt) {
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          float o[32];
-          if (rs.c1 > rs.c0) {
-            tmem_ld16(tmem + lane_base + 64 + 64 * tt + 32 * hh, o);
-            tmem_ld16(tmem + lane_base + 64 + 64 * tt + 32 * hh + 16, o + 16);
-            tmem_wait_ld();
+        float o[64];
+        if (any) {
+          tmem_ld32(tmem + lane_base + kOCol + 64 * tt, o);
+          tmem_ld32(tmem + lane_base + kOCol + 64 * tt + 32, o + 32);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) o[i] = 0.f;
+        }
+        if (any && tt == NT - 1) {
+          tc_fence_before();
+          mbar_arrive(epi_done);                           // O^T read: the next item's PV may overwrite it
+        }
+        const int d = 128 * tt + e;
+#pragma unroll
+        for (int h = 0; h < 64; ++h) o[h] *= bc_m[64 + h];
+        if (EPI == EPI_COMBINE && p.O_in) {
+#pragma unroll
+          for (int h = 0; h < 64; ++h)
+            if (h < p.H) o[h] = fmaf(bc_m[128 + h], __ldg(p.O_in + (obase + h) * D + d), o[h]);
+        }
+        if (EPI == EPI_COMBINE && p.inv_rope && tt == NT - 1 && e >= 128 - p.rope_dim) {
+          // inverse rotation by -pos: (a, b) -> (a cos + b sin, -a sin + b cos),
+          // a = dim r0 + j, b = dim r0 + j + half
+          const int half = p.rope_dim / 2;
+          const int lr = e - (128 - p.rope_dim);            // 0 .. rope_dim - 1
+#pragma unroll
+          for (int h = 0; h < 64; ++h) xs[h * 64 + lr] = o[h];
+          named_bar_sync(3, 64);
+          const bool first = lr < half;
+          const int pl = first ? lr + half : lr - half;
+          const float2 csj = cs[first ? lr : lr - half];
+#pragma unroll
+          for (int h = 0; h < 64; ++h) {
+            const float w = xs[h * 64 + pl];
+            o[h] = first ? o[h] * csj.x + w * csj.y : o[h] * csj.x - w * csj.y;
+          }
+        }
+        if (EPI == EPI_COMBINE) {
+          if (p.out_bf16) {
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + obase * D + d;
+#pragma unroll
+            for (int h = 0; h < 64; ++h)
+              if (h < p.H) dst[(int64_t)h * D] = __float2bfloat16_rn(o[h]);
           } else {
+            float* dst = reinterpret_cast<float*>(p.out) + obase * D + d;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+            for (int h = 0; h < 64; ++h)
+              if (h < p.H) dst[(int64_t)h * D] = o[h];
           }
+        } else {
+          float* dst = p.O_part + obase * D + d;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) stage[i * 128 + e] = o[i] * bc_m[64 + 32 * hh + i];
-          named_bar_sync(2, 128);
-          // phase B: 16 threads per head row, 8 consecutive d each
-          const int cl0 = e >> 4, dl = (e & 15) * 8;
-#pragma unroll 1
-          for (int cl = cl0; cl < 32; cl += 8) {
-            const int c = 32 * hh + cl;
-            if (c >= p.H) break;
-            float v[8];
-            const float4 a0 = *reinterpret_cast<const float4*>(stage + cl * 128 + dl);
-            const float4 a1 = *reinterpret_cast<const float4*>(stage + cl * 128 + dl + 4);
-            v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w; v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
-            const int d0 = tt * 128 + dl;
-            const int64_t grow = (obase + c) * D + d0;
-            if (EPI == EPI_COMBINE) {
-              if (p.O_in) {
-                const float cp = bc_m[128 + c];
-                const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.O_in + grow));
-                const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.O_in + grow) + 1);
-                v[0] = fmaf(cp, b0.x, v[0]); v[1] = fmaf(cp, b0.y, v[1]); v[2] = fmaf(cp, b0.z, v[2]);
-                v[3] = fmaf(cp, b0.w, v[3]); v[4] = fmaf(cp, b1.x, v[4]); v[5] = fmaf(cp, b1.y, v[5]);
-                v[6] = fmaf(cp, b1.z, v[6]); v[7] = fmaf(cp, b1.w, v[7]);
-              }
-              if (p.inv_rope && d0 >= r0) {
-                // inverse rotation by -pos: (a, b) -> (a cos + b sin, -a sin + b cos)
-                const int half = p.rope_dim / 2;
-                const int jj0 = d0 - r0;
-                const bool first = jj0 < half;
-                const int pd = dl + (first ? half : -half);
-                float w[8];
-                const float4 c0 = *reinterpret_cast<const float4*>(stage + cl * 128 + pd);
-                const float4 c1 = *reinterpret_cast<const float4*>(stage + cl * 128 + pd + 4);
-                w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w; w[4] = c1.x; w[5] = c1.y; w[6] = c1.z; w[7] = c1.w;
-                if (p.O_in) {
-                  const float cp = bc_m[128 + c];
-                  const int64_t prow = grow + (first ? half : -half);
-                  const float4 e0 = __ldg(reinterpret_cast<const float4*>(p.O_in + prow));
-                  const float4 e1 = __ldg(reinterpret_cast<const float4*>(p.O_in + prow) + 1);
-                  w[0] = fmaf(cp, e0.x, w[0]); w[1] = fmaf(cp, e0.y, w[1]); w[2] = fmaf(cp, e0.z, w[2]);
-                  w[3] = fmaf(cp, e0.w, w[3]); w[4] = fmaf(cp, e1.x, w[4]); w[5] = fmaf(cp, e1.y, w[5]);
-                  w[6] = fmaf(cp, e1.z, w[6]); w[7] = fmaf(cp, e1.w, w[7]);
-                }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float2 csj = cs[(jj0 + i) % half];
-                  v[i] = first ? v[i] * csj.x + w[i] * csj.y : v[i] * csj.x - w[i] * csj.y;
-                }
-              }
-              if (p.out_bf16) {
-                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + grow) = to_bf16x8(v);
-              } else {
-                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + grow);
-                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-              }
-            } else {
-              float4* dst = reinterpret_cast<float4*>(p.O_part + grow);
-              dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-              dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-            }
-          }
-          named_bar_sync(2, 128);   // staging buffer reused by the next half
+          for (int h = 0; h < 64; ++h)
+            if (h < p.H) dst[(int64_t)h * D] = o[h];
         }
       }
-      if (rs.c1 > rs.c0) {
-        tc_fence_before();
-        mbar_arrive(epi_done);
-        ++icount;
-      } else {
-        // keep the cos/sin double buffer in step only for items that used it
-        ++icount;
-      }
-      named_bar_sync(1, 128);   // s_red / bc reuse across items
+      ++icount;
+      named_bar_sync(1, 128);   // s_red / bc / exchange reuse across items
     }
   }
   __syncwarp();                 // reconverge role warps before the CTA barrier
@@ -960,8 +946,8 @@ struct AttnMaps {
 template <int D, int KV, int EPI>
 csa_status_t launch_attn(const AttnParams& p, const AttnMaps& m, cudaStream_t st) {
   constexpr int NS = D / 64, NT = D / 128;
-  const size_t smem = 1024 + NS * (kNQ * 128) + NS * (kRows * 128) + kRows * 128 +
-                      (2 * 4 * 64 + 4 * 3 * 64) * 4 + 64 * 8 + (5 + NS + NT) * 8 + 16;
+  const size_t smem = 1024 + NS * (kNQ * 128) + 2 * NS * (kRows * 128) + 2 * (kRows * 128) +
+                      (2 * 4 * 64 + 4 * 3 * 64) * 4 + 64 * 8 + (9 + 4 * NT) * 8 + 16;
   auto kern = attn_kernel<D, KV, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attention: cannot reserve %zu bytes of shared memory: %s", smem, cudaGetErrorString(e));
@@ -972,7 +958,7 @@ csa_status_t launch_attn(const AttnParams& p, const AttnMaps& m, cudaStream_t st
   return check_launch("attention");
 }
 
-// Builds the tile maps that apply (bf16 rows, 64 x 128-row boxes, 128-byte
+// Builds the tile maps that apply (bf16 rows, 64 x 64-row boxes, 128-byte
 // swizzle) and sets the matching flags; other maps stay zero and unused.
 csa_status_t build_maps(AttnParams& p, AttnMaps& m, int D, csa_dtype_t q_dtype, csa_dtype_t kv_dtype,
                         csa_dtype_t tok_dtype) {

@@ -68,12 +68,11 @@ struct IdxParams {
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  // a few tight polls, then back off with nanosleep so that waiting warps do not
-  // flood the shared-memory pipe that the loads and stores of other warps use
+  // mbarrier.try_wait suspends in hardware until the phase completes (or a short
+  // system time limit passes); the clock and the abort flag are read every 64 polls
   uint64_t start = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (i > 8) __nanosleep(i < 64 ? 32 : 128);
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
       const uint64_t now = global_ns();
