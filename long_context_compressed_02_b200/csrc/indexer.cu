@@ -65,7 +65,33 @@ struct IdxParams {
   float* scores;          // [n_seq, T, cap]
   int64_t cap;
   int T, HI, DI, m, TQ, N, tiles_per_chunk;
+  int n_seq, n_qblocks;
+  int64_t n_items;        // n_seq x n_qblocks x key chunks
 };
+
+// One work item of the persistent scores kernel: a key chunk of one token
+// block of one sequence.  Items run sequence-fastest, then token block (the
+// latest, longest blocks first), then key chunk, so that a CTA's grid-stride
+// share mixes long and short rows.
+struct IdxItem {
+  int b, t0, tile0, n_tiles;
+  int64_t pos0;
+};
+__device__ __forceinline__ IdxItem idx_item(const IdxParams& p, int64_t item) {
+  IdxItem r;
+  r.b = (int)(item % p.n_seq);
+  const int64_t rest = item / p.n_seq;
+  const int qb = p.n_qblocks - 1 - (int)(rest % p.n_qblocks);
+  const int chunk = (int)(rest / p.n_qblocks);
+  r.t0 = qb * p.TQ;
+  const int t_last = min(p.T, r.t0 + p.TQ) - 1;
+  r.pos0 = p.q_pos[r.b];
+  const int64_t nv_max = min(p.cap, (r.pos0 + t_last + 1) / p.m);
+  const int n_tiles_all = (int)((nv_max + 127) / 128);
+  r.tile0 = chunk * p.tiles_per_chunk;
+  r.n_tiles = max(0, min(n_tiles_all - r.tile0, p.tiles_per_chunk));
+  return r;
+}
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   // mbarrier.try_wait suspends in hardware until the phase completes (or a short
@@ -97,54 +123,36 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   extern __shared__ uint8_t smem_raw[];
   // aligned by offsetting the shared array itself, so accesses stay in the shared window
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const int b = blockIdx.z, qb = blockIdx.y, chunk = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t0 = qb * p.TQ;
-  const int t_last = min(p.T, t0 + p.TQ) - 1;
-  const int64_t pos0 = p.q_pos[b];
-  const int64_t nv_max = min(p.cap, (pos0 + t_last + 1) / p.m);
-  const int n_tiles_all = (int)((nv_max + 127) / 128);
-  const int tile0 = chunk * p.tiles_per_chunk;
-  const int n_tiles = min(n_tiles_all - tile0, p.tiles_per_chunk);
-  if (n_tiles <= 0) return;
 
   const uint32_t a_bytes = 128u * p.DI;
   const uint32_t b_bytes = (uint32_t)p.N * p.DI;
-  uint8_t* sB = smem;
-  uint8_t* sA = smem + ((b_bytes + 1023u) & ~1023u);
+  const uint32_t b_stride = (b_bytes + 1023u) & ~1023u;
+  uint8_t* sB = smem;                                         // [2] query tiles (item parity)
+  uint8_t* sA = smem + 2 * b_stride;                          // [kStages] key tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sA + kStages * a_bytes);
   uint64_t* full = bars;                 // [kStages]
   uint64_t* empty = bars + kStages;      // [kStages]
   uint64_t* tfull = bars + 2 * kStages;  // [2]
   uint64_t* tempty = tfull + 2;          // [2]
-  uint64_t* qbar = tempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(qbar + 1);
+  uint64_t* qfull = tempty + 2;          // [2]
+  uint64_t* qempty = qfull + 2;          // [2]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(qempty + 2);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
-  int* s_nv = s_abort + 1;                                    // [TQ] visible entries per token
+  // per epilogue group and item parity: visible entries per token, column weights w * qs
+  int* s_nv = s_abort + 1;                                    // [2 groups][2][TQ]
   float* s_w = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(s_nv + p.TQ) + 15) & ~uintptr_t(15));   // [N] = w * qs per column
+      (reinterpret_cast<uintptr_t>(s_nv + 4 * p.TQ) + 15) & ~uintptr_t(15));   // [2 groups][2][N]
 
   const uint32_t tmem_cols = p.N <= 16 ? 32u : (p.N <= 32 ? 64u : (p.N <= 64 ? 128u : (p.N <= 128 ? 256u : 512u)));
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiThreads / 2); }
-    mbar_init(qbar, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiThreads / 2);
+      mbar_init(&qfull[a], 1); mbar_init(&qempty[a], 1);
+    }
     *s_abort = 0;
     fence_mbar_init();
-  }
-  for (int c = tid; c < p.N; c += kIdxThreads) {
-    const int tq = c / p.HI, h = c % p.HI;
-    const int t = t0 + tq;
-    float v = 0.f;
-    if (t < p.T) {
-      const int64_t o = ((int64_t)b * p.T + t) * p.HI + h;
-      v = p.w[o] * (p.qs ? p.qs[o] : 1.f);
-    }
-    s_w[c] = v;
-  }
-  for (int tq = tid; tq < p.TQ; tq += kIdxThreads) {
-    const int t = t0 + tq;
-    s_nv[tq] = t < p.T ? (int)min(p.cap, (pos0 + t + 1) / p.m) : 0;
   }
   if (warp == 1) tmem_alloc(s_tmem, tmem_cols);
   tc_fence_before();
@@ -156,19 +164,31 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   const uint32_t swz = p.DI == 128 ? SWZ_128B : (p.DI == 64 ? SWZ_64B : SWZ_32B);
   const uint32_t sbo = 8u * p.DI;
 
+  // Every role walks the same item sequence; the key-tile ring (stage, phase),
+  // the accumulator pair and the query-tile pair all continue across items.
   if (warp == 0) {
     // ---------------- TMA producer (lane 0)
     if (lane == 0) {
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_q);
-      mbar_expect_tx(qbar, b_bytes);
-      tma_load_2d(sB, &tmap_q, 0, (int32_t)(((int64_t)b * p.T + t0) * p.HI), qbar);
-      for (int it = 0; it < n_tiles; ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!wait_bar(&empty[s], ph ^ 1, abort_flag)) break;
-        mbar_expect_tx(&full[s], a_bytes);
-        tma_load_2d(sA + s * a_bytes, &tmap_k, 0, (int32_t)((int64_t)b * p.cap + (int64_t)(tile0 + it) * 128), &full[s]);
+      uint32_t gt = 0, ic = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const IdxItem it = idx_item(p, item);
+        if (it.n_tiles == 0) continue;
+        const uint32_t qs = ic & 1;
+        if (!wait_bar(&qempty[qs], ((ic >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(&qfull[qs], b_bytes);
+        tma_load_2d(sB + qs * b_stride, &tmap_q, 0, (int32_t)(((int64_t)it.b * p.T + it.t0) * p.HI), &qfull[qs]);
+        for (int j = 0; j < it.n_tiles; ++j, ++gt) {
+          const int s = gt % kStages;
+          const uint32_t ph = (gt / kStages) & 1;
+          if (!wait_bar(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&full[s], a_bytes);
+          tma_load_2d(sA + s * a_bytes, &tmap_k, 0, (int32_t)((int64_t)it.b * p.cap + (int64_t)(it.tile0 + j) * 128),
+                      &full[s]);
+        }
+        ++ic;
       }
     }
   } else if (warp == 1) {
@@ -177,16 +197,23 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       const uint32_t idesc = make_idesc(128, p.N, 0, 0, 0, 0);
       // base descriptors once; each MMA only adds a start-address offset (>> 4)
       const uint64_t dA = smem_desc(smem_u32(sA), 16, sbo, swz);
-      const uint64_t dB = smem_desc(smem_u32(sB), 16, sbo, swz);
+      const uint64_t dB0 = smem_desc(smem_u32(sB), 16, sbo, swz);
       const int nk = p.DI / 32;
-      if (wait_bar(qbar, 0, abort_flag)) {
-        for (int it = 0; it < n_tiles; ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          const int acc = it & 1;
-          const uint32_t aph = (it >> 1) & 1;
-          if (!wait_bar(&full[s], ph, abort_flag)) break;
-          if (!wait_bar(&tempty[acc], aph ^ 1, abort_flag)) break;
+      uint32_t gt = 0, ic = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const IdxItem it = idx_item(p, item);
+        if (it.n_tiles == 0) continue;
+        const uint32_t qs = ic & 1;
+        if (!wait_bar(&qfull[qs], (ic >> 1) & 1, abort_flag)) { ok = false; break; }
+        const uint64_t dB = dB0 + ((qs * b_stride) >> 4);
+        for (int j = 0; j < it.n_tiles; ++j, ++gt) {
+          const int s = gt % kStages;
+          const uint32_t ph = (gt / kStages) & 1;
+          const int acc = gt & 1;
+          const uint32_t aph = (gt >> 1) & 1;
+          if (!wait_bar(&full[s], ph, abort_flag)) { ok = false; break; }
+          if (!wait_bar(&tempty[acc], aph ^ 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint64_t dAs = dA + ((s * a_bytes) >> 4);
           const uint32_t d = tmem + acc * p.N;
@@ -199,6 +226,9 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
           mma_commit(&empty[s]);
           mma_commit(&tfull[acc]);
         }
+        if (!ok) break;
+        mma_commit(&qempty[qs]);          // the query tile may be reloaded once these MMAs retire
+        ++ic;
       }
     }
   } else {
@@ -208,65 +238,97 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     const int ew = warp - 2;
     const int sp = warp & 3;
     const int grp = ew >> 2;
+    const int gtid = tid - 64 - 128 * grp;    // 0 .. 127 within the group
     const int log2hi = __ffs(p.HI) - 1;
-    const uint32_t w_addr = smem_u32(s_w);
     const int key_in_tile = sp * 32 + lane;
-    auto key_scale = [&](int it) -> float {
-      const int64_t key = (int64_t)(tile0 + it) * 128 + key_in_tile;
-      return (key < p.cap && it < n_tiles) ? (p.ks ? __ldg(p.ks + (int64_t)b * p.cap + key) : 1.f) : 0.f;
-    };
-    float ksc_next = key_scale(grp);
-    for (int it = grp; it < n_tiles; it += 2) {
-      const int acc = grp;
-      const uint32_t aph = (it >> 1) & 1;
-      const int64_t key = (int64_t)(tile0 + it) * 128 + key_in_tile;
-      const float ksc = ksc_next;
-      ksc_next = key_scale(it + 2);          // issued a tile ahead: off the critical path
-      if (!wait_bar(&tfull[acc], aph, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t tb = tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N;
-      float run = 0.f;
-      for (int cc = 0; cc < p.N; cc += 32) {
-        float v[32];
-        tmem_ld32(tb + cc, v);
-        tmem_wait_ld();
-        float pr[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 w4 = ld_shared_f4(w_addr + (cc + 4 * i) * 4);
-          pr[4 * i + 0] = w4.x * fmaxf(v[4 * i + 0], 0.f);
-          pr[4 * i + 1] = w4.y * fmaxf(v[4 * i + 1], 0.f);
-          pr[4 * i + 2] = w4.z * fmaxf(v[4 * i + 2], 0.f);
-          pr[4 * i + 3] = w4.w * fmaxf(v[4 * i + 3], 0.f);
+    uint32_t gt = 0, ic = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const IdxItem it = idx_item(p, item);
+      if (it.n_tiles == 0) continue;
+      // this group's copy of the block's column weights and visible-entry
+      // counts, double-buffered by item parity (the other buffer may still be
+      // read by a thread of this group finishing the previous item)
+      float* gw = s_w + (2 * grp + (ic & 1)) * p.N;
+      int* gnv = s_nv + (2 * grp + (ic & 1)) * p.TQ;
+      ++ic;
+      for (int c = gtid; c < p.N; c += 128) {
+        const int tq = c / p.HI, h = c % p.HI;
+        const int t = it.t0 + tq;
+        float v = 0.f;
+        if (t < p.T) {
+          const int64_t o = ((int64_t)it.b * p.T + t) * p.HI + h;
+          v = p.w[o] * (p.qs ? p.qs[o] : 1.f);
         }
-        // pairwise sums inside each group of min(HI, 32) head columns
+        gw[c] = v;
+      }
+      for (int tq = gtid; tq < p.TQ; tq += 128) {
+        const int t = it.t0 + tq;
+        gnv[tq] = t < p.T ? (int)min(p.cap, (it.pos0 + t + 1) / p.m) : 0;
+      }
+      named_bar_sync(1 + grp, 128);
+      const uint32_t w_addr = smem_u32(gw);
+      // this group's tiles of the item: global tile numbers gt with gt % 2 == grp
+      const int j0 = ((int)(gt & 1) == grp) ? 0 : 1;
+      auto key_scale = [&](int j) -> float {
+        const int64_t key = (int64_t)(it.tile0 + j) * 128 + key_in_tile;
+        return (key < p.cap && j < it.n_tiles) ? (p.ks ? __ldg(p.ks + (int64_t)it.b * p.cap + key) : 1.f) : 0.f;
+      };
+      float ksc_next = key_scale(j0);
+      for (int j = j0; j < it.n_tiles; j += 2) {
+        const uint32_t g = gt + j;
+        const int acc = grp;
+        const uint32_t aph = (g >> 1) & 1;
+        const int64_t key = (int64_t)(it.tile0 + j) * 128 + key_in_tile;
+        const float ksc = ksc_next;
+        ksc_next = key_scale(j + 2);          // issued a tile ahead: off the critical path
+        if (!wait_bar(&tfull[acc], aph, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tb = tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N;
+        float run = 0.f;
+        for (int cc = 0; cc < p.N; cc += 32) {
+          float v[32];
+          tmem_ld32(tb + cc, v);
+          tmem_wait_ld();
+          float pr[32];
 #pragma unroll
-        for (int lv = 0; lv < 5; ++lv) {
-          const int w = 1 << lv;
-          if (w < p.HI) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 2 * w) pr[i] += pr[i + w];
+          for (int i = 0; i < 8; ++i) {
+            const float4 w4 = ld_shared_f4(w_addr + (cc + 4 * i) * 4);
+            pr[4 * i + 0] = w4.x * fmaxf(v[4 * i + 0], 0.f);
+            pr[4 * i + 1] = w4.y * fmaxf(v[4 * i + 1], 0.f);
+            pr[4 * i + 2] = w4.z * fmaxf(v[4 * i + 2], 0.f);
+            pr[4 * i + 3] = w4.w * fmaxf(v[4 * i + 3], 0.f);
           }
-        }
-        if (p.HI >= 32) {
-          run += pr[0];
-          if (((cc + 32) & (p.HI - 1)) == 0) {
-            const int tq = (cc + 31) >> log2hi;
-            if (key < s_nv[tq]) p.scores[((int64_t)b * p.T + t0 + tq) * p.cap + key] = run * ksc;
-            run = 0.f;
-          }
-        } else {
+          // pairwise sums inside each group of min(HI, 32) head columns
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if ((j & (p.HI - 1)) == 0) {
-              const int tq = (cc + j) >> log2hi;
-              if (key < s_nv[tq]) p.scores[((int64_t)b * p.T + t0 + tq) * p.cap + key] = pr[j] * ksc;
+          for (int lv = 0; lv < 5; ++lv) {
+            const int w = 1 << lv;
+            if (w < p.HI) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 2 * w) pr[i] += pr[i + w];
+            }
+          }
+          if (p.HI >= 32) {
+            run += pr[0];
+            if (((cc + 32) & (p.HI - 1)) == 0) {
+              const int tq = (cc + 31) >> log2hi;
+              if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = run * ksc;
+              run = 0.f;
+            }
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+              if ((jj & (p.HI - 1)) == 0) {
+                const int tq = (cc + jj) >> log2hi;
+                if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = pr[jj] * ksc;
+              }
             }
           }
         }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      gt += it.n_tiles;
     }
   }
   __syncwarp();                 // reconverge role warps before the CTA barrier
@@ -282,6 +344,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
 constexpr int kTopkThreads = 512;
 constexpr int kChunk = 16384;          // keys per shared-memory chunk (64 KB)
 constexpr int kMergeCap = 16384;       // candidates per row in the merge stage
+constexpr int kHistBins = 4096;        // rows split into chunks: histogram of the top 12 key bits
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f + 0.0f);   // -0 -> +0 so that equal values tie
@@ -427,13 +490,72 @@ struct TopkParams {
   uint32_t* cand_key;      // [rows, n_chunks, k]
   int32_t* cand_idx;       // [rows, n_chunks, k]
   int32_t* cand_cnt;       // [rows, n_chunks]
+  uint32_t* hist;          // [rows, kHistBins] (rows split into chunks)
 };
 
-// Stage 1 (or the only stage when n_chunks == 1): one CTA per (chunk, row).
+// Rows split into chunks, pass 1: histogram of the top 12 bits of every
+// visible key of the row, one CTA per (row, chunk), merged in global memory.
 __global__ void __launch_bounds__(kTopkThreads)
+topk_hist_kernel(TopkParams p) {
+  __shared__ uint32_t h[kHistBins];
+  const int64_t row = blockIdx.x;
+  const int chunk = blockIdx.y;
+  const int b = (int)(row / p.T), t = (int)(row % p.T);
+  const int64_t nv = min(p.cap, (p.q_pos[b] + t + 1) / p.m);
+  const int64_t lo = (int64_t)chunk * kChunk;
+  const int n = (int)max((int64_t)0, min((int64_t)kChunk, nv - lo));
+  if (n == 0) return;
+  for (int i = threadIdx.x; i < kHistBins; i += kTopkThreads) h[i] = 0;
+  __syncthreads();
+  const float* src = p.scores + row * p.cap + lo;
+  for (int e = threadIdx.x; e < n; e += kTopkThreads) atomicAdd(&h[order_key(src[e]) >> 20], 1u);
+  __syncthreads();
+  uint32_t* g = p.hist + row * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += kTopkThreads)
+    if (h[i]) atomicAdd(&g[i], h[i]);
+}
+
+// The row's threshold bin: the highest bin B such that bins >= B hold at least
+// k keys (0 when the row has fewer than k keys).  No key of a lower bin can be
+// among the row's top k.  All threads call; the result is broadcast.  Thread t
+// owns the 8 bins [4096 - 8 (t + 1), 4096 - 8 t), so a prefix scan in thread
+// order counts the keys in higher bins.
+__device__ uint32_t topk_threshold_bin(const uint32_t* g, int k, SelectSmem& ss, uint32_t* s_out) {
+  constexpr int kPer = kHistBins / kTopkThreads;         // 8
+  const int tid = threadIdx.x;
+  const int top = kHistBins - kPer * tid;
+  uint32_t c[kPer], s = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) { c[i] = g[top - 1 - i]; s += c[i]; }
+  if (tid == 0) *s_out = 0;
+  const uint64_t incl = block_scan_incl((uint64_t)s, ss);   // syncs: the reset above is visible
+  const uint32_t excl = (uint32_t)incl - s;
+  if (excl < (uint32_t)k && (uint32_t)k <= (uint32_t)incl) {
+    uint32_t cum = excl;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      cum += c[i];
+      if (cum >= (uint32_t)k) { *s_out = (uint32_t)(top - 1 - i); break; }
+    }
+  }
+  __syncthreads();
+  const uint32_t B = *s_out;
+  __syncthreads();
+  return B;
+}
+
+// Stage 1 (or the only stage when n_chunks == 1): one CTA per (chunk, row).
+// With several chunks, only keys in or above the row's threshold bin (from
+// the histogram pass) can be selected: they are compacted in index order
+// first, so the local selection runs on a few hundred keys.
+// (Two instances, so that the filtered path's extra state does not cost the
+// single-chunk path occupancy.)
+template <bool FILTERED>
+__global__ void __launch_bounds__(kTopkThreads, FILTERED ? 2 : 4)
 topk_chunk_kernel(TopkParams p) {
-  extern __shared__ uint32_t s_keys[];   // kChunk
+  extern __shared__ uint32_t s_keys[];   // kChunk keys (or kChunk / 2 keys + kChunk / 2 ids)
   __shared__ SelectSmem ss;
+  __shared__ uint32_t s_B;
   const int64_t row = blockIdx.x;
   const int chunk = blockIdx.y;
   const int b = (int)(row / p.T), t = (int)(row % p.T);
@@ -441,16 +563,68 @@ topk_chunk_kernel(TopkParams p) {
   const int64_t lo = (int64_t)chunk * kChunk;
   const int n = (int)max((int64_t)0, min((int64_t)kChunk, nv - lo));
   const float* src = p.scores + row * p.cap + lo;
-  for (int e = threadIdx.x; e < n; e += kTopkThreads) s_keys[e] = order_key(src[e]);
-  __syncthreads();
-  if (p.n_chunks == 1) {
+  if constexpr (!FILTERED) {
+    for (int e = threadIdx.x; e < n; e += kTopkThreads) s_keys[e] = order_key(src[e]);
+    __syncthreads();
     int32_t* out = p.idx + row * p.k;
     int cnt = block_select(s_keys, nullptr, lo, n, p.k, out, nullptr, ss);
     for (int i = cnt + threadIdx.x; i < p.k; i += kTopkThreads) out[i] = -1;
+    return;
   } else {
+    // Only keys in or above the row's threshold bin can be selected.  Warp w
+    // owns the 1024 consecutive keys [1024 w, 1024 w + 1024) of the chunk: a
+    // counting pass (ballots) gives each warp its output offset, then a writing
+    // pass emits the survivors in index order.
+    __shared__ uint32_t s_wcnt[kTopkThreads / 32];
+    constexpr int kWarps = kTopkThreads / 32;
+    constexpr int kPerWarp = kChunk / kWarps;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t B = topk_threshold_bin(p.hist + row * kHistBins, p.k, ss, &s_B);
+    const int w0 = warp * kPerWarp;
+    uint32_t cnt = 0;
+    for (int j = 0; j < kPerWarp; j += 32) {
+      const int e = w0 + j + lane;
+      const bool pass = e < n && (order_key(src[e]) >> 20) >= B;
+      cnt += __popc(__ballot_sync(0xffffffffu, pass));
+    }
+    if (lane == 0) s_wcnt[warp] = cnt;
+    __syncthreads();
+    uint32_t off = 0, n_f = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) { const uint32_t c = s_wcnt[w]; off += w < warp ? c : 0u; n_f += c; }
     const int64_t o = (row * p.n_chunks + chunk) * p.k;
-    int cnt = block_select(s_keys, nullptr, lo, n, p.k, p.cand_idx + o, p.cand_key + o, ss);
-    if (threadIdx.x == 0) p.cand_cnt[row * p.n_chunks + chunk] = cnt;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    if (n_f <= (uint32_t)p.k || n_f <= (uint32_t)(kChunk / 2)) {
+      // every survivor is a candidate (written straight out), or the local
+      // top-k is taken among the survivors staged in shared memory
+      const bool direct = n_f <= (uint32_t)p.k;
+      int32_t* s_ids = reinterpret_cast<int32_t*>(s_keys + kChunk / 2);
+      for (int j = 0; j < kPerWarp; j += 32) {
+        const int e = w0 + j + lane;
+        const uint32_t key = e < n ? order_key(src[e]) : 0u;
+        const bool pass = e < n && (key >> 20) >= B;
+        const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+        if (pass) {
+          const uint32_t pos = off + __popc(bal & lt_mask);
+          if (direct) { p.cand_key[o + pos] = key; p.cand_idx[o + pos] = (int32_t)(lo + e); }
+          else { s_keys[pos] = key; s_ids[pos] = (int32_t)(lo + e); }
+        }
+        off += __popc(bal);
+      }
+      if (direct) {
+        if (threadIdx.x == 0) p.cand_cnt[row * p.n_chunks + chunk] = (int)n_f;
+        return;
+      }
+      __syncthreads();
+      const int c = block_select(s_keys, s_ids, 0, (int)n_f, p.k, p.cand_idx + o, p.cand_key + o, ss);
+      if (threadIdx.x == 0) p.cand_cnt[row * p.n_chunks + chunk] = c;
+      return;
+    }
+    // many keys share the threshold bin: local top-k of the whole chunk by position
+    for (int e = threadIdx.x; e < n; e += kTopkThreads) s_keys[e] = order_key(src[e]);
+    __syncthreads();
+    const int c = block_select(s_keys, nullptr, lo, n, p.k, p.cand_idx + o, p.cand_key + o, ss);
+    if (threadIdx.x == 0) p.cand_cnt[row * p.n_chunks + chunk] = c;
   }
 }
 
@@ -464,19 +638,47 @@ topk_merge_kernel(TopkParams p) {
   __shared__ SelectSmem ss;
   __shared__ int s_off[65];
   const int64_t row = blockIdx.x;
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int c = 0; c < p.n_chunks; ++c) { s_off[c] = acc; acc += p.cand_cnt[row * p.n_chunks + c]; }
-    s_off[p.n_chunks] = acc;
+  if (threadIdx.x < 64) {
+    // chunk offsets: the (<= 64) counts are loaded in parallel and scanned by two warps
+    const int c = threadIdx.x;
+    const int v = c < p.n_chunks ? p.cand_cnt[row * p.n_chunks + c] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int nn = __shfl_up_sync(0xffffffffu, incl, o);
+      if ((c & 31) >= o) incl += nn;
+    }
+    if (c == 31) s_off[64] = incl;                       // first warp's total (scratch)
+    s_off[c] = incl - v;                                  // exclusive, within the warp
   }
   __syncthreads();
+  if (threadIdx.x >= 32 && threadIdx.x < 64) s_off[threadIdx.x] += s_off[64];
+  __syncthreads();
+  if (threadIdx.x == 0) s_off[p.n_chunks] = (p.n_chunks == 64) ? s_off[63] + p.cand_cnt[row * p.n_chunks + 63]
+                                                             : s_off[p.n_chunks];
+  __syncthreads();
   const int n = s_off[p.n_chunks];
-  for (int c = 0; c < p.n_chunks; ++c) {
-    const int cnt = s_off[c + 1] - s_off[c];
-    const int64_t o = (row * p.n_chunks + c) * p.k;
-    for (int i = threadIdx.x; i < cnt; i += kTopkThreads) {
-      s_keys[s_off[c] + i] = p.cand_key[o + i];
-      s_ids[s_off[c] + i] = p.cand_idx[o + i];
+  // one flat pass over all candidates (chunk found by binary search on the
+  // offsets), loads batched ahead of the stores so that they overlap
+  constexpr int kBatch = 4;
+  for (int i0 = threadIdx.x; i0 < n; i0 += kBatch * kTopkThreads) {
+    uint32_t kk[kBatch];
+    int32_t id[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * kTopkThreads;
+      if (i < n) {
+        int lo = 0, hi = p.n_chunks - 1;                 // last chunk c with s_off[c] <= i
+        while (lo < hi) { const int mid = (lo + hi + 1) >> 1; if (s_off[mid] <= i) lo = mid; else hi = mid - 1; }
+        const int64_t src = (row * p.n_chunks + lo) * p.k + (i - s_off[lo]);
+        kk[u] = p.cand_key[src];
+        id[u] = p.cand_idx[src];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * kTopkThreads;
+      if (i < n) { s_keys[i] = kk[u]; s_ids[i] = id[u]; }
     }
   }
   __syncthreads();
@@ -486,7 +688,7 @@ topk_merge_kernel(TopkParams p) {
 }
 
 struct WsLayout {
-  size_t scores, cand_key, cand_idx, cand_cnt, total;
+  size_t scores, cand_key, cand_idx, cand_cnt, hist, total;
   int n_chunks;
 };
 
@@ -502,6 +704,7 @@ WsLayout ws_layout(int n_seq, int T, int64_t cap, int k) {
     L.cand_key = off; off = align_up(off + rows * L.n_chunks * (size_t)k * 4, 256);
     L.cand_idx = off; off = align_up(off + rows * L.n_chunks * (size_t)k * 4, 256);
     L.cand_cnt = off; off = align_up(off + rows * L.n_chunks * 4, 256);
+    L.hist = off; off = align_up(off + rows * (size_t)kHistBins * 4, 256);
   }
   L.total = off;
   return L;
@@ -555,23 +758,27 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
 
   const int n_qblocks = (T + TQ - 1) / TQ;
   const int64_t tiles = (cap + 127) / 128;
-  int64_t n_kchunks = 1;
-  const int64_t ctas = (int64_t)n_seq * n_qblocks;
   const int sms = num_sms();
-  if (ctas < sms) n_kchunks = std::max<int64_t>(1, std::min<int64_t>(tiles, sms / ctas));
-  ip.tiles_per_chunk = (int)((tiles + n_kchunks - 1) / n_kchunks);
-  n_kchunks = (tiles + ip.tiles_per_chunk - 1) / ip.tiles_per_chunk;
-  CSA_REQUIRE(n_qblocks <= 65535 && n_seq <= 65535, "csa_index_topk: grid too large");
-
+  // key chunks: one per token block when there are many blocks (prefill);
+  // otherwise about 4 chunks per SM at full row length (decode), so that
+  // rows of unequal length spread over every CTA of the persistent grid
+  const int64_t rows_blocks = (int64_t)n_seq * n_qblocks;
+  int64_t chunk_tiles = tiles;
+  if (rows_blocks < 2 * (int64_t)sms)
+    chunk_tiles = std::max<int64_t>(8, std::min<int64_t>(tiles, (rows_blocks * tiles + 4 * sms - 1) / (4 * sms)));
+  ip.tiles_per_chunk = (int)chunk_tiles;
+  const int64_t n_kchunks = (tiles + chunk_tiles - 1) / chunk_tiles;
+  ip.n_seq = n_seq; ip.n_qblocks = n_qblocks;
+  ip.n_items = rows_blocks * n_kchunks;
   CUtensorMap mk, mq;
   if (!make_byte_map(&mk, kI, (uint64_t)n_seq * cap, DI, 128) ||
       !make_byte_map(&mq, qI, (uint64_t)n_seq * T * HI, DI, N))
     return fail(CSA_ERR_CUDA, "csa_index_topk: cuTensorMapEncodeTiled failed");
 
-  const size_t smem = 1024 + ((N * DI + 1023) / 1024) * 1024 + (size_t)kStages * 128 * DI +
-                      (2 * kStages + 5) * 8 + 8 + TQ * 4 + 16 + N * 4;
+  const size_t smem = 1024 + 2 * (((size_t)N * DI + 1023) / 1024) * 1024 + (size_t)kStages * 128 * DI +
+                      (2 * kStages + 8) * 8 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4;
   cudaFuncSetAttribute(indexer_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  dim3 grid((unsigned)n_kchunks, (unsigned)n_qblocks, (unsigned)n_seq);
+  const int grid = (int)std::min<int64_t>(ip.n_items, sms);
   indexer_scores_kernel<<<grid, kIdxThreads, smem, stream>>>(mk, mq, ip);
   csa_status_t st = check_launch("csa_index_topk(scores)");
   if (st != CSA_OK) return st;
@@ -582,13 +789,24 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
   tp.cand_key = reinterpret_cast<uint32_t*>(ws + L.cand_key);
   tp.cand_idx = reinterpret_cast<int32_t*>(ws + L.cand_idx);
   tp.cand_cnt = reinterpret_cast<int32_t*>(ws + L.cand_cnt);
+  tp.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
   const int64_t rows = (int64_t)n_seq * T;
   CSA_REQUIRE(rows <= 0x7fffffff, "csa_index_topk: too many rows");
-  // key buffer sized to the longest chunk actually present (rows of <= 16384 entries)
-  const size_t smem1 = (size_t)std::min<int64_t>(kChunk, cap) * sizeof(uint32_t);
-  cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  // key buffer sized to the longest chunk actually present (rows of <= 16384
+  // entries); rows split into chunks also hold the filtered keys' indices
+  const size_t smem1 = L.n_chunks > 1 ? (size_t)kChunk * sizeof(uint32_t)
+                                      : (size_t)std::min<int64_t>(kChunk, cap) * sizeof(uint32_t);
+  auto chunk_kernel = L.n_chunks > 1 ? topk_chunk_kernel<true> : topk_chunk_kernel<false>;
+  cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   dim3 g1((unsigned)rows, (unsigned)L.n_chunks);
-  topk_chunk_kernel<<<g1, kTopkThreads, smem1, stream>>>(tp);
+  if (L.n_chunks > 1) {
+    cudaError_t e = cudaMemsetAsync(tp.hist, 0, (size_t)rows * kHistBins * sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_index_topk: histogram reset failed: %s", cudaGetErrorString(e));
+    topk_hist_kernel<<<g1, kTopkThreads, 0, stream>>>(tp);
+    st = check_launch("csa_index_topk(histogram)");
+    if (st != CSA_OK) return st;
+  }
+  chunk_kernel<<<g1, kTopkThreads, smem1, stream>>>(tp);
   st = check_launch("csa_index_topk(select)");
   if (st != CSA_OK) return st;
   if (L.n_chunks > 1) {
