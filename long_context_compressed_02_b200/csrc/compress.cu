@@ -13,6 +13,7 @@
 // moves them with 16-byte (bf16) or 2 x 16-byte (fp32) vector loads, so a group
 // of D/8 threads reads one row with fully coalesced transactions.  No tensor
 // cores: there is no contraction here.
+#include <cmath>
 #include <cuda_bf16.h>
 #include <math_constants.h>
 #include "common.cuh"
@@ -195,24 +196,37 @@ __device__ __forceinline__ float2 rope_cs_fast(int64_t pos, int j, int rope_dim,
   return make_float2(cs, sn);
 }
 
+// cos / sin of pos * theta_j with theta_j = ratio^j (ratio = base^(-2/rope_dim),
+// computed on the host in double): the power by squaring and the angle
+// reduction stay in double, so angles at positions near 2^20 keep ~1e-9 rad.
+__device__ __forceinline__ float2 rope_cs_pow(int64_t pos, int j, double ratio) {
+  double inv_freq = 1.0, base = ratio;
+  for (int e = j; e > 0; e >>= 1) {
+    if (e & 1) inv_freq *= base;
+    base *= base;
+  }
+  double a = (double)pos * inv_freq;
+  a -= floor(a * 0.15915494309189535) * 6.283185307179586;
+  float sn, cs;
+  sincosf((float)a, &sn, &cs);
+  return make_float2(cs, sn);
+}
+
 // Rows of `rows_per_pos` share one position; a CTA handles `ppb` positions.
 // A warp normalises two rows at a time; lane owns D/32 consecutive channels.
 // Lanes holding RoPE dims also load their partner channels (d -+ half) directly,
-// so the rotation needs no cross-lane exchange.
+// so the rotation needs no cross-lane exchange.  Each warp issues its first
+// rows' loads before the CTA builds its cos/sin table, so the table's math
+// overlaps the memory latency.
 template <typename Tin, typename Tout, int CPL>
 __global__ void __launch_bounds__(kThreads)
 rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int D, int rows_per_pos, int64_t pos0,
-                    int ppb, int norm, int rope_dim, float rope_base, float eps, Tout* __restrict__ out) {
+                    int ppb, int norm, int rope_dim, double ratio, float eps, Tout* __restrict__ out) {
   constexpr int RPW = 2;
   __shared__ float2 s_cs[32][32];   // [position in CTA][pair]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t p_first = (int64_t)blockIdx.x * ppb;
   const int half = rope_dim / 2;
-  for (int e = tid; e < ppb * half; e += kThreads) {
-    const int pl = e / half, j = e % half;
-    s_cs[pl][j] = rope_cs_fast(pos0 + p_first + pl, j, rope_dim, rope_base);
-  }
-  __syncthreads();
   const int64_t r_begin = p_first * rows_per_pos;
   const int64_t r_end = min(rows, (p_first + ppb) * rows_per_pos);
   const int r0d = D - rope_dim;
@@ -220,8 +234,8 @@ rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int D, int rows_per
   const bool in_rope = rope_dim > 0 && d0 >= r0d;
   const bool first_half = d0 < r0d + half;
   const int pd0 = first_half ? d0 + half : d0 - half;     // partner channels
-  for (int64_t rb = r_begin + warp * RPW; rb < r_end; rb += (kThreads / 32) * RPW) {
-    float v[RPW][CPL], u[RPW][CPL];
+  float v[RPW][CPL], u[RPW][CPL];
+  auto load_rows = [&](int64_t rb) {
 #pragma unroll
     for (int k = 0; k < RPW; ++k) {
       const int64_t r = min(rb + k, r_end - 1);
@@ -232,6 +246,15 @@ rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int D, int rows_per
         for (int c = 0; c < CPL; c += 8) Vec8<Tin>::load(x + r * D + pd0 + c, u[k] + c);
       }
     }
+  };
+  int64_t rb = r_begin + warp * RPW;
+  if (rb < r_end) load_rows(rb);
+  for (int e = tid; e < ppb * half; e += kThreads) {
+    const int pl = e / half, j = e % half;
+    s_cs[pl][j] = rope_cs_pow(pos0 + p_first + pl, j, ratio);
+  }
+  __syncthreads();
+  for (; rb < r_end; rb += (kThreads / 32) * RPW) {
 #pragma unroll
     for (int k = 0; k < RPW; ++k) {
       const int64_t r = rb + k;
@@ -262,6 +285,8 @@ rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int D, int rows_per
         for (int c = 0; c < CPL; c += 8) Vec8<Tout>::store(out + r * D + d0 + c, o + c);
       }
     }
+    const int64_t nb = rb + (kThreads / 32) * RPW;
+    if (nb < r_end) load_rows(nb);
   }
 }
 
@@ -291,13 +316,15 @@ csa_status_t launch_compress(const void* C, const void* Z, const void* Cb, const
 template <typename Tin, typename Tout, int CPL>
 csa_status_t launch_norm(const void* x, int64_t rows, int D, int rpp, int64_t pos0, int norm, int rope_dim,
                          float rope_base, float eps, void* out, cudaStream_t st) {
-  int ppb = rpp >= 32 ? 1 : 32 / rpp;      // 32 rows per CTA pass (8 warps x 4 rows)
+  // positions per CTA: at least 32 rows, two positions of a multi-head row block
+  int ppb = rpp >= 32 ? 2 : 32 / rpp;
   int64_t npos = (rows + rpp - 1) / rpp;
   int64_t grid = (npos + ppb - 1) / ppb;
   if (grid == 0) return CSA_OK;
   if (grid > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "csa_rmsnorm_rope: too many rows");
   rmsnorm_rope_kernel<Tin, Tout, CPL><<<(unsigned)grid, kThreads, 0, st>>>(
-      (const Tin*)x, rows, D, rpp, pos0, ppb, norm, rope_dim, rope_base, eps, (Tout*)out);
+      (const Tin*)x, rows, D, rpp, pos0, ppb, norm, rope_dim,
+      rope_dim > 0 ? std::pow((double)rope_base, -2.0 / (double)rope_dim) : 1.0, eps, (Tout*)out);
   return check_launch("csa_rmsnorm_rope");
 }
 
