@@ -158,7 +158,8 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None):
     ws = torch.empty(csa.csa_index_topk_workspace(Bn, 1, ne, k), dtype=torch.uint8, device=dev)
     idx = torch.empty(Bn, 1, k, dtype=torch.int32, device=dev)
     out = torch.empty(Bn, 1, H, D, dtype=torch.bfloat16, device=dev)
-    # split each token's 5 chunks (4 x 128 selected entries + the window) over CTAs
+    # split each token's 10 half chunks (8 x 64 selected entries + the window)
+    # into ranges of about two (more splits cost more in partials than they gain)
     n_split = max(1, min(5, csa.num_sms() // Bn))
     aws = torch.empty(csa.csa_fused_attention_workspace(Bn, 1, H, D, n_split), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -214,6 +215,8 @@ def mixed_decode_leg(dev, steps, warmup, csa, synth, torch, seed=0):
     Bn, k, W, H, D, HI, DI = (cfg[x] for x in ("batch", "k", "W", "H", "D", "HI", "DI"))
     L = cfg["lengths"]
     sms = csa.num_sms()
+    # split-KV ranges per sequence (items are claimed dynamically, so unequal
+    # sequence lengths balance across CTAs)
     split = {"csa": max(1, min(9, sms // Bn)), "hca": 16}
     bufs = []
     for lay in layers:

@@ -96,6 +96,7 @@ struct AttnParams {
   float rope_base;
   int tma_q, tma_kv, tma_tok;   // TMA tile loads for bf16 queries / dense entries / window rows
   int n_split;                  // ranges of half chunks per query token (partials merged afterwards)
+  uint32_t* item_counter;       // non-null: items are claimed dynamically from this zeroed counter
 };
 
 // Rows are consumed in half chunks of 64 (one ring slot each).  The window
@@ -291,7 +292,10 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
   uint64_t* p_full = bars + 7;               // [2]   P^T in shared memory (and O^T rescaled)
   uint64_t* kv_full = bars + 9;              // [2][NT] slab pair of a slot loaded
   uint64_t* pv_done = kv_full + 2 * NT;      // [2][NT] PV tile of a slot retired
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(pv_done + 2 * NT);
+  uint64_t* item_full = pv_done + 2 * NT;    // [4] item ring (dynamic item claiming)
+  uint64_t* item_empty = item_full + 4;      // [4]
+  int64_t* s_items = reinterpret_cast<int64_t*>(item_empty + 4);   // [4]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_items + 4);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -301,6 +305,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
       mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128); mbar_init(&p_full[i], 128);
       for (int t = 0; t < NT; ++t) { mbar_init(&kv_full[i * NT + t], 128); mbar_init(&pv_done[i * NT + t], 1); }
     }
+    for (int i = 0; i < 4; ++i) { mbar_init(&item_full[i], 1); mbar_init(&item_empty[i], 9); }
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -311,6 +316,24 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
   const uint32_t tmem = *s_tmem;
   volatile int* abort_flag = s_abort;
   const int64_t n_items = (int64_t)p.n_seq * p.T * p.n_split;
+  // Item sequence k = 0, 1, ... of this CTA: grid-stride, or (with a counter)
+  // claimed by one loader thread with an atomic and handed to every role warp
+  // through a 4-slot ring, so CTAs that drew short items take more of them.
+  // Whole-warp call; every role warp (9 of them) releases each slot once.
+  auto get_item = [&](uint32_t k, bool fetcher) -> int64_t {
+    if (p.item_counter == nullptr) return (int64_t)blockIdx.x + (int64_t)k * gridDim.x;
+    const uint32_t slot = k & 3, par = (k >> 2) & 1;
+    if (fetcher) {
+      if (wait_bar(&item_empty[slot], par ^ 1, abort_flag)) s_items[slot] = (int64_t)atomicAdd(p.item_counter, 1u);
+      else s_items[slot] = n_items;
+      mbar_arrive(&item_full[slot]);
+    }
+    int64_t it = n_items;
+    if (wait_bar(&item_full[slot], par, abort_flag)) it = s_items[slot];
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&item_empty[slot]);
+    return it;
+  };
 
   if (warp >= 4 && warp < 8) {
     // ============================ loaders
@@ -319,7 +342,9 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
     const int my_r = lt & 63, part = lt >> 6; // converting loads: one row, slabs part, part + 2, ...
     uint32_t g = 0, qcount = 0;
     bool ok = true;
-    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    for (uint32_t kk = 0; ok; ++kk) {
+      const int64_t item = get_item(kk, lt == 0);
+      if (item >= n_items) break;
       const int64_t bt = item / p.n_split;
       const int sp = (int)(item % p.n_split);
       const int b = (int)(bt / p.T), t = (int)(bt % p.T);
@@ -560,7 +585,9 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
       }
       return true;
     };
-    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    for (uint32_t kk = 0; ok; ++kk) {
+      const int64_t item = get_item(kk, false);
+      if (item >= n_items) break;
       const int64_t bt = item / p.n_split;
       const int sp = (int)(item % p.n_split);
       const int b = (int)(bt / p.T), t = (int)(bt % p.T);
@@ -624,7 +651,9 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
     const int rA = 16 * warp + (lane >> 2), rB = rA + 8;
     uint32_t g = 0, icount = 0;
     bool ok = true;
-    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    for (uint32_t kk = 0; ok; ++kk) {
+      const int64_t item = get_item(kk, false);
+      if (item >= n_items) break;
       const int64_t bt = item / p.n_split;
       const int sp = (int)(item % p.n_split);
       const int b = (int)(bt / p.T), t = (int)(bt % p.T);
@@ -947,7 +976,7 @@ template <int D, int KV, int EPI>
 csa_status_t launch_attn(const AttnParams& p, const AttnMaps& m, cudaStream_t st) {
   constexpr int NS = D / 64, NT = D / 128;
   const size_t smem = 1024 + NS * (kNQ * 128) + 2 * NS * (kRows * 128) + 2 * (kRows * 128) +
-                      (2 * 4 * 64 + 4 * 3 * 64) * 4 + 64 * 8 + (9 + 4 * NT) * 8 + 16;
+                      (2 * 4 * 64 + 4 * 3 * 64) * 4 + 64 * 8 + (9 + 4 * NT + 8) * 8 + 4 * 8 + 16;
   auto kern = attn_kernel<D, KV, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attention: cannot reserve %zu bytes of shared memory: %s", smem, cudaGetErrorString(e));
@@ -1117,7 +1146,8 @@ extern "C" csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, 
 extern "C" size_t csa_fused_attention_workspace(int n_seq, int T, int H, int D, int n_split) {
   if (n_seq <= 0 || T <= 0 || H <= 0 || D <= 0 || n_split <= 0) return 0;
   const size_t parts = (size_t)n_seq * T * n_split * H;
-  return ((parts * D * 4 + 255) / 256) * 256 + parts * 4;
+  // partial outputs, partial lse, then the item counter of dynamic claiming
+  return ((parts * D * 4 + 255) / 256) * 256 + ((parts * 4 + 255) / 256) * 256 + 256;
 }
 
 extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q_dtype, const void* kv,
@@ -1155,6 +1185,9 @@ extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q
   p.kv2 = kv_tok; p.cap2 = tok_cap; p.src2 = window_mode == 0 ? SRC2_WINDOW : SRC2_CACHE; p.W = W;
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = Os; p.lse_part = Ls; p.rope_dim = rope_dim; p.n_split = n_split;
+  p.item_counter = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(Ls) + ((parts * 4 + 255) / 256) * 256);
+  cudaError_t ce = cudaMemsetAsync(p.item_counter, 0, sizeof(uint32_t), stream);
+  if (ce != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_fused_attention_splitkv: counter reset failed: %s", cudaGetErrorString(ce));
   s = dispatch<EPI_PARTIAL>(p, D, q_dtype, kv_dtype, tok_dtype, stream);
   if (s != CSA_OK) return s;
   const int64_t toks = (int64_t)n_seq * T;

@@ -55,7 +55,7 @@ bool make_byte_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t r
 // ------------------------------------------------------------------ scores
 constexpr int kIdxThreads = 320;      // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr int kEpiThreads = 256;
-constexpr int kMaxStages = 8;        // key-tile ring depth (deeper rings measured slower)
+constexpr int kStages = 8;           // key-tile ring depth (deeper rings measured slower)
 
 struct IdxParams {
   const float* qs;        // [n_seq, T, HI] or null
@@ -65,7 +65,7 @@ struct IdxParams {
   float* scores;          // [n_seq, T, cap]
   int64_t cap;
   int T, HI, DI, m, TQ, N, tiles_per_chunk;
-  int n_seq, n_qblocks, stages;
+  int n_seq, n_qblocks;
   int64_t n_items;        // n_seq x n_qblocks x key chunks
 };
 
@@ -130,10 +130,9 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   const uint32_t b_stride = (b_bytes + 1023u) & ~1023u;
   uint8_t* sB = smem;                                         // [2] query tiles (item parity)
   uint8_t* sA = smem + 2 * b_stride;                          // [kStages] key tiles
-  const int kStages = p.stages;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sA + kStages * a_bytes);
-  uint64_t* full = bars;                 // [stages]
-  uint64_t* empty = bars + kStages;      // [stages]
+  uint64_t* full = bars;                 // [kStages]
+  uint64_t* empty = bars + kStages;      // [kStages]
   uint64_t* tfull = bars + 2 * kStages;  // [2]
   uint64_t* tempty = tfull + 2;          // [2]
   uint64_t* qfull = tempty + 2;          // [2]
@@ -776,12 +775,8 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
       !make_byte_map(&mq, qI, (uint64_t)n_seq * T * HI, DI, N))
     return fail(CSA_ERR_CUDA, "csa_index_topk: cuTensorMapEncodeTiled failed");
 
-  const size_t fixed = 1024 + 2 * (((size_t)N * DI + 1023) / 1024) * 1024 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4;
-  const size_t per_stage = (size_t)128 * DI + 2 * 8;
-  const size_t budget = 227 * 1024 - 8 * 8;                // less the 8 fixed barriers
-  ip.stages = (int)std::min<size_t>(kMaxStages, (budget - fixed) / per_stage);
-  CSA_REQUIRE(ip.stages >= 2, "csa_index_topk: not enough shared memory for the key ring");
-  const size_t smem = fixed + (size_t)ip.stages * per_stage + 8 * 8;   // + tfull, tempty, qfull, qempty
+  const size_t smem = 1024 + 2 * (((size_t)N * DI + 1023) / 1024) * 1024 + (size_t)kStages * 128 * DI +
+                      (2 * kStages + 8) * 8 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4;
   cudaFuncSetAttribute(indexer_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int grid = (int)std::min<int64_t>(ip.n_items, sms);
   indexer_scores_kernel<<<grid, kIdxThreads, smem, stream>>>(mk, mq, ip);
