@@ -67,6 +67,7 @@ struct IdxParams {
   int T, HI, DI, m, TQ, N, tiles_per_chunk;
   int n_seq, n_qblocks;
   int64_t n_items;        // n_seq x n_qblocks x key chunks
+  uint32_t* item_counter; // zeroed before the launch: items are claimed dynamically
 };
 
 // One work item of the persistent scores kernel: a key chunk of one token
@@ -137,7 +138,10 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   uint64_t* tempty = tfull + 2;          // [2]
   uint64_t* qfull = tempty + 2;          // [2]
   uint64_t* qempty = qfull + 2;          // [2]
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(qempty + 2);
+  uint64_t* ifull = qempty + 2;          // [4] claimed-item ring
+  uint64_t* iempty = ifull + 4;          // [4]
+  int64_t* s_items = reinterpret_cast<int64_t*>(iempty + 4);   // [4]
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_items + 4);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
   // per epilogue group and item parity: visible entries per token, column weights w * qs
   int* s_nv = s_abort + 1;                                    // [2 groups][2][TQ]
@@ -151,6 +155,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiThreads / 2);
       mbar_init(&qfull[a], 1); mbar_init(&qempty[a], 1);
     }
+    for (int i = 0; i < 4; ++i) { mbar_init(&ifull[i], 1); mbar_init(&iempty[i], 2); }
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -160,6 +165,29 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   volatile int* abort_flag = s_abort;
+
+  // Non-empty items are claimed from a global counter by the TMA producer (so
+  // CTAs that drew short rows take more items) and handed to the MMA issuer
+  // and the epilogue through a 4-slot ring; an index >= n_items ends the loop.
+  // The epilogue's 8 warps release a slot through one elected arrival (after
+  // a named barrier), the MMA issuer through the other.
+  auto claim_item = [&](uint32_t k) {
+    const uint32_t slot = k & 3, par = (k >> 2) & 1;
+    int64_t item = p.n_items;
+    if (wait_bar(&iempty[slot], par ^ 1, abort_flag)) {
+      for (;;) {
+        item = (int64_t)atomicAdd(p.item_counter, 1u);
+        if (item >= p.n_items || idx_item(p, item).n_tiles > 0) break;
+      }
+    }
+    s_items[slot] = item;
+    mbar_arrive(&ifull[slot]);
+  };
+  auto read_item = [&](uint32_t k) -> int64_t {
+    const uint32_t slot = k & 3, par = (k >> 2) & 1;
+    return wait_bar(&ifull[slot], par, abort_flag) ? s_items[slot] : p.n_items;
+  };
+  auto release_item = [&](uint32_t k) { mbar_arrive(&iempty[k & 3]); };
 
   const uint32_t swz = p.DI == 128 ? SWZ_128B : (p.DI == 64 ? SWZ_64B : SWZ_32B);
   const uint32_t sbo = 8u * p.DI;
@@ -173,9 +201,11 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       tma_prefetch_desc(&tmap_q);
       uint32_t gt = 0, ic = 0;
       bool ok = true;
-      for (int64_t item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (uint32_t kk = 0; ok; ++kk) {
+        claim_item(kk);
+        const int64_t item = s_items[kk & 3];
+        if (item >= p.n_items) break;
         const IdxItem it = idx_item(p, item);
-        if (it.n_tiles == 0) continue;
         const uint32_t qs = ic & 1;
         if (!wait_bar(&qempty[qs], ((ic >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_expect_tx(&qfull[qs], b_bytes);
@@ -201,9 +231,11 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       const int nk = p.DI / 32;
       uint32_t gt = 0, ic = 0;
       bool ok = true;
-      for (int64_t item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (uint32_t kk = 0; ok; ++kk) {
+        const int64_t item = read_item(kk);
+        release_item(kk);
+        if (item >= p.n_items) break;
         const IdxItem it = idx_item(p, item);
-        if (it.n_tiles == 0) continue;
         const uint32_t qs = ic & 1;
         if (!wait_bar(&qfull[qs], (ic >> 1) & 1, abort_flag)) { ok = false; break; }
         const uint64_t dB = dB0 + ((qs * b_stride) >> 4);
@@ -243,9 +275,12 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     const int key_in_tile = sp * 32 + lane;
     uint32_t gt = 0, ic = 0;
     bool ok = true;
-    for (int64_t item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+    for (uint32_t kk = 0; ok; ++kk) {
+      const int64_t item = read_item(kk);
+      named_bar_sync(3, kEpiThreads);            // all 8 warps have read the slot
+      if (tid == 64) release_item(kk);
+      if (item >= p.n_items) break;
       const IdxItem it = idx_item(p, item);
-      if (it.n_tiles == 0) continue;
       // this group's copy of the block's column weights and visible-entry
       // counts, double-buffered by item parity (the other buffer may still be
       // read by a thread of this group finishing the previous item)
@@ -688,7 +723,7 @@ topk_merge_kernel(TopkParams p) {
 }
 
 struct WsLayout {
-  size_t scores, cand_key, cand_idx, cand_cnt, hist, total;
+  size_t scores, cand_key, cand_idx, cand_cnt, hist, counter, total;
   int n_chunks;
 };
 
@@ -706,6 +741,7 @@ WsLayout ws_layout(int n_seq, int T, int64_t cap, int k) {
     L.cand_cnt = off; off = align_up(off + rows * L.n_chunks * 4, 256);
     L.hist = off; off = align_up(off + rows * (size_t)kHistBins * 4, 256);
   }
+  L.counter = off; off = align_up(off + 4, 256);
   L.total = off;
   return L;
 }
@@ -776,7 +812,12 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
     return fail(CSA_ERR_CUDA, "csa_index_topk: cuTensorMapEncodeTiled failed");
 
   const size_t smem = 1024 + 2 * (((size_t)N * DI + 1023) / 1024) * 1024 + (size_t)kStages * 128 * DI +
-                      (2 * kStages + 8) * 8 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4;
+                      (2 * kStages + 16) * 8 + 4 * 8 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4;
+  ip.item_counter = reinterpret_cast<uint32_t*>(ws + L.counter);
+  {
+    cudaError_t e = cudaMemsetAsync(ip.item_counter, 0, sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_index_topk: counter reset failed: %s", cudaGetErrorString(e));
+  }
   cudaFuncSetAttribute(indexer_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int grid = (int)std::min<int64_t>(ip.n_items, sms);
   indexer_scores_kernel<<<grid, kIdxThreads, smem, stream>>>(mk, mq, ip);

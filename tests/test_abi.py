@@ -44,8 +44,9 @@ def test_abi_version_and_status_strings(L):
 
 
 def test_workspace_size_is_host_arithmetic(L):
-    # prefill: one chunk, only the score matrix; decode: chunked candidates too
-    assert L.csa_index_topk_workspace(1, 16384, 4096, 512) == 16384 * 4096 * 4
+    # prefill: one chunk, the score matrix and the item counter (one 256-byte
+    # block); decode: chunked candidates and key histograms too
+    assert L.csa_index_topk_workspace(1, 16384, 4096, 512) == 16384 * 4096 * 4 + 256
     dec = L.csa_index_topk_workspace(16, 1, 262144, 512)
     assert dec >= 16 * 262144 * 4 + 2 * 16 * 16 * 512 * 4
     assert L.csa_index_topk_workspace(0, 1, 1, 1) == 0
