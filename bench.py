@@ -149,11 +149,11 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None):
+def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1):
     """CSA decode at 2^20 context, batch 16 (one new token per sequence): indexer
     scan over the e4m3 key cache + top-k, then the fused attention over the 512
     selected e4m3 entries, the 128-row bf16 SWA cache and the sink."""
-    inp, cfg = synth.decode_inputs_device("csa_decode_1m", dev, seed=1, batch=batch)
+    inp, cfg = synth.decode_inputs_device("csa_decode_1m", dev, seed=seed, batch=batch)
     Bn, ne, k, W, H, D, HI, DI = (cfg[x] for x in ("batch", "n_e", "k", "W", "H", "D", "HI", "DI"))
     ws = torch.empty(csa.csa_index_topk_workspace(Bn, 1, ne, k), dtype=torch.uint8, device=dev)
     idx = torch.empty(Bn, 1, k, dtype=torch.int32, device=dev)
@@ -345,9 +345,8 @@ def main():
     ap.add_argument("--no-hca", action="store_true", help="skip the HCA prefill leg (S 131072)")
     ap.add_argument("--no-mixed", action="store_true", help="skip the 4-layer mixed decode leg")
     args = ap.parse_args()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from long_context_compressed_02_b200 import replicas
+    rank, world, local = replicas.rank_world()
 
     if args.impl == "reference":
         run_reference(args, rank, world)
@@ -369,13 +368,14 @@ def main():
     if args.no_prefill:
         out = {}
         if not args.no_decode:
-            out["decode_1m"] = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch)
+            out["decode_1m"] = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch,
+                                        seed=replicas.replica_seed(rank, base=1))
         if not args.no_mixed:
-            out["decode_mixed"] = mixed_decode_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=rank)
+            out["decode_mixed"] = mixed_decode_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=replicas.replica_seed(rank))
         if rank == 0:
             print(json.dumps(out), flush=True)
         return
-    inp, cfg = synth.prefill_inputs_device(WORKLOAD, dev, seed=rank, S=args.S)
+    inp, cfg = synth.prefill_inputs_device(WORKLOAD, dev, seed=replicas.replica_seed(rank), S=args.S)
     S, H, D, m, k, W, HI, DI = (cfg[x] for x in ("S", "H", "D", "m", "k", "W", "HI", "DI"))
     ne = S // m
     bf = torch.bfloat16
@@ -433,18 +433,16 @@ def main():
     ms = t_start.elapsed_time(t_end) / args.steps
     per = {n: float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]))
            for j, n in enumerate(names)}
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = replicas.max_over_ranks(ms, device=dev)      # the slowest replica's step time
 
     fl_sparse, fl_window, fl_index = _flops(S, H, D, m, k, W, HI, DI)
     fl_total = fl_sparse + fl_window + fl_index
-    value = world * fl_total / (ms * 1e-3) / 1e12
+    value = replicas.job_rate(fl_total, world, ms * 1e-3) / 1e12
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers (every rank its own
+    # replica; the job's time is the slowest rank's)
     e2e = None
-    if rank == 0 and not args.no_e2e:
+    if not args.no_e2e:
         keys = ["q", "C", "Z", "B", "qI_codes", "w", "kI_codes", "sink"]
         pinned = {kk: torch.empty(inp[kk].shape, dtype=inp[kk].dtype, pin_memory=True) for kk in keys}
         for kk in keys:
@@ -453,7 +451,7 @@ def main():
         h2d = sum(pinned[kk].numel() * pinned[kk].element_size() for kk in keys)
         d2h = out_host.numel() * out_host.element_size()
         n_e2e = max(2, min(args.steps, 5))
-        torch.cuda.synchronize()
+        barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -463,10 +461,10 @@ def main():
             step()
             out_host.copy_(out, non_blocking=True)
         b.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = a.elapsed_time(b) / n_e2e
-        e2e = {"value": fl_total / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        barrier()
+        e2e_ms = replicas.max_over_ranks(a.elapsed_time(b) / n_e2e, device=dev)
+        e2e = {"value": replicas.job_rate(fl_total, world, e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     # ---- roofline of the dominant call
     hbm, bf16_burst, bf16_sus, src = _peaks()
@@ -485,7 +483,8 @@ def main():
 
     decode = None
     if not args.no_decode and args.S is None:
-        decode = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch)
+        decode = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch,
+                                        seed=replicas.replica_seed(rank, base=1))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = host_inputs(inp)
@@ -505,10 +504,10 @@ def main():
         del inp, qn, kt, kv, idx, ws, out
         torch.cuda.empty_cache()
         if not args.no_hca:
-            hca = hca_prefill_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=rank)
+            hca = hca_prefill_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=replicas.replica_seed(rank))
             torch.cuda.empty_cache()
         if not args.no_mixed:
-            mixed = mixed_decode_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=rank)
+            mixed = mixed_decode_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=replicas.replica_seed(rank))
             torch.cuda.empty_cache()
 
     if rank == 0:
@@ -521,7 +520,7 @@ def main():
                            "l2": "inputs larger than L2 (q alone is 1 GiB)",
                            "flops_per_step": {"sparse_mqa": fl_sparse, "swa_window": fl_window,
                                               "indexer_fp8": fl_index}},
-                "prefill_tokens_per_s": world * S / (ms * 1e-3),
+                "prefill_tokens_per_s": replicas.job_rate(S, world, ms * 1e-3),
                 "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode,
                 "hca_prefill": hca, "decode_mixed": mixed,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
