@@ -121,7 +121,12 @@ csa_status_t csa_rmsnorm_rope(const void* x, csa_dtype_t in_dtype, int64_t rows,
  *   kI       [n_seq, cap, DI] e4m3       kI_scale [n_seq, cap] fp32 or NULL (1)
  *   q_pos    [n_seq] int64 (device)
  *   idx      [n_seq, T, k] int32 out
- *   workspace / ws_bytes: at least csa_index_topk_workspace(n_seq, T, cap, k).
+ *   workspace / ws_bytes: at least csa_index_topk_workspace(n_seq, T, cap, k)
+ *            bytes, 16-byte aligned, owned by the caller: the fp32 score matrix,
+ *            for rows longer than 16384 entries the per-chunk candidates and a
+ *            key histogram per row, and the work-item counter (reset by the call
+ *            with a stream-ordered memset).  Contents are undefined afterwards;
+ *            calls sharing one workspace must be ordered on one stream.
  * Requires DI in {32, 64, 128}; HI in {1,2,4,...,64} (power of two <= 64 whose
  * product with the token block is a multiple of 16); 1 <= k <= 2048; cap >= 1.
  * ------------------------------------------------------------------------- */
@@ -233,12 +238,17 @@ csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, const void*
 
 /* ---------------------------------------------------------------------------
  * csa_fused_attention_splitkv — csa_fused_attention with each query token's
- * row set split into n_split consecutive chunk ranges processed in parallel
- * (more CTAs when there are few query tokens, e.g. decode), followed by a merge
- * of the n_split partial results and the sink in one softmax and the optional
- * inverse RoPE.  Same result as csa_fused_attention up to rounding.
+ * row set split into n_split consecutive ranges of 64-row half chunks processed
+ * in parallel (more CTAs when there are few query tokens, e.g. decode), followed
+ * by a merge of the n_split partial results and the sink in one softmax and the
+ * optional inverse RoPE.  Same result as csa_fused_attention up to rounding.
+ * CTAs claim (token, range) items from a counter in the workspace, so ranges of
+ * unequal length (sequences of unequal context) balance across the GPU.
  *   n_split in [1, 16]; workspace of csa_fused_attention_workspace(n_seq, T, H, D,
- *   n_split) bytes (partials: fp32 [n_seq*T*n_split, H, D] + lse).
+ *   n_split) bytes, 16-byte aligned, owned by the caller (partials: fp32
+ *   [n_seq*T*n_split, H, D] + lse, then the item counter, reset by the call with a
+ *   stream-ordered memset); calls sharing one workspace must be ordered on one
+ *   stream.
  * ------------------------------------------------------------------------- */
 size_t csa_fused_attention_workspace(int n_seq, int T, int H, int D, int n_split);
 csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q_dtype, const void* kv, csa_dtype_t kv_dtype,
