@@ -14,6 +14,7 @@
 // of D/8 threads reads one row with fully coalesced transactions.  No tensor
 // cores: there is no contraction here.
 #include <cmath>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <math_constants.h>
 #include "common.cuh"
@@ -290,6 +291,99 @@ rmsnorm_rope_kernel(const Tin* __restrict__ x, int64_t rows, int D, int rows_per
   }
 }
 
+__device__ __forceinline__ void bf16x8_to_float(uint4 raw, float* v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+// bf16 rows of D = 512 (the prefill workloads): as rmsnorm_rope_kernel, but each
+// warp keeps four rows in flight, held as raw bf16 vectors until they are used,
+// which doubles the bytes in flight per SM at the same register budget.
+template <typename Tout>
+__global__ void __launch_bounds__(kThreads)
+rmsnorm_rope_bf16_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int rows_per_pos, int64_t pos0,
+                         int ppb, int norm, int rope_dim, double ratio, float eps, Tout* __restrict__ out) {
+  constexpr int D = 512, CPL = 16, RPW = 4;
+  __shared__ float2 s_cs[32][32];   // [position in CTA][pair]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t p_first = (int64_t)blockIdx.x * ppb;
+  const int half = rope_dim / 2;
+  const int64_t r_begin = p_first * rows_per_pos;
+  const int64_t r_end = min(rows, (p_first + ppb) * rows_per_pos);
+  const int r0d = D - rope_dim;
+  const int d0 = lane * CPL;
+  const bool in_rope = rope_dim > 0 && d0 >= r0d;
+  const bool first_half = d0 < r0d + half;
+  const int pd0 = first_half ? d0 + half : d0 - half;     // partner channels
+  uint4 rv[RPW][2], ru[RPW][2];
+  auto load_rows = [&](int64_t rb) {
+#pragma unroll
+    for (int k = 0; k < RPW; ++k) {
+      const int64_t r = min(rb + k, r_end - 1);
+      const uint4* src = reinterpret_cast<const uint4*>(x + r * D + d0);
+      rv[k][0] = __ldg(src);
+      rv[k][1] = __ldg(src + 1);
+      if (in_rope) {
+        const uint4* sp = reinterpret_cast<const uint4*>(x + r * D + pd0);
+        ru[k][0] = __ldg(sp);
+        ru[k][1] = __ldg(sp + 1);
+      }
+    }
+  };
+  int64_t rb = r_begin + warp * RPW;
+  if (rb < r_end) load_rows(rb);
+  for (int e = tid; e < ppb * half; e += kThreads) {
+    const int pl = e / half, j = e % half;
+    s_cs[pl][j] = rope_cs_pow(pos0 + p_first + pl, j, ratio);
+  }
+  __syncthreads();
+  for (; rb < r_end; rb += (kThreads / 32) * RPW) {
+#pragma unroll
+    for (int k = 0; k < RPW; ++k) {
+      const int64_t r = rb + k;
+      float v[CPL];
+      bf16x8_to_float(rv[k][0], v);
+      bf16x8_to_float(rv[k][1], v + 8);
+      float inv = 1.f;
+      if (norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) ss = fmaf(v[c], v[c], ss);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        inv = rsqrtf(ss / (float)D + eps);
+      }
+      float o[CPL];
+      if (in_rope) {
+        float u[CPL];
+        bf16x8_to_float(ru[k][0], u);
+        bf16x8_to_float(ru[k][1], u + 8);
+        const int pl = (int)(min(r, r_end - 1) / rows_per_pos - p_first);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          const float2 cs = s_cs[pl][(d0 + c - r0d) % half];
+          const float a = v[c] * inv, bb = u[c] * inv;
+          o[c] = first_half ? a * cs.x - bb * cs.y : bb * cs.y + a * cs.x;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) o[c] = v[c] * inv;
+      }
+      if (r < r_end) {
+#pragma unroll
+        for (int c = 0; c < CPL; c += 8) Vec8<Tout>::store(out + r * D + d0 + c, o + c);
+      }
+    }
+    const int64_t nb = rb + (kThreads / 32) * RPW;
+    if (nb < r_end) load_rows(nb);
+  }
+}
+
 template <typename Tin, typename Tout>
 csa_status_t launch_compress(const void* C, const void* Z, const void* Cb, const void* Zb, const float* B,
                              int64_t n_e, int D, int m, int overlap, int norm, int rope_dim,
@@ -322,9 +416,14 @@ csa_status_t launch_norm(const void* x, int64_t rows, int D, int rpp, int64_t po
   int64_t grid = (npos + ppb - 1) / ppb;
   if (grid == 0) return CSA_OK;
   if (grid > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "csa_rmsnorm_rope: too many rows");
-  rmsnorm_rope_kernel<Tin, Tout, CPL><<<(unsigned)grid, kThreads, 0, st>>>(
-      (const Tin*)x, rows, D, rpp, pos0, ppb, norm, rope_dim,
-      rope_dim > 0 ? std::pow((double)rope_base, -2.0 / (double)rope_dim) : 1.0, eps, (Tout*)out);
+  const double ratio = rope_dim > 0 ? std::pow((double)rope_base, -2.0 / (double)rope_dim) : 1.0;
+  if constexpr (std::is_same<Tin, __nv_bfloat16>::value && CPL == 16) {
+    rmsnorm_rope_bf16_kernel<Tout><<<(unsigned)grid, kThreads, 0, st>>>(
+        (const __nv_bfloat16*)x, rows, rpp, pos0, ppb, norm, rope_dim, ratio, eps, (Tout*)out);
+  } else {
+    rmsnorm_rope_kernel<Tin, Tout, CPL><<<(unsigned)grid, kThreads, 0, st>>>(
+        (const Tin*)x, rows, D, rpp, pos0, ppb, norm, rope_dim, ratio, eps, (Tout*)out);
+  }
   return check_launch("csa_rmsnorm_rope");
 }
 
