@@ -34,6 +34,14 @@ METRIC = "CSA/HCA decode tokens/s @1M ctx and prefill TFLOP/s, % of HBM/TC roofl
 WORKLOAD = "csa_prefill"
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernels, from ncu captures of smaller cases of the same kernels scaled
+# by the units processed: the fused attention at S 4096 (507.8 MB) x 4 for
+# S 16384; the indexer scores kernel at decode batch 4 (144.1 MB) x 4 for
+# batch 16.  Reset to None whenever one of these kernels changes.
+PROFILED_TRAFFIC = {"fused_attention": 4 * 507.76e6, "index_topk": 4 * 144.10e6}
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -205,7 +213,9 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1):
             "algorithmic_bytes_per_step": algo,
             "hbm_frac_step": algo / (ms * 1e-3) / 1e9 / hbm,
             "roofline": {"kernel": "index_topk", "bound": "hbm", "achieved": ach_idx, "peak": hbm, "unit": "GB/s",
-                         "frac": ach_idx / hbm, "traffic": None, "peak_source": f"{src} copy bandwidth"}}
+                         "frac": ach_idx / hbm,
+                         "traffic": PROFILED_TRAFFIC["index_topk"] if Bn == 16 else None,
+                         "peak_source": f"{src} copy bandwidth"}}
 
 
 def mixed_decode_leg(dev, steps, warmup, csa, synth, torch, seed=0):
@@ -475,7 +485,8 @@ def main():
         fl, bound, peak = algo[dom]
         ach = fl / (per[dom] * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": None,
+                "frac": ach / peak,
+                "traffic": PROFILED_TRAFFIC.get(dom) if args.S is None else None,
                 "peak_source": f"{src} bf16 sustained" + (" x2 (fp8 nominal ratio)" if dom == "index_topk" else "")}
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s", "frac": None,
