@@ -400,22 +400,25 @@ def main():
     stream = torch.cuda.current_stream()
     names = ["q_norm_rope", "kv_tok_norm_rope", "compress", "index_topk", "fused_attention"]
 
-    def step(ev=None):
+    def step(ev=None, x=None, o=None):
+        x = inp if x is None else x            # this step's inputs and output buffer
+        o = out if o is None else o
+
         def mark(i):
             if ev is not None:
                 ev[i].record(stream)
         mark(0)
-        csa.csa_rmsnorm_rope(inp["q"], rows_per_pos=H, out=qn)
+        csa.csa_rmsnorm_rope(x["q"], rows_per_pos=H, out=qn)
         mark(1)
-        csa.csa_rmsnorm_rope(inp["C"], rows_per_pos=1, out=kt)
+        csa.csa_rmsnorm_rope(x["C"], rows_per_pos=1, out=kt)
         mark(2)
-        csa.csa_compress(inp["C"], inp["Z"], inp["B"], m, True, norm=True, rope_dim=64, out=kv)
+        csa.csa_compress(x["C"], x["Z"], x["B"], m, True, norm=True, rope_dim=64, out=kv)
         mark(3)
-        csa.csa_index_topk(inp["qI_codes"][None], inp["w"][None], inp["kI_codes"][None], pos, m, k,
+        csa.csa_index_topk(x["qI_codes"][None], x["w"][None], x["kI_codes"][None], pos, m, k,
                            workspace=ws, idx=idx)
         mark(4)
-        csa.csa_fused_attention(qn[None], kv[None], kt[None], pos, W, inp["sink"], idx=idx, inv_rope=True,
-                                rope_dim=64, out=out)
+        csa.csa_fused_attention(qn[None], kv[None], kt[None], pos, W, x["sink"], idx=idx, inv_rope=True,
+                                rope_dim=64, out=o)
         mark(5)
 
     launches_per_step = 6      # 2 norm/rope, compress, indexer scores, top-k, fused attention
@@ -450,31 +453,57 @@ def main():
     value = replicas.job_rate(fl_total, world, ms * 1e-3) / 1e12
 
     # ---- end to end through the public API with host buffers (every rank its own
-    # replica; the job's time is the slowest rank's)
+    # replica; the job's time is the slowest rank's).  Each step uploads its
+    # inputs from pinned host memory and downloads its output; uploads, compute
+    # and downloads of consecutive steps overlap on three streams with
+    # double-buffered device inputs and outputs (a serving pipeline's shape).
     e2e = None
     if not args.no_e2e:
         keys = ["q", "C", "Z", "B", "qI_codes", "w", "kI_codes", "sink"]
         pinned = {kk: torch.empty(inp[kk].shape, dtype=inp[kk].dtype, pin_memory=True) for kk in keys}
         for kk in keys:
             pinned[kk].copy_(inp[kk])
-        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dev_in = [inp, {kk: torch.empty_like(inp[kk]) for kk in keys}]
+        dev_out = [out, torch.empty_like(out)]
+        out_host = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
         h2d = sum(pinned[kk].numel() * pinned[kk].element_size() for kk in keys)
-        d2h = out_host.numel() * out_host.element_size()
-        n_e2e = max(2, min(args.steps, 5))
+        d2h = out_host[0].numel() * out_host[0].element_size()
+        n_e2e = max(4, min(args.steps, 8))
+        s_up, s_down = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in_ready", "in_free", "out_ready", "out_free")}
         barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(n_e2e):
-            for kk in keys:
-                inp[kk].copy_(pinned[kk], non_blocking=True)
-            step()
-            out_host.copy_(out, non_blocking=True)
+        s_up.wait_event(a)
+        s_down.wait_event(a)
+        for i in range(n_e2e):
+            j = i % 2
+            if i >= 2:
+                s_up.wait_event(ev["in_free"][j])          # step i - 2 has consumed this input set
+            with torch.cuda.stream(s_up):
+                for kk in keys:
+                    dev_in[j][kk].copy_(pinned[kk], non_blocking=True)
+                ev["in_ready"][j].record(s_up)
+            stream.wait_event(ev["in_ready"][j])
+            if i >= 2:
+                stream.wait_event(ev["out_free"][j])        # step i - 2's output has been downloaded
+            step(x=dev_in[j], o=dev_out[j])
+            ev["in_free"][j].record(stream)
+            ev["out_ready"][j].record(stream)
+            s_down.wait_event(ev["out_ready"][j])
+            with torch.cuda.stream(s_down):
+                out_host[j].copy_(dev_out[j], non_blocking=True)
+                ev["out_free"][j].record(s_down)
+        for j in range(2):
+            stream.wait_event(ev["out_free"][j])
         b.record(stream)
         barrier()
         e2e_ms = replicas.max_over_ranks(a.elapsed_time(b) / n_e2e, device=dev)
         e2e = {"value": replicas.job_rate(fl_total, world, e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e, "pipelined": "uploads / compute / downloads of consecutive steps overlap"}
+        del dev_in, dev_out
 
     # ---- roofline of the dominant call
     hbm, bf16_burst, bf16_sus, src = _peaks()
