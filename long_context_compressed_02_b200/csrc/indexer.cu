@@ -143,10 +143,10 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   int64_t* s_items = reinterpret_cast<int64_t*>(iempty + 4);   // [4]
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_items + 4);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
-  // per epilogue group and item parity: visible entries per token, column weights w * qs
-  int* s_nv = s_abort + 1;                                    // [2 groups][2][TQ]
+  // per item-ring slot: visible entries per token, column weights w * qs
+  int* s_nv = s_abort + 1;                                    // [4][TQ]
   float* s_w = reinterpret_cast<float*>(
-      (reinterpret_cast<uintptr_t>(s_nv + 4 * p.TQ) + 15) & ~uintptr_t(15));   // [2 groups][2][N]
+      (reinterpret_cast<uintptr_t>(s_nv + 4 * p.TQ) + 15) & ~uintptr_t(15));   // [4][N]
 
   const uint32_t tmem_cols = p.N <= 16 ? 32u : (p.N <= 32 ? 64u : (p.N <= 64 ? 128u : (p.N <= 128 ? 256u : 512u)));
   if (tid == 0) {
@@ -155,7 +155,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiThreads / 2);
       mbar_init(&qfull[a], 1); mbar_init(&qempty[a], 1);
     }
-    for (int i = 0; i < 4; ++i) { mbar_init(&ifull[i], 1); mbar_init(&iempty[i], 2); }
+    for (int i = 0; i < 4; ++i) { mbar_init(&ifull[i], 32); mbar_init(&iempty[i], 1 + kEpiThreads / 32); }
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -166,22 +166,44 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   const uint32_t tmem = *s_tmem;
   volatile int* abort_flag = s_abort;
 
-  // Non-empty items are claimed from a global counter by the TMA producer (so
-  // CTAs that drew short rows take more items) and handed to the MMA issuer
-  // and the epilogue through a 4-slot ring; an index >= n_items ends the loop.
-  // The epilogue's 8 warps release a slot through one elected arrival (after
-  // a named barrier), the MMA issuer through the other.
+  // Non-empty items are claimed from a global counter by the producer warp (so
+  // CTAs that drew short rows take more items), which also fills the slot's
+  // column weights and visible-entry counts, and handed to the MMA issuer and
+  // the epilogue through a 4-slot ring; an index >= n_items ends the loop.  A
+  // slot is released by the MMA issuer once read and by each epilogue warp once
+  // it has finished the item's tiles.  Whole-warp call for the producer.
   auto claim_item = [&](uint32_t k) {
     const uint32_t slot = k & 3, par = (k >> 2) & 1;
     int64_t item = p.n_items;
-    if (wait_bar(&iempty[slot], par ^ 1, abort_flag)) {
+    if (lane == 0 && wait_bar(&iempty[slot], par ^ 1, abort_flag)) {
       for (;;) {
         item = (int64_t)atomicAdd(p.item_counter, 1u);
         if (item >= p.n_items || idx_item(p, item).n_tiles > 0) break;
       }
     }
-    s_items[slot] = item;
-    mbar_arrive(&ifull[slot]);
+    item = __shfl_sync(0xffffffffu, item, 0);
+    if (item < p.n_items) {
+      const IdxItem it = idx_item(p, item);
+      float* gw = s_w + slot * p.N;
+      int* gnv = s_nv + slot * p.TQ;
+      for (int c = lane; c < p.N; c += 32) {
+        const int tq = c / p.HI, h = c % p.HI;
+        const int t = it.t0 + tq;
+        float v = 0.f;
+        if (t < p.T) {
+          const int64_t o = ((int64_t)it.b * p.T + t) * p.HI + h;
+          v = p.w[o] * (p.qs ? p.qs[o] : 1.f);
+        }
+        gw[c] = v;
+      }
+      for (int tq = lane; tq < p.TQ; tq += 32) {
+        const int t = it.t0 + tq;
+        gnv[tq] = t < p.T ? (int)min(p.cap, (it.pos0 + t + 1) / p.m) : 0;
+      }
+    }
+    if (lane == 0) s_items[slot] = item;
+    mbar_arrive(&ifull[slot]);                // 32 arrivals: every lane's writes are released
+    return item;
   };
   auto read_item = [&](uint32_t k) -> int64_t {
     const uint32_t slot = k & 3, par = (k >> 2) & 1;
@@ -195,30 +217,37 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   // Every role walks the same item sequence; the key-tile ring (stage, phase),
   // the accumulator pair and the query-tile pair all continue across items.
   if (warp == 0) {
-    // ---------------- TMA producer (lane 0)
-    if (lane == 0) {
-      tma_prefetch_desc(&tmap_k);
-      tma_prefetch_desc(&tmap_q);
+    // ---------------- producer: the warp claims items and fills their weights;
+    // lane 0 issues the TMA loads
+    {
+      if (lane == 0) {
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_q);
+      }
       uint32_t gt = 0, ic = 0;
       bool ok = true;
       for (uint32_t kk = 0; ok; ++kk) {
-        claim_item(kk);
-        const int64_t item = s_items[kk & 3];
+        const int64_t item = claim_item(kk);
         if (item >= p.n_items) break;
-        const IdxItem it = idx_item(p, item);
-        const uint32_t qs = ic & 1;
-        if (!wait_bar(&qempty[qs], ((ic >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(&qfull[qs], b_bytes);
-        tma_load_2d(sB + qs * b_stride, &tmap_q, 0, (int32_t)(((int64_t)it.b * p.T + it.t0) * p.HI), &qfull[qs]);
-        for (int j = 0; j < it.n_tiles; ++j, ++gt) {
-          const int s = gt % kStages;
-          const uint32_t ph = (gt / kStages) & 1;
-          if (!wait_bar(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(&full[s], a_bytes);
-          tma_load_2d(sA + s * a_bytes, &tmap_k, 0, (int32_t)((int64_t)it.b * p.cap + (int64_t)(it.tile0 + j) * 128),
-                      &full[s]);
+        if (lane == 0) {
+          const IdxItem it = idx_item(p, item);
+          const uint32_t qs = ic & 1;
+          if (!wait_bar(&qempty[qs], ((ic >> 1) & 1) ^ 1, abort_flag)) ok = false;
+          if (ok) {
+            mbar_expect_tx(&qfull[qs], b_bytes);
+            tma_load_2d(sB + qs * b_stride, &tmap_q, 0, (int32_t)(((int64_t)it.b * p.T + it.t0) * p.HI), &qfull[qs]);
+          }
+          for (int j = 0; j < it.n_tiles && ok; ++j, ++gt) {
+            const int s = gt % kStages;
+            const uint32_t ph = (gt / kStages) & 1;
+            if (!wait_bar(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
+            mbar_expect_tx(&full[s], a_bytes);
+            tma_load_2d(sA + s * a_bytes, &tmap_k, 0,
+                        (int32_t)((int64_t)it.b * p.cap + (int64_t)(it.tile0 + j) * 128), &full[s]);
+          }
+          ++ic;
         }
-        ++ic;
+        ok = __shfl_sync(0xffffffffu, ok, 0);   // the warp leaves together
       }
     }
   } else if (warp == 1) {
@@ -270,38 +299,21 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     const int ew = warp - 2;
     const int sp = warp & 3;
     const int grp = ew >> 2;
-    const int gtid = tid - 64 - 128 * grp;    // 0 .. 127 within the group
     const int log2hi = __ffs(p.HI) - 1;
     const int key_in_tile = sp * 32 + lane;
-    uint32_t gt = 0, ic = 0;
+    uint32_t gt = 0;
     bool ok = true;
     for (uint32_t kk = 0; ok; ++kk) {
       const int64_t item = read_item(kk);
-      named_bar_sync(3, kEpiThreads);            // all 8 warps have read the slot
-      if (tid == 64) release_item(kk);
-      if (item >= p.n_items) break;
+      if (item >= p.n_items) {
+        __syncwarp();
+        if (lane == 0) release_item(kk);
+        break;
+      }
       const IdxItem it = idx_item(p, item);
-      // this group's copy of the block's column weights and visible-entry
-      // counts, double-buffered by item parity (the other buffer may still be
-      // read by a thread of this group finishing the previous item)
-      float* gw = s_w + (2 * grp + (ic & 1)) * p.N;
-      int* gnv = s_nv + (2 * grp + (ic & 1)) * p.TQ;
-      ++ic;
-      for (int c = gtid; c < p.N; c += 128) {
-        const int tq = c / p.HI, h = c % p.HI;
-        const int t = it.t0 + tq;
-        float v = 0.f;
-        if (t < p.T) {
-          const int64_t o = ((int64_t)it.b * p.T + t) * p.HI + h;
-          v = p.w[o] * (p.qs ? p.qs[o] : 1.f);
-        }
-        gw[c] = v;
-      }
-      for (int tq = gtid; tq < p.TQ; tq += 128) {
-        const int t = it.t0 + tq;
-        gnv[tq] = t < p.T ? (int)min(p.cap, (it.pos0 + t + 1) / p.m) : 0;
-      }
-      named_bar_sync(1 + grp, 128);
+      // the slot's column weights and visible-entry counts (filled by the producer)
+      const float* gw = s_w + (kk & 3) * p.N;
+      const int* gnv = s_nv + (kk & 3) * p.TQ;
       const uint32_t w_addr = smem_u32(gw);
       // this group's tiles of the item: global tile numbers gt with gt % 2 == grp
       const int j0 = ((int)(gt & 1) == grp) ? 0 : 1;
@@ -363,6 +375,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
       }
+      __syncwarp();
+      if (lane == 0) release_item(kk);       // this warp is done with the slot's weights
       gt += it.n_tiles;
     }
   }

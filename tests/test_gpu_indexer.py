@@ -92,6 +92,27 @@ def test_ties_go_to_lower_index():
     assert np.array_equal(got[0], np.repeat(np.arange(50, dtype=np.int32)[None], T, 0))
 
 
+@pytest.mark.parametrize("mode", ["all_equal", "coarse_ties"])
+def test_long_rows_with_crowded_threshold_bin(mode):
+    """Rows of more than 16384 entries (histogram-filtered selection) where the
+    threshold bin holds most of a chunk: every score equal (the filter keeps
+    whole chunks and the local selection runs on all of them), or only a few
+    distinct score values (ties broken by the lower index across chunks)."""
+    rng = np.random.default_rng(8)
+    n_seq, cap, HI, DI, m, k = 2, 40000, 8, 32, 4, 512
+    if mode == "all_equal":
+        kI = np.repeat(synth.grid_codes(rng, (1, 1, DI)), cap, axis=1).repeat(n_seq, axis=0)
+    else:
+        pool = synth.grid_codes(rng, (3, DI))              # three distinct keys
+        kI = pool[rng.integers(0, 3, size=(n_seq, cap))]
+    qI = synth.grid_codes(rng, (n_seq, 1, HI, DI))
+    w = (np.floor(rng.random((n_seq, 1, HI)) * 16) / 16).astype(np.float32)
+    q_pos = [4 * cap - 1, 4 * 30000 + 2]
+    got = _run(qI, w, kI, q_pos, m, k)
+    ref = _oracle(qI, w, kI, q_pos, m, k)
+    assert np.array_equal(got, ref)
+
+
 def test_continuous_inputs_within_rounding_bound():
     inp, cfg = synth.prefill_inputs("csa_prefill", S=3000, grid=False)
     k = 256
