@@ -19,19 +19,26 @@
 // K-major A operand of the first product and, read through an MN-major
 // descriptor, the A operand of the second; nothing is transposed or copied.
 // Rows stream through a ring of two 64-row slots (half chunks), so the loads
-// of half chunk h+1 overlap the S, softmax and PV work of half chunk h, and
-// S(h+1) is issued ahead of PV(h) so the softmax of h+1 overlaps PV(h).
-// Softmax runs per column (head) over TMEM lanes (rows): the M=64 S^T is
-// read with the 16x256b TMEM shape (all 32 threads of a warp hold data),
-// column maxima and sums use a 3-level butterfly plus a 4-warp exchange; the
-// running max is only raised when it grows by more than 2^8, so O^T is
-// rarely rescaled.
+// of half chunk h+1 overlap the S, softmax and PV work of half chunk h; S(h+1)
+// is issued before PV(h), so the softmax of h overlaps the S products of h+1.
+// S goes to two TMEM accumulators (even / odd slabs, alternating MMA by MMA,
+// since an MMA into the accumulator of the one before waits for it), summed by
+// the softmax.  Softmax runs per column (head) over TMEM lanes (rows): the
+// M=64 S^T is read with the 16x256b TMEM shape (all 32 threads of a warp hold
+// data), column maxima and sums use a 3-level butterfly plus a 4-warp
+// exchange; the running max is only raised when it grows by more than 2^8, so
+// O^T is rarely rescaled.  The epilogue scales O^T straight from TMEM into
+// global memory (the RoPE dimension pairs d, d+32 sit in different warps and
+// are exchanged through shared memory for the inverse rotation).
 //
 // Roles (288 threads): warps 0-3 softmax + epilogue, warps 4-7 loaders
-// (gathers through cp.async tracked on mbarriers, TMA boxes for contiguous
-// rows, or load-convert for fp32 / e4m3 stores), warp 8 TMEM allocation +
-// MMA issue.  Each slot is refilled slab pair by slab pair as the PV tile
-// that read it retires, and S MMAs start on a slab pair as soon as it lands.
+// (gathers through cp.async, fenced and signalled per slab pair by the
+// producer, TMA boxes for contiguous rows, or load-convert for fp32 / e4m3
+// stores), warp 8 TMEM allocation + MMA issue.  Each slot is refilled slab
+// pair by slab pair as the PV tile pair that read it retires, and S MMAs start
+// on a slab pair as soon as it lands.  Work items (query token, range of half
+// chunks) are taken grid-stride, or, for split-KV calls, claimed from a
+// counter so that ranges of unequal length balance.
 #include <algorithm>
 #include <cstring>
 #include <cuda_bf16.h>

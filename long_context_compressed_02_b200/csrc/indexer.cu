@@ -10,18 +10,23 @@
 // Kernel 1 (indexer_scores_kernel) is an FP8 e4m3 tensor-core contraction:
 //   D[key, (token, head)] = kI[key, :] . qI[token, head, :]
 // with M = 128 keys per tile (A operand, streamed by TMA through a ring of
-// shared-memory stages), N = TQ tokens x HI heads (B operand, loaded once per
-// CTA), K = DI, fp32 accumulation in TMEM (two accumulators so the epilogue
-// of tile j overlaps the MMA of tile j+1).  The epilogue applies ReLU, the
-// head weights w * qs, the key scale ks and the visibility mask, and writes
-// one fp32 score per (token, key).
+// shared-memory stages), N = TQ tokens x HI heads (B operand, one tile per work
+// item, double-buffered), K = DI, fp32 accumulation in TMEM (two accumulators
+// so the epilogue of tile j overlaps the MMA of tile j+1).  The epilogue
+// applies ReLU, the head weights w * qs, the key scale ks and the visibility
+// mask, and writes one fp32 score per (token, key).  The kernel is persistent:
+// work items (sequence, token block, key chunk) are claimed from a global
+// counter, so rows of unequal length balance across the GPU.
 //
-// Kernels 2/3 select the top-k per query row by a 4-pass 8-bit radix select
-// on order-preserving uint32 keys, then compact in index order, so the result
-// is ascending, deterministic, and ties go to the lower entry index.  Rows
-// longer than one shared-memory chunk are split into chunks (local top-k
-// each) and the candidates merged; the global top-k restricted to a chunk is
-// always within that chunk's local top-k, so the merge is exact.
+// Top-k per query row: rows of up to 16384 visible entries are selected in
+// shared memory by an 8-bit radix select (starting below the bits every key
+// shares) followed by an order-preserving compaction, so the result is
+// ascending, deterministic, and ties go to the lower entry index.  Longer
+// rows first build a histogram of the top 12 key bits; the threshold bin it
+// gives bounds the row's k-th largest key from below, so each 16384-entry
+// chunk keeps only keys at or above it (exact: the global top-k restricted to
+// a chunk is among them), selects locally only if more than k survive, and
+// one CTA per row merges the survivors.
 #include <algorithm>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
