@@ -157,7 +157,7 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1):
+def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1, n_split=None):
     """CSA decode at 2^20 context, batch 16 (one new token per sequence): indexer
     scan over the e4m3 key cache + top-k, then the fused attention over the 512
     selected e4m3 entries, the 128-row bf16 SWA cache and the sink."""
@@ -168,7 +168,8 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1):
     out = torch.empty(Bn, 1, H, D, dtype=torch.bfloat16, device=dev)
     # split each token's 10 half chunks (8 x 64 selected entries + the window)
     # into ranges of about two (more splits cost more in partials than they gain)
-    n_split = max(1, min(5, csa.num_sms() // Bn))
+    if n_split is None:
+        n_split = max(1, min(5, csa.num_sms() // Bn))
     aws = torch.empty(csa.csa_fused_attention_workspace(Bn, 1, H, D, n_split), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -218,7 +219,7 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1):
                          "peak_source": f"{src} copy bandwidth"}}
 
 
-def mixed_decode_leg(dev, steps, warmup, csa, synth, torch, seed=0):
+def mixed_decode_leg(dev, steps, warmup, csa, synth, torch, seed=0, split=None):
     """The 4-layer decode stack (CSA, HCA, CSA, HCA), batch 32, per-sequence
     contexts U[64K, 1M]: one new token per sequence through all four layers."""
     layers, q_pos, cfg = synth.mixed_decode_inputs_device(dev, seed=seed)
@@ -227,7 +228,8 @@ def mixed_decode_leg(dev, steps, warmup, csa, synth, torch, seed=0):
     sms = csa.num_sms()
     # split-KV ranges per sequence (items are claimed dynamically, so unequal
     # sequence lengths balance across CTAs)
-    split = {"csa": max(1, min(9, sms // Bn)), "hca": 16}
+    if split is None:
+        split = {"csa": max(1, min(9, sms // Bn)), "hca": 16}
     bufs = []
     for lay in layers:
         b = {"out": torch.empty(Bn, 1, H, D, dtype=torch.bfloat16, device=dev)}
