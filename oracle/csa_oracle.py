@@ -55,6 +55,7 @@ __all__ = [
     "window_sink_combine", "merge_partials",
     "csa_layer", "hca_layer", "csa_layer_matrix", "hca_layer_matrix",
     "csa_decode", "hca_decode", "flop_counts",
+    "fp8_row_quantize", "stream_append",
 ]
 
 # ----------------------------------------------------------------------------
@@ -492,6 +493,48 @@ def hca_decode(q, kv, swa, sink, t, *, m=128, inv_rope=True, rope_dim=64, rope_b
                             inv_rope=inv_rope, rope_dim=rope_dim, rope_base=rope_base,
                             window_rows=[swa])
     return O[0]
+
+
+# ----------------------------------------------------------------------------
+# Decode-time cache writer: the compressor applied to a token stream, one token
+# at a time, emitting a cache row when a block completes  [CS "KV 压缩" (entries
+# are produced block by block), "其他辅助设计" (non-RoPE dims in FP8, RoPE dims
+# in BF16); LD (FP8 caches)].
+# ----------------------------------------------------------------------------
+
+def fp8_row_quantize(x, rope_dim: int = 64):
+    """One cache row: the first D - rope_dim dims as e4m3 codes under the row
+    scale amax / 448 (value = decode(code) * scale; scale 1 for an all-zero
+    row), the last rope_dim dims rounded to bf16.  Returns (codes [D - r] uint8,
+    rope [r] float64 bf16-valued, scale float64)."""
+    x = np.asarray(x, np.float64)
+    D = x.shape[-1]
+    nope = x[..., :D - rope_dim]
+    amax = np.abs(nope).max(axis=-1)
+    scale = np.where(amax > 0, amax / 448.0, 1.0)
+    codes = e4m3_encode(nope / scale[..., None])
+    return codes, bf16_round(x[..., D - rope_dim:]), scale
+
+
+def stream_append(ring_C, ring_Z, c, z, pos: int, B, m: int, overlap: bool, *, norm_rope: bool = True,
+                  rope_dim: int = 64, rope_base: float = 10000.0):
+    """Store token `pos` (rows c, z) in the sequence's ring of the last 2m
+    tokens (slot pos % 2m) and, when its block is complete ((pos + 1) % m == 0),
+    return (i, entry) for entry i = (pos + 1) / m - 1: the compressor over the
+    current block (and, overlapping, the previous one) read from the ring, then
+    RMSNorm and RoPE at position i * m.  Otherwise returns None."""
+    L = 2 * m
+    ring_C[pos % L] = c
+    ring_Z[pos % L] = z
+    if (pos + 1) % m:
+        return None
+    i = (pos + 1) // m - 1
+    first = (i - 1) * m if (overlap and i > 0) else i * m
+    rows = [(first + j) % L for j in range((i + 1) * m - first)]
+    entry = compress(np.asarray(ring_C)[rows], np.asarray(ring_Z)[rows], B, m, overlap)[-1]
+    if norm_rope:
+        entry = rope_partial(rmsnorm(entry), i * m, rope_dim, rope_base)
+    return i, entry
 
 
 def flop_counts(S, H, D, m, k=None, W=128, HI=0, DI=0, dense=False):
