@@ -107,6 +107,37 @@ csa_status_t csa_rmsnorm_rope(const void* x, csa_dtype_t in_dtype, int64_t rows,
                               cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * csa_compress_append — decode-time cache writer ([CS] "KV 压缩": entries are
+ * pooled block by block; "其他辅助设计": the non-RoPE dims are stored in FP8,
+ * the 64 RoPE dims in BF16; [LD]: FP8 caches).  For every sequence b, the new
+ * token at position p = q_pos[b] (rows c_tok[b], z_tok[b]) is stored in slot
+ * p % 2m of the sequence's ring of the last 2m tokens; when it completes block
+ * i = (p + 1) / m - 1, entry i is pooled from the ring exactly as csa_compress
+ * pools it (per-channel softmax of Z + B over the current block and, with
+ * overlap, the previous one), RMS-normalised (norm != 0), rotated at position
+ * i * m, and written as cache row i:
+ *     kv_nope[b, i, :D - rope_dim] = e4m3(entry / s),  s = max|entry[:D - rope_dim]| / 448
+ *                                    (s = 1 for an all-zero row; round to nearest even, saturating)
+ *     kv_rope[b, i, :]             = bf16(entry[D - rope_dim:])
+ *     kv_scale[b, i]               = s
+ * Tokens that complete no block only update the ring.
+ *   c_tok, z_tok  [n_seq, D] in_dtype (F32 or BF16)    B [2m, D] (overlap) or [m, D] fp32
+ *   q_pos         [n_seq] int64 (device): the new token's position
+ *   ring_C/ring_Z [n_seq, 2m, D] in_dtype, caller-owned state: slot u % 2m holds
+ *                 token u's rows; a stream that starts after a prefill copies the
+ *                 last 2m prefill tokens' rows into their slots first
+ *   kv_nope [n_seq, cap, D - rope_dim] e4m3, kv_rope [n_seq, cap, rope_dim] bf16,
+ *   kv_scale [n_seq, cap] fp32: the cache layout the attention calls read; a
+ *                 block whose index is >= cap writes nothing
+ * Requires D a multiple of 8 in [64, 2048], 1 <= m <= 1024, rope_dim 0 or 64.
+ * One CTA per sequence; asynchronous on `stream`.
+ * ------------------------------------------------------------------------- */
+csa_status_t csa_compress_append(const void* c_tok, const void* z_tok, csa_dtype_t in_dtype, const float* B,
+                                 int n_seq, int D, int m, int overlap, const int64_t* q_pos, void* ring_C,
+                                 void* ring_Z, uint8_t* kv_nope, void* kv_rope, float* kv_scale, int64_t cap,
+                                 int norm, int rope_dim, float rope_base, float eps, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * csa_index_topk — lightning indexer + top-k ([CS] "闪电索引器": index heads,
  * ReLU of the similarity, weighted over heads; only the top-k entries are kept
  * for the query, [LD]).  For query token t of sequence b at p = q_pos[b] + t:

@@ -58,6 +58,7 @@ def lib():
         "csa_fused_attention_workspace": ([I, I, I, I, I], SZ),
         "csa_fused_attention_splitkv": ([P, I, P, I, P, P, I64, P, I, I, P, I, I64, I, I, P, P, I, I, I, I, I, F, I, F,
                                          I, P, SZ, P, I, P], I),
+        "csa_compress_append": ([P, P, I, P, I, I, I, I, P, P, P, P, P, P, I64, I, I, F, F, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -120,6 +121,23 @@ def csa_compress(C, Z, B, m, overlap, *, Cb=None, Zb=None, norm=False, rope_dim=
                               _DT[C.dtype], int(norm), rope_dim, rope_base, eps, _ptr(out), _DT[out.dtype],
                               _stream(stream)), "csa_compress")
     return out
+
+
+def csa_compress_append(c_tok, z_tok, B, m, overlap, q_pos, ring_C, ring_Z, kv_nope, kv_rope, kv_scale, *,
+                        norm=True, rope_dim=64, rope_base=10000.0, eps=1e-6, stream=None):
+    """Decode-time cache writer: appends each sequence's new token (c_tok, z_tok
+    [n_seq, D]) at position q_pos[b] to its ring of the last 2m tokens
+    (ring_C, ring_Z [n_seq, 2m, D], same dtype) and, when the token completes a
+    block, writes the block's entry into the e4m3 cache row (kv_nope
+    [n_seq, cap, D-64] uint8, kv_rope [n_seq, cap, 64] bf16, kv_scale [n_seq, cap])."""
+    for t, n in ((c_tok, "c_tok"), (z_tok, "z_tok"), (B, "B"), (q_pos, "q_pos"), (ring_C, "ring_C"),
+                 (ring_Z, "ring_Z"), (kv_nope, "kv_nope"), (kv_rope, "kv_rope"), (kv_scale, "kv_scale")):
+        _dev(t, n)
+    n_seq, D = c_tok.shape
+    _check(lib().csa_compress_append(_ptr(c_tok), _ptr(z_tok), _DT[c_tok.dtype], _ptr(B), n_seq, D, m, int(overlap),
+                                     _ptr(q_pos), _ptr(ring_C), _ptr(ring_Z), _ptr(kv_nope), _ptr(kv_rope),
+                                     _ptr(kv_scale), kv_nope.shape[1], int(norm), rope_dim, rope_base, eps,
+                                     _stream(stream)), "csa_compress_append")
 
 
 def csa_rmsnorm_rope(x, rows_per_pos=1, pos0=0, *, norm=True, rope_dim=64, rope_base=10000.0, eps=1e-6,

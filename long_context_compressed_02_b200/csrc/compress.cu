@@ -16,6 +16,7 @@
 #include <cmath>
 #include <type_traits>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <math_constants.h>
 #include "common.cuh"
 
@@ -81,7 +82,6 @@ compress_kernel(const Tin* __restrict__ C, const Tin* __restrict__ Z, const Tin*
   float* s_red = sm + 3 * kThreads * 8;
 
   const int tid = threadIdx.x;
-  const int ngroups = kThreads / tpg;
   const int g = tid / tpg, c8 = tid % tpg;
   const int el = g / gpe, sub = g % gpe;
   const bool active_group = g < epc * gpe;
@@ -188,14 +188,6 @@ compress_kernel(const Tin* __restrict__ C, const Tin* __restrict__ Z, const Tin*
 // cos/sin for RoPE pair j at position pos: the angle pos * base^(-2j/r) is formed
 // and reduced modulo 2*pi in double (positions reach 2^20 and beyond), then the
 // reduced angle is evaluated in single precision.
-__device__ __forceinline__ float2 rope_cs_fast(int64_t pos, int j, int rope_dim, float rope_base) {
-  const double inv_freq = exp2(-2.0 * (double)j / (double)rope_dim * log2((double)rope_base));
-  double a = (double)pos * inv_freq;
-  a -= floor(a * 0.15915494309189535) * 6.283185307179586;
-  float sn, cs;
-  sincosf((float)a, &sn, &cs);
-  return make_float2(cs, sn);
-}
 
 // cos / sin of pos * theta_j with theta_j = ratio^j (ratio = base^(-2/rope_dim),
 // computed on the host in double): the power by squaring and the angle
@@ -384,6 +376,103 @@ rmsnorm_rope_bf16_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int 
   }
 }
 
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Block-wide reduction of one float per thread (sum or max); every thread
+// receives the result.
+template <bool MAX>
+__device__ __forceinline__ float block_reduce(float v, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = MAX ? fmaxf(v, w) : v + w;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();                                   // s_red free from any earlier use
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  float r = s_red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) r = MAX ? fmaxf(r, s_red[w]) : r + s_red[w];
+  return r;
+}
+
+// Decode-time cache writer.  One CTA per sequence: the new token's (C, Z) rows
+// go to slot pos % 2m of the sequence's ring of the last 2m tokens; if the
+// token completes block i = (pos + 1) / m - 1, the block's entry is pooled from
+// the ring (per-channel softmax of Z + B over the current block, and the
+// previous one when overlapping), RMS-normalised, rotated at position i * m,
+// and written as cache row i: the first D - rope_dim dims as e4m3 codes under
+// the row scale amax / 448, the RoPE dims as bf16, the scale as fp32.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads)
+compress_append_kernel(const Tin* __restrict__ c_tok, const Tin* __restrict__ z_tok, const float* __restrict__ B,
+                       int D, int m, int overlap, const int64_t* __restrict__ q_pos, Tin* __restrict__ ring_C,
+                       Tin* __restrict__ ring_Z, uint8_t* __restrict__ kv_nope, __nv_bfloat16* __restrict__ kv_rope,
+                       float* __restrict__ kv_scale, int64_t cap, int norm, int rope_dim, double ratio, float eps) {
+  extern __shared__ float s_row[];          // [D] the pooled entry
+  __shared__ float s_red[kThreads / 32];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int64_t pos = q_pos[b];
+  const int L = 2 * m;
+  Tin* rc = ring_C + (int64_t)b * L * D;
+  Tin* rz = ring_Z + (int64_t)b * L * D;
+  const int slot = (int)(pos % L);
+  // every thread only reads back its own channels, so no barrier is needed here
+  for (int c = tid; c < D; c += kThreads) {
+    rc[(int64_t)slot * D + c] = c_tok[(int64_t)b * D + c];
+    rz[(int64_t)slot * D + c] = z_tok[(int64_t)b * D + c];
+  }
+  if ((pos + 1) % m != 0) return;
+  const int64_t i = (pos + 1) / m - 1;
+  if (i >= cap) return;                     // the cache has no row for it (documented)
+  const int64_t first = (overlap && i > 0) ? (i - 1) * m : i * m;
+  const int nrows = (int)((i + 1) * m - first);
+  float ss = 0.f;
+  for (int c = tid; c < D; c += kThreads) {
+    float mx = -CUDART_INF_F, sum = 0.f, acc = 0.f;
+    for (int j = 0; j < nrows; ++j) {
+      const int sl = (int)((first + j) % L);
+      // bias row: the previous block uses rows 0..m-1, the current one m..2m-1
+      // (overlapping); a lone or non-overlapping block uses its own offset
+      const int brow = overlap ? (nrows == L ? j : m + j) : j;
+      const float lg = to_f(rz[(int64_t)sl * D + c]) + B[(int64_t)brow * D + c];
+      const float cv = to_f(rc[(int64_t)sl * D + c]);
+      if (lg > mx) {
+        const float a = __expf(mx - lg);
+        sum *= a;
+        acc *= a;
+        mx = lg;
+      }
+      const float e = __expf(lg - mx);
+      sum += e;
+      acc = fmaf(e, cv, acc);
+    }
+    const float v = acc / sum;
+    s_row[c] = v;
+    ss = fmaf(v, v, ss);
+  }
+  const float tot = block_reduce<false>(ss, s_red);
+  const float inv = norm ? rsqrtf(tot / (float)D + eps) : 1.f;
+  const int r0 = D - rope_dim, half = rope_dim / 2;
+  float am = 0.f;
+  for (int c = tid; c < r0; c += kThreads) am = fmaxf(am, fabsf(s_row[c] * inv));
+  const float amax = block_reduce<true>(am, s_red);   // its barrier also publishes s_row
+  const float scale = amax > 0.f ? amax / 448.f : 1.f;
+  const int64_t row = (int64_t)b * cap + i;
+  for (int c = tid; c < r0; c += kThreads)
+    kv_nope[row * r0 + c] = (uint8_t)__nv_cvt_float_to_fp8(s_row[c] * inv / scale, __NV_SATFINITE, __NV_E4M3);
+  for (int j = tid; j < rope_dim; j += kThreads) {
+    const int jj = j % half;
+    const float2 cs = rope_cs_pow(i * m, jj, ratio);
+    const float a = s_row[r0 + jj] * inv, bb = s_row[r0 + half + jj] * inv;
+    const float o = j < half ? a * cs.x - bb * cs.y : a * cs.y + bb * cs.x;
+    kv_rope[row * rope_dim + j] = __float2bfloat16_rn(o);
+  }
+  if (tid == 0) kv_scale[row] = scale;
+}
+
 template <typename Tin, typename Tout>
 csa_status_t launch_compress(const void* C, const void* Z, const void* Cb, const void* Zb, const float* B,
                              int64_t n_e, int D, int m, int overlap, int norm, int rope_dim,
@@ -483,4 +572,36 @@ extern "C" csa_status_t csa_rmsnorm_rope(const void* x, csa_dtype_t in_dtype, in
   if (in_dtype == CSA_BF16 && out_dtype == CSA_BF16) { CSA_NORM_CASE(__nv_bfloat16, __nv_bfloat16) }
 #undef CSA_NORM_CASE
   return fail(CSA_ERR_UNSUPPORTED, "csa_rmsnorm_rope: unsupported combination");
+}
+
+extern "C" csa_status_t csa_compress_append(const void* c_tok, const void* z_tok, csa_dtype_t in_dtype,
+                                            const float* B, int n_seq, int D, int m, int overlap,
+                                            const int64_t* q_pos, void* ring_C, void* ring_Z, uint8_t* kv_nope,
+                                            void* kv_rope, float* kv_scale, int64_t cap, int norm, int rope_dim,
+                                            float rope_base, float eps, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(n_seq >= 0 && cap >= 1, "csa_compress_append: n_seq >= 0 and cap >= 1 required");
+  CSA_REQUIRE(D % 8 == 0 && D >= 64 && D <= 2048, "csa_compress_append: D must be a multiple of 8 in [64, 2048]");
+  CSA_REQUIRE(m >= 1 && m <= 1024, "csa_compress_append: m must be in [1, 1024]");
+  CSA_REQUIRE(overlap == 0 || overlap == 1, "csa_compress_append: overlap must be 0 or 1");
+  CSA_REQUIRE(rope_dim == 0 || (rope_dim == 64 && D > 64), "csa_compress_append: rope_dim must be 0 or 64 (< D)");
+  CSA_REQUIRE(in_dtype == CSA_F32 || in_dtype == CSA_BF16, "csa_compress_append: in_dtype must be F32 or BF16");
+  if (n_seq == 0) return CSA_OK;
+  CSA_REQUIRE(c_tok && z_tok && B && q_pos && ring_C && ring_Z && kv_nope && kv_scale && (rope_dim == 0 || kv_rope),
+              "csa_compress_append: null pointer");
+  CSA_REQUIRE(aligned16(c_tok) && aligned16(z_tok) && aligned16(B) && aligned16(q_pos) && aligned16(ring_C) &&
+              aligned16(ring_Z) && aligned16(kv_nope) && aligned16(kv_scale) && (!kv_rope || aligned16(kv_rope)),
+              "csa_compress_append: pointers must be 16-byte aligned");
+  const double ratio = rope_dim > 0 ? std::pow((double)rope_base, -2.0 / (double)rope_dim) : 1.0;
+  const size_t smem = (size_t)D * sizeof(float);
+  if (in_dtype == CSA_F32) {
+    compress_append_kernel<float><<<n_seq, kThreads, smem, stream>>>(
+        (const float*)c_tok, (const float*)z_tok, B, D, m, overlap, q_pos, (float*)ring_C, (float*)ring_Z, kv_nope,
+        (__nv_bfloat16*)kv_rope, kv_scale, cap, norm, rope_dim, ratio, eps);
+  } else {
+    compress_append_kernel<__nv_bfloat16><<<n_seq, kThreads, smem, stream>>>(
+        (const __nv_bfloat16*)c_tok, (const __nv_bfloat16*)z_tok, B, D, m, overlap, q_pos, (__nv_bfloat16*)ring_C,
+        (__nv_bfloat16*)ring_Z, kv_nope, (__nv_bfloat16*)kv_rope, kv_scale, cap, norm, rope_dim, ratio, eps);
+  }
+  return check_launch("csa_compress_append");
 }
