@@ -432,22 +432,36 @@ compress_append_kernel(const Tin* __restrict__ c_tok, const Tin* __restrict__ z_
   float ss = 0.f;
   for (int c = tid; c < D; c += kThreads) {
     float mx = -CUDART_INF_F, sum = 0.f, acc = 0.f;
-    for (int j = 0; j < nrows; ++j) {
-      const int sl = (int)((first + j) % L);
-      // bias row: the previous block uses rows 0..m-1, the current one m..2m-1
-      // (overlapping); a lone or non-overlapping block uses its own offset
-      const int brow = overlap ? (nrows == L ? j : m + j) : j;
-      const float lg = to_f(rz[(int64_t)sl * D + c]) + B[(int64_t)brow * D + c];
-      const float cv = to_f(rc[(int64_t)sl * D + c]);
-      if (lg > mx) {
-        const float a = __expf(mx - lg);
-        sum *= a;
-        acc *= a;
-        mx = lg;
+    // rows in batches of 8, all loads of a batch issued before the softmax update
+    for (int j0 = 0; j0 < nrows; j0 += 8) {
+      float lg[8], cv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u;
+        lg[u] = -CUDART_INF_F;
+        cv[u] = 0.f;
+        if (j < nrows) {
+          const int sl = (int)((first + j) % L);
+          // bias row: the previous block uses rows 0..m-1, the current one m..2m-1
+          // (overlapping); a lone or non-overlapping block uses its own offset
+          const int brow = overlap ? (nrows == L ? j : m + j) : j;
+          lg[u] = to_f(rz[(int64_t)sl * D + c]) + B[(int64_t)brow * D + c];
+          cv[u] = to_f(rc[(int64_t)sl * D + c]);
+        }
       }
-      const float e = __expf(lg - mx);
-      sum += e;
-      acc = fmaf(e, cv, acc);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (j0 + u >= nrows) break;
+        if (lg[u] > mx) {
+          const float a = __expf(mx - lg[u]);
+          sum *= a;
+          acc *= a;
+          mx = lg[u];
+        }
+        const float e = __expf(lg[u] - mx);
+        sum += e;
+        acc = fmaf(e, cv[u], acc);
+      }
     }
     const float v = acc / sum;
     s_row[c] = v;
