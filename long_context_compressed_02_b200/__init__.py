@@ -134,6 +134,13 @@ def csa_compress_append(c_tok, z_tok, B, m, overlap, q_pos, ring_C, ring_Z, kv_n
                  (ring_Z, "ring_Z"), (kv_nope, "kv_nope"), (kv_rope, "kv_rope"), (kv_scale, "kv_scale")):
         _dev(t, n)
     n_seq, D = c_tok.shape
+    if z_tok.shape != c_tok.shape or ring_C.dtype != c_tok.dtype or ring_Z.dtype != c_tok.dtype or \
+            tuple(ring_C.shape) != (n_seq, 2 * m, D) or tuple(ring_Z.shape) != (n_seq, 2 * m, D):
+        raise CsaError("csa_compress_append: c_tok/z_tok [n_seq, D] and rings [n_seq, 2m, D] of one dtype expected")
+    if kv_nope.shape[:2] != kv_rope.shape[:2] or tuple(kv_scale.shape) != tuple(kv_nope.shape[:2]) or \
+            kv_nope.shape[0] != n_seq or kv_nope.shape[2] + rope_dim != D:
+        raise CsaError("csa_compress_append: cache rows [n_seq, cap, D - rope_dim] / [n_seq, cap, rope_dim] / "
+                       "[n_seq, cap] expected")
     _check(lib().csa_compress_append(_ptr(c_tok), _ptr(z_tok), _DT[c_tok.dtype], _ptr(B), n_seq, D, m, int(overlap),
                                      _ptr(q_pos), _ptr(ring_C), _ptr(ring_Z), _ptr(kv_nope), _ptr(kv_rope),
                                      _ptr(kv_scale), kv_nope.shape[1], int(norm), rope_dim, rope_base, eps,

@@ -86,6 +86,27 @@ def test_host_argument_validation(L):
     assert st == 1 and b"inv_rope" in L.csa_last_error()
 
 
+def test_cache_writer_host_validation(L):
+    """csa_compress_append rejects bad shapes and pointers before any device work."""
+    v = ctypes.c_void_p(16)
+    args = dict(c=v, z=v, dt=1, B=v, n=2, D=512, m=4, ov=1, pos=v, rc=v, rz=v, kn=v, kr=v, ks=v, cap=16, norm=1,
+                rope=64, base=10000.0, eps=1e-6)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return L.csa_compress_append(a["c"], a["z"], a["dt"], a["B"], a["n"], a["D"], a["m"], a["ov"], a["pos"],
+                                     a["rc"], a["rz"], a["kn"], a["kr"], a["ks"], a["cap"], a["norm"], a["rope"],
+                                     a["base"], a["eps"], None)
+    assert call(D=500) == 1 and b"multiple of 8" in L.csa_last_error()
+    assert call(m=0) == 1 and b"m must be" in L.csa_last_error()
+    assert call(rope=32) == 1 and b"rope_dim" in L.csa_last_error()
+    assert call(dt=2) == 1 and b"in_dtype" in L.csa_last_error()
+    assert call(cap=0) == 1
+    assert call(rz=None) == 1 and b"null" in L.csa_last_error()
+    assert call(kn=ctypes.c_void_p(24)) == 1 and b"aligned" in L.csa_last_error()
+    assert call(n=0) == 0                                    # nothing to do
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     import long_context_compressed_02_b200 as csa
