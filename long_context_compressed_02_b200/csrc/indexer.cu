@@ -395,7 +395,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
 }
 
 // ------------------------------------------------------------------ top-k
-constexpr int kTopkThreads = 512;
+constexpr int kTopkThreads = 512;      // histogram, filtered-chunk and merge kernels
+constexpr int kTopkThreadsSmall = 256; // rows of one chunk: smaller CTAs, twice as many in flight
 constexpr int kChunk = 16384;          // keys per shared-memory chunk (64 KB)
 constexpr int kMergeCap = 16384;       // candidates per row in the merge stage
 constexpr int kHistBins = 4096;        // rows split into chunks: histogram of the top 12 key bits
@@ -405,16 +406,18 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+template <int NTH>
 struct SelectSmem {
-  uint32_t whist[kTopkThreads / 32][256];
-  uint32_t wlo[kTopkThreads / 32], whi[kTopkThreads / 32];
+  uint32_t whist[NTH / 32][256];
+  uint32_t wlo[NTH / 32], whi[NTH / 32];
   uint32_t hist[256];
-  uint64_t warp_tot[kTopkThreads / 32];
+  uint64_t warp_tot[NTH / 32];
   uint32_t digit, above;
 };
 
 // Block-wide inclusive scan of a packed (gt << 32 | eq) count.
-__device__ __forceinline__ uint64_t block_scan_incl(uint64_t v, SelectSmem& ss) {
+template <int NTH>
+__device__ __forceinline__ uint64_t block_scan_incl(uint64_t v, SelectSmem<NTH>& ss) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -432,8 +435,9 @@ __device__ __forceinline__ uint64_t block_scan_incl(uint64_t v, SelectSmem& ss) 
 // Selects the top-k of keys[0..n) (ties to the lower position) and writes
 // out[pos] = ids[e] (or id_base + e when ids == null) in ascending position
 // order; also returns the count written (min(k, n)).  All threads participate.
+template <int NTH>
 __device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id_base, int n, int k,
-                            int32_t* out_idx, uint32_t* out_key, SelectSmem& ss) {
+                            int32_t* out_idx, uint32_t* out_key, SelectSmem<NTH>& ss) {
   const int tid = threadIdx.x;
   uint32_t T = 0;
   int need_eq = 0;
@@ -443,7 +447,7 @@ __device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id
     // every key: the 8-bit digits start just below them, so the first histogram
     // spreads over the data instead of piling onto one bin.
     uint32_t lo = 0xffffffffu, hi = 0u;
-    for (int e = tid; e < n; e += kTopkThreads) { const uint32_t key = keys[e]; lo = min(lo, key); hi = max(hi, key); }
+    for (int e = tid; e < n; e += NTH) { const uint32_t key = keys[e]; lo = min(lo, key); hi = max(hi, key); }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
@@ -452,7 +456,7 @@ __device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id
     if ((tid & 31) == 0) { ss.wlo[tid >> 5] = lo; ss.whi[tid >> 5] = hi; }
     __syncthreads();
     lo = ss.wlo[0]; hi = ss.whi[0];
-    for (int w = 1; w < kTopkThreads / 32; ++w) { lo = min(lo, ss.wlo[w]); hi = max(hi, ss.whi[w]); }
+    for (int w = 1; w < NTH / 32; ++w) { lo = min(lo, ss.wlo[w]); hi = max(hi, ss.whi[w]); }
     const uint32_t diff = lo ^ hi;
     const int top = diff ? 31 - __clz(diff) : -1;           // highest differing bit
     uint32_t mask = top >= 31 ? 0u : ~((2u << top) - 1u);   // common high bits
@@ -461,18 +465,18 @@ __device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id
     for (int shift = top - 7; shift > -8; shift -= 8) {
       const int sh = max(shift, 0);
       const uint32_t dmask = shift >= 0 ? 255u : (255u >> (-shift));   // width of this digit
-      for (int i = tid; i < 256 * (kTopkThreads / 32); i += kTopkThreads) (&ss.whist[0][0])[i] = 0;
+      for (int i = tid; i < 256 * (NTH / 32); i += NTH) (&ss.whist[0][0])[i] = 0;
       __syncthreads();
       // per-warp private histograms
-      for (int e = tid; e < n; e += kTopkThreads) {
+      for (int e = tid; e < n; e += NTH) {
         const uint32_t key = keys[e];
         if ((key & mask) == prefix) atomicAdd(&ss.whist[tid >> 5][(key >> sh) & dmask], 1u);
       }
       __syncthreads();
-      for (int i = tid; i < 256; i += kTopkThreads) {
+      for (int i = tid; i < 256; i += NTH) {
         uint32_t t = 0;
 #pragma unroll
-        for (int w = 0; w < kTopkThreads / 32; ++w) t += ss.whist[w][i];
+        for (int w = 0; w < NTH / 32; ++w) t += ss.whist[w][i];
         ss.hist[i] = t;
       }
       __syncthreads();
@@ -508,7 +512,7 @@ __device__ int block_select(const uint32_t* keys, const int32_t* ids, int64_t id
     need_eq = remaining;
   }
   // stable compaction in position order
-  const int per = (n + kTopkThreads - 1) / kTopkThreads;
+  const int per = (n + NTH - 1) / NTH;
   const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
   uint32_t gt = 0, eq = 0;
   if (!all) {
@@ -574,7 +578,7 @@ topk_hist_kernel(TopkParams p) {
 // among the row's top k.  All threads call; the result is broadcast.  Thread t
 // owns the 8 bins [4096 - 8 (t + 1), 4096 - 8 t), so a prefix scan in thread
 // order counts the keys in higher bins.
-__device__ uint32_t topk_threshold_bin(const uint32_t* g, int k, SelectSmem& ss, uint32_t* s_out) {
+__device__ uint32_t topk_threshold_bin(const uint32_t* g, int k, SelectSmem<kTopkThreads>& ss, uint32_t* s_out) {
   constexpr int kPer = kHistBins / kTopkThreads;         // 8
   const int tid = threadIdx.x;
   const int top = kHistBins - kPer * tid;
@@ -605,10 +609,11 @@ __device__ uint32_t topk_threshold_bin(const uint32_t* g, int k, SelectSmem& ss,
 // (Two instances, so that the filtered path's extra state does not cost the
 // single-chunk path occupancy.)
 template <bool FILTERED>
-__global__ void __launch_bounds__(kTopkThreads, FILTERED ? 2 : 4)
+__global__ void __launch_bounds__(FILTERED ? kTopkThreads : kTopkThreadsSmall, FILTERED ? 2 : 8)
 topk_chunk_kernel(TopkParams p) {
   extern __shared__ uint32_t s_keys[];   // kChunk keys (or kChunk / 2 keys + kChunk / 2 ids)
-  __shared__ SelectSmem ss;
+  constexpr int NTH = FILTERED ? kTopkThreads : kTopkThreadsSmall;
+  __shared__ SelectSmem<NTH> ss;
   __shared__ uint32_t s_B;
   const int64_t row = blockIdx.x;
   const int chunk = blockIdx.y;
@@ -618,19 +623,19 @@ topk_chunk_kernel(TopkParams p) {
   const int n = (int)max((int64_t)0, min((int64_t)kChunk, nv - lo));
   const float* src = p.scores + row * p.cap + lo;
   if constexpr (!FILTERED) {
-    for (int e = threadIdx.x; e < n; e += kTopkThreads) s_keys[e] = order_key(src[e]);
+    for (int e = threadIdx.x; e < n; e += NTH) s_keys[e] = order_key(src[e]);
     __syncthreads();
     int32_t* out = p.idx + row * p.k;
     int cnt = block_select(s_keys, nullptr, lo, n, p.k, out, nullptr, ss);
-    for (int i = cnt + threadIdx.x; i < p.k; i += kTopkThreads) out[i] = -1;
+    for (int i = cnt + threadIdx.x; i < p.k; i += NTH) out[i] = -1;
     return;
   } else {
     // Only keys in or above the row's threshold bin can be selected.  Warp w
     // owns the 1024 consecutive keys [1024 w, 1024 w + 1024) of the chunk: a
     // counting pass (ballots) gives each warp its output offset, then a writing
     // pass emits the survivors in index order.
-    __shared__ uint32_t s_wcnt[kTopkThreads / 32];
-    constexpr int kWarps = kTopkThreads / 32;
+    __shared__ uint32_t s_wcnt[NTH / 32];
+    constexpr int kWarps = NTH / 32;
     constexpr int kPerWarp = kChunk / kWarps;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t B = topk_threshold_bin(p.hist + row * kHistBins, p.k, ss, &s_B);
@@ -675,7 +680,7 @@ topk_chunk_kernel(TopkParams p) {
       return;
     }
     // many keys share the threshold bin: local top-k of the whole chunk by position
-    for (int e = threadIdx.x; e < n; e += kTopkThreads) s_keys[e] = order_key(src[e]);
+    for (int e = threadIdx.x; e < n; e += NTH) s_keys[e] = order_key(src[e]);
     __syncthreads();
     const int c = block_select(s_keys, nullptr, lo, n, p.k, p.cand_idx + o, p.cand_key + o, ss);
     if (threadIdx.x == 0) p.cand_cnt[row * p.n_chunks + chunk] = c;
@@ -689,7 +694,7 @@ topk_merge_kernel(TopkParams p) {
   extern __shared__ uint32_t s_mem[];
   uint32_t* s_keys = s_mem;                                   // kMergeCap
   int32_t* s_ids = reinterpret_cast<int32_t*>(s_mem + kMergeCap);
-  __shared__ SelectSmem ss;
+  __shared__ SelectSmem<kTopkThreads> ss;
   __shared__ int s_off[65];
   const int64_t row = blockIdx.x;
   if (threadIdx.x < 64) {
@@ -866,7 +871,7 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
     st = check_launch("csa_index_topk(histogram)");
     if (st != CSA_OK) return st;
   }
-  chunk_kernel<<<g1, kTopkThreads, smem1, stream>>>(tp);
+  chunk_kernel<<<g1, L.n_chunks > 1 ? kTopkThreads : kTopkThreadsSmall, smem1, stream>>>(tp);
   st = check_launch("csa_index_topk(select)");
   if (st != CSA_OK) return st;
   if (L.n_chunks > 1) {
