@@ -219,7 +219,7 @@ def test_fused_equals_separate_calls():
     sep = csa.swa_sink_combine(q, kt, pos, W, sink, Op, Lp, inv_rope=True, out_dtype=torch.float32)
     fus = csa.csa_fused_attention(q, kv, kt, pos, W, sink, idx=idx, inv_rope=True, out_dtype=torch.float32)
     csa.check_device_error()
-    # both paths are bf16-probability approximations of the same softmax: the benchmark spec tolerance
+    # both paths are bf16-probability approximations of the same softmax: the parity tolerance
     assert_close(host(fus), host(sep), what="fused vs separate")
 
 
