@@ -90,6 +90,35 @@ def test_flash_prefill_full_size_sampled_rows():
     assert_close(host(out[torch.from_numpy(rows).cuda()]), ref, what="full-size sampled rows")
 
 
+def test_hca_prefill_full_size_sampled_rows():
+    """The HCA benchmark workload (S 131072, 64 x 512, m' 128, 1024 entries)
+    through the fused layer on the GPU; sampled rows (block edges, the first
+    and last tokens) against the oracle's definition, assembled from its steps
+    so that only the sampled queries are brought to the host."""
+    import long_context_compressed_02_b200 as csa
+    inp, cfg = synth.prefill_inputs_device("hca_prefill", "cuda", seed=0)
+    m, W = cfg["m"], cfg["W"]
+    out = csa.hca_layer_prefill(inp["q"], inp["C"], inp["Z"], inp["B"], inp["sink"], m=m, W=W, norm_rope=True,
+                                inv_rope=True)
+    csa.check_device_error()
+    rows = np.array([0, 127, 128, 129, 255, 4095, 65535, 65536, 131071])
+    ri = torch.from_numpy(rows).cuda()
+    q_rows = inp["q"][ri].float().cpu().numpy().astype(np.float64)
+    C = inp["C"].float().cpu().numpy().astype(np.float64)
+    Z = inp["Z"].float().cpu().numpy().astype(np.float64)
+    B = inp["B"].cpu().numpy().astype(np.float64)
+    sink = inp["sink"].cpu().numpy()
+    qn = O.bf16_round(O.rope_partial(O.rmsnorm(q_rows), rows[:, None], 64))
+    lo = max(0, rows.min() - W)                      # window rows the sampled queries can see
+    kt = np.zeros_like(C)
+    kt[lo:] = O.bf16_round(O.rope_partial(O.rmsnorm(C[lo:]), np.arange(lo, C.shape[0]), 64))
+    kv = O.bf16_round(O.rope_partial(O.rmsnorm(O.compress(C, Z, B, m, False)),
+                                     np.arange(C.shape[0] // m) * m, 64))
+    Op, lp = O.dense_attention_partial(qn, kv, O.n_visible(rows, m))
+    ref = O.window_sink_combine(qn, kt, rows, W, sink, Op, lp, inv_rope=True, rope_dim=64)
+    assert_close(host(out[ri]), ref, what="HCA full-size sampled rows")
+
+
 @pytest.mark.parametrize("grid", [True, False])
 def test_csa_decode_1m_full_size_sampled(grid):
     """The 1M-context decode workload (16 sequences x 2^18 e4m3 entries): the
