@@ -38,7 +38,14 @@ argument whose default is the reading):
   * RMSNorm over all D dims, eps 1e-6, unit gain [CS "其他辅助设计"];
   * partial RoPE on dims [D-64, D), pairs (d, d+32), theta_j = 10000^(-2j/64);
     positions: query t, CSA/HCA entry i -> i*m, window token u -> u;
-  * inverse RoPE (rotation by -t) on the last 64 dims of the output [LD].
+  * inverse RoPE (rotation by -t) on the last 64 dims of the output [LD];
+  * the first layers of the stack are window-only: window + sink, no
+    compressed branch [LQ §3, note after the config block];
+  * grouped output projection [LQ §3 config: output_proj_groups 8,
+    intermediate_attn_dim 1024, hidden_size 4096]: consecutive heads form a
+    group, each group has its own [d_mid, (H/G)*D] matrix, the concatenated
+    group outputs go through one [d_model, G*d_mid] matrix, no bias; the
+    intermediate is stored as bf16 like every other activation of the layer.
 """
 from __future__ import annotations
 
@@ -56,6 +63,7 @@ __all__ = [
     "csa_layer", "hca_layer", "csa_layer_matrix", "hca_layer_matrix",
     "csa_decode", "hca_decode", "flop_counts",
     "fp8_row_quantize", "stream_append",
+    "swa_layer", "grouped_out_proj",
 ]
 
 # ----------------------------------------------------------------------------
@@ -493,6 +501,58 @@ def hca_decode(q, kv, swa, sink, t, *, m=128, inv_rope=True, rope_dim=64, rope_b
                             inv_rope=inv_rope, rope_dim=rope_dim, rope_base=rope_base,
                             window_rows=[swa])
     return O[0]
+
+
+# ----------------------------------------------------------------------------
+# The rest of the layer stack [LQ §3, config block and the note after it]: the
+# first layers attend through the sliding window only, and every layer's
+# attention output goes through a grouped output projection
+# (output_proj_groups 8, intermediate_attn_dim 1024, hidden_size 4096).
+# ----------------------------------------------------------------------------
+
+def swa_layer(q, C, sink, *, W: int = 128, norm_rope: bool = False, inv_rope: bool = False,
+              rope_dim: int = 64, rope_base: float = 10000.0, store_round=None, rows=None):
+    """Sliding-window-only layer: each query attends to the raw tokens
+    [max(0, t-W+1), t] and the sink in one softmax; no compressed branch.
+    Same normalisation, RoPE and window rows as csa_layer / hca_layer."""
+    S = np.asarray(C).shape[0]
+    rows = np.arange(S) if rows is None else np.asarray(rows)
+    qr = np.asarray(q, np.float64)[rows]
+    qn, kt = _prep(qr, C, rows, norm_rope, rope_dim, rope_base)
+    if store_round:
+        qn, kt = store_round(qn), store_round(kt)
+    T, H, _ = qn.shape
+    empty_O, empty_lse = np.zeros(qn.shape), np.full((T, H), -np.inf)
+    return window_sink_combine(qn, kt, rows, W, sink, empty_O, empty_lse, inv_rope=inv_rope,
+                               rope_dim=rope_dim, rope_base=rope_base)
+
+
+def grouped_out_proj(O, w_grp, w_out, *, mid_round=None, return_mid: bool = False):
+    """Grouped output projection of an attention output O [T, H, D].
+
+    The H heads form G = w_grp.shape[0] groups of H/G consecutive heads.  Group
+    g's heads, concatenated in head order ([T, (H/G)*D]), are mapped by its own
+    matrix w_grp[g] ([d_mid, (H/G)*D], laid out [out, in]) to d_mid dims; the
+    G results, concatenated in group order ([T, G*d_mid]), are mapped by
+    w_out ([d_model, G*d_mid]) to the model width.  No bias.  mid_round rounds
+    the intermediate to its storage type (e.g. bf16_round).
+    Returns out [T, d_model] (and the intermediate if return_mid)."""
+    O = np.asarray(O, np.float64)
+    w_grp = np.asarray(w_grp, np.float64)
+    T, H, D = O.shape
+    G, d_mid, d_in = w_grp.shape
+    if H % G or d_in != (H // G) * D:
+        raise ValueError("w_grp must be [G, d_mid, (H/G)*D] with G dividing H")
+    hg = H // G
+    parts = []
+    for g in range(G):
+        X = O[:, g * hg:(g + 1) * hg, :].reshape(T, hg * D)
+        parts.append(X @ w_grp[g].T)
+    mid = np.concatenate(parts, axis=1)
+    if mid_round is not None:
+        mid = mid_round(mid)
+    out = mid @ np.asarray(w_out, np.float64).T
+    return (out, mid) if return_mid else out
 
 
 # ----------------------------------------------------------------------------
