@@ -367,6 +367,45 @@ def hca_prefill_leg(dev, steps, warmup, csa, synth, torch, seed=0):
                          "peak_source": f"{src} bf16 sustained"}}
 
 
+def out_proj_leg(dev, steps, warmup, csa, synth, torch, seed=0, S=None):
+    """Grouped output projection of one prefill layer's attention output:
+    16384 tokens, 64 heads x 512 in 8 groups -> 8 x 1024 (bf16 intermediate)
+    -> 4096; two launches of the tcgen05 GEMM kernel per step.  The input
+    (1 GiB) is larger than L2."""
+    x, cfg = synth.out_proj_inputs_device(dev, seed=seed, S=S)
+    S, H, D, G, dm, dmod = (cfg[k] for k in ("S", "H", "D", "G", "d_mid", "d_model"))
+    bf = torch.bfloat16
+    mid = torch.empty(S, G * dm, dtype=bf, device=dev)
+    out = torch.empty(S, dmod, dtype=bf, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        csa.csa_grouped_out_proj(x["o"], x["w_grp"], x["w_out"], mid=mid, out=out)
+
+    for _ in range(max(3, warmup)):
+        step()
+    csa.check_device_error()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    fl_group = 2 * S * H * D * dm
+    fl_out = 2 * S * G * dm * dmod
+    _, bf16_burst, _, src = _peaks()
+    ach = (fl_group + fl_out) / (ms * 1e-3) / 1e12
+    return {"workload": "out_proj", "S": S, "H": H, "D": D, "groups": G, "d_mid": dm, "d_model": dmod,
+            "ms_per_step": ms, "tflops": ach, "tokens_per_s": S / (ms * 1e-3),
+            "flops_per_step": {"group_stage": fl_group, "output_stage": fl_out},
+            "roofline": {"kernel": "proj_gemm", "bound": "tensor", "achieved": ach, "peak": bf16_burst,
+                         "unit": "TFLOP/s", "frac": ach / bf16_burst, "traffic": None,
+                         "peak_source": f"{src} bf16 burst (the leg runs alone, a few ms)"}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -381,6 +420,8 @@ def main():
     ap.add_argument("--no-prefill", action="store_true", help="run only the decode legs (profiling cases only)")
     ap.add_argument("--no-hca", action="store_true", help="skip the HCA prefill leg (S 131072)")
     ap.add_argument("--no-mixed", action="store_true", help="skip the 4-layer mixed decode leg")
+    ap.add_argument("--no-out-proj", action="store_true", help="skip the grouped output projection leg")
+    ap.add_argument("--out-proj-only", action="store_true", help="run only the output projection leg (profiling)")
     args = ap.parse_args()
     from long_context_compressed_02_b200 import replicas
     rank, world, local = replicas.rank_world()
@@ -402,6 +443,11 @@ def main():
     build.build()
     csa.lib()
 
+    if args.out_proj_only:
+        leg = out_proj_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=replicas.replica_seed(rank), S=args.S)
+        if rank == 0:
+            print(json.dumps({"out_proj": leg}), flush=True)
+        return
     if args.no_prefill:
         out = {}
         if not args.no_decode:
@@ -566,7 +612,7 @@ def main():
                "sample": f"{n_rows} evenly spaced query rows of the same S=16384 layer (float64 numpy oracle, "
                          f"{dt:.1f} s including its full-sequence compressor and window-row passes)"}
 
-    hca = mixed = None
+    hca = mixed = proj = None
     if args.S is None:
         del inp, qn, kt, kv, idx, ws, out
         torch.cuda.empty_cache()
@@ -575,6 +621,9 @@ def main():
             torch.cuda.empty_cache()
         if not args.no_mixed:
             mixed = mixed_decode_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=replicas.replica_seed(rank))
+            torch.cuda.empty_cache()
+        if not args.no_out_proj:
+            proj = out_proj_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=replicas.replica_seed(rank))
             torch.cuda.empty_cache()
 
     if rank == 0:
@@ -589,7 +638,7 @@ def main():
                                               "indexer_fp8": fl_index}},
                 "prefill_tokens_per_s": replicas.job_rate(S, world, ms * 1e-3),
                 "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode,
-                "hca_prefill": hca, "decode_mixed": mixed,
+                "hca_prefill": hca, "decode_mixed": mixed, "out_proj": proj,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -291,6 +291,27 @@ csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q_dtype, con
                                          int n_split, void* workspace, size_t ws_bytes, void* out,
                                          csa_dtype_t out_dtype, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * csa_grouped_out_proj — grouped output projection of a layer's attention
+ * output ([LQ] §3 config block: output_proj_groups 8, intermediate_attn_dim
+ * 1024, hidden_size 4096).  The H heads form G groups of H/G consecutive heads;
+ *   mid[t, g*d_mid + r] = sum_j w_grp[g, r, j] * o[t, g*H/G + j/D, j%D]
+ *                         (j < (H/G)*D: the group's heads concatenated in order)
+ *   out[t, c]           = sum_i w_out[c, i] * mid[t, i]        (i < G*d_mid)
+ * No bias.  Weights are laid out [out_features, in_features].
+ *   o      [M, H, D] BF16 (e.g. the output of csa_fused_attention).
+ *   w_grp  [G, d_mid, (H/G)*D] BF16.   w_out [d_model, G*d_mid] BF16.
+ *   mid    [M, G*d_mid] BF16, caller-owned; holds the rounded intermediate on
+ *          return (fp32 accumulation, one bf16 rounding).
+ *   out    [M, d_model], out_dtype F32 or BF16 (fp32 accumulation).
+ * Two launches on `stream` (group stage, output stage).  (H/G)*D must be a
+ * multiple of 64, d_mid and d_model multiples of 256 (else
+ * CSA_ERR_UNSUPPORTED); M = 0 is a no-op (pointers may then be NULL).
+ * ------------------------------------------------------------------------- */
+csa_status_t csa_grouped_out_proj(const void* o, const void* w_grp, const void* w_out, int M, int H, int D,
+                                  int G, int d_mid, int d_model, void* mid, void* out, csa_dtype_t out_dtype,
+                                  cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -6,9 +6,11 @@ the current stream.  There is no fallback: if libcsa.so is missing or a call
 fails, an exception is raised.
 
 Entry points (same names as the C ABI):
-  csa_compress, csa_rmsnorm_rope, csa_index_topk, csa_sparse_mqa,
-  hca_dense_attn, swa_sink_combine, csa_fused_attention
-and two compositions of them: csa_layer_prefill, hca_layer_prefill.
+  csa_compress, csa_compress_append, csa_rmsnorm_rope, csa_index_topk,
+  csa_sparse_mqa, hca_dense_attn, swa_sink_combine, csa_fused_attention,
+  csa_grouped_out_proj
+and compositions of them: csa_layer_prefill, hca_layer_prefill,
+swa_layer_prefill, csa_layer_decode, hca_layer_decode, swa_layer_decode.
 """
 from __future__ import annotations
 
@@ -59,6 +61,7 @@ def lib():
         "csa_fused_attention_splitkv": ([P, I, P, I, P, P, I64, P, I, I, P, I, I64, I, I, P, P, I, I, I, I, I, F, I, F,
                                          I, P, SZ, P, I, P], I),
         "csa_compress_append": ([P, P, I, P, I, I, I, I, P, P, P, P, P, P, I64, I, I, F, F, P], I),
+        "csa_grouped_out_proj": ([P, P, P, I, I, I, I, I, I, P, P, I, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -280,6 +283,31 @@ def csa_fused_attention(q, kv, kv_tok, q_pos, W, sink, *, idx=None, m=1, kv_rope
     return out
 
 
+def csa_grouped_out_proj(o, w_grp, w_out, *, mid=None, out=None, out_dtype=torch.bfloat16, return_mid=False,
+                         stream=None):
+    """Grouped output projection: o [M, H, D] bf16; w_grp [G, d_mid, (H/G)*D]
+    bf16 (group g = heads g*H/G ..); w_out [d_model, G*d_mid] bf16.  Returns
+    out [M, d_model] (and the bf16 intermediate [M, G*d_mid] if return_mid)."""
+    for t, n in ((o, "o"), (w_grp, "w_grp"), (w_out, "w_out"), (mid, "mid"), (out, "out")):
+        _dev(t, n)
+    M, H, D = o.shape
+    G, d_mid, d_in = w_grp.shape
+    d_model = w_out.shape[0]
+    if o.dtype != torch.bfloat16 or w_grp.dtype != torch.bfloat16 or w_out.dtype != torch.bfloat16:
+        raise CsaError("csa_grouped_out_proj: o, w_grp and w_out must be bf16")
+    if H % G or d_in != (H // G) * D or tuple(w_out.shape) != (d_model, G * d_mid):
+        raise CsaError("csa_grouped_out_proj: w_grp [G, d_mid, (H/G)*D] and w_out [d_model, G*d_mid] expected")
+    if mid is None:
+        mid = torch.empty((M, G * d_mid), dtype=torch.bfloat16, device=o.device)
+    if out is None:
+        out = torch.empty((M, d_model), dtype=out_dtype, device=o.device)
+    if mid.dtype != torch.bfloat16 or tuple(mid.shape) != (M, G * d_mid) or tuple(out.shape) != (M, d_model):
+        raise CsaError("csa_grouped_out_proj: mid [M, G*d_mid] bf16 and out [M, d_model] expected")
+    _check(lib().csa_grouped_out_proj(_ptr(o), _ptr(w_grp), _ptr(w_out), M, H, D, G, d_mid, d_model, _ptr(mid),
+                                      _ptr(out), _DT[out.dtype], _stream(stream)), "csa_grouped_out_proj")
+    return (out, mid) if return_mid else out
+
+
 # ---------------------------------------------------------------- layers
 
 def csa_layer_prefill(q, C, Z, B, qI, w, kI, sink, *, k, m=4, W=128, norm_rope=False, inv_rope=False,
@@ -331,6 +359,31 @@ def hca_layer_prefill(q, C, Z, B, sink, *, m=128, W=128, norm_rope=False, inv_ro
         out = swa_sink_combine(qn[None], kt[None], pos, W, sink, Op, Lp, window_mode=0, inv_rope=inv_rope,
                                rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
     return out[0]
+
+
+def swa_layer_prefill(q, C, sink, *, W=128, norm_rope=False, inv_rope=False, rope_dim=64, rope_base=10000.0,
+                      kv_dtype=None):
+    """One sliding-window-only layer (batch 1): window + sink attention over the
+    raw tokens, no compressed branch.  q [S, H, D], C [S, D], sink [H]."""
+    S, H, D = q.shape
+    kv_dtype = q.dtype if kv_dtype is None else kv_dtype
+    pos = torch.zeros(1, dtype=torch.int64, device=q.device)
+    if norm_rope:
+        qn = csa_rmsnorm_rope(q, rows_per_pos=H, rope_dim=rope_dim, rope_base=rope_base)
+        kt = csa_rmsnorm_rope(C, rows_per_pos=1, rope_dim=rope_dim, rope_base=rope_base, out_dtype=kv_dtype)
+    else:
+        qn, kt = q, C
+    out = swa_sink_combine(qn[None], kt[None], pos, W, sink, window_mode=0, inv_rope=inv_rope,
+                           rope_dim=rope_dim if norm_rope else 0, rope_base=rope_base)
+    return out[0]
+
+
+def swa_layer_decode(lay, q_pos, *, W=128, out=None, stream=None):
+    """One sliding-window-only layer, one decode step per sequence: the SWA
+    cache and the sink in one softmax, inverse RoPE at q_pos.  `lay` holds q,
+    swa and sink (the layout of synth's decode inputs)."""
+    return swa_sink_combine(lay["q"], lay["swa"], q_pos, W, lay["sink"], window_mode=1, inv_rope=True,
+                            rope_dim=64, out=out, stream=stream)
 
 
 def csa_layer_decode(lay, q_pos, *, k, m=4, W=128, n_split=1, idx=None, out=None, index_workspace=None,

@@ -31,6 +31,7 @@ inline int num_sms() {
 // exposes a reader that returns and clears it (synchronous).
 uint32_t read_clear_err_indexer();
 uint32_t read_clear_err_attention();
+uint32_t read_clear_err_proj();
 
 }  // namespace csa
 

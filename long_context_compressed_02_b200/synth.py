@@ -12,6 +12,8 @@ Workloads (names used across tests and the benchmark):
   csa_decode_1m batch 16, context 2^20, caches: e4m3 KV [2^18, 448] + bf16 RoPE
                 [2^18, 64] + fp32 row scale; e4m3 indexer keys [2^18, 128] + scale.
   mixed_decode  batch 32, context U[64K, 1M], layers CSA, HCA, CSA, HCA, top-k 1024.
+  out_proj      grouped output projection of a prefill layer's attention output:
+                S 16384 tokens, 64 heads x 512 in 8 groups -> 8 x 1024 -> 4096.
 """
 from __future__ import annotations
 
@@ -27,6 +29,7 @@ WORKLOADS = {
                         norm_rope=True, inv_rope=True, sink="normal"),
     "csa_decode_1m": dict(batch=16, ctx=1 << 20, H=64, D=512, m=4, HI=64, DI=128, k=512, W=128,
                           rope_dim=64),
+    "out_proj": dict(S=16384, H=64, D=512, G=8, d_mid=1024, d_model=4096),
     "mixed_decode": dict(batch=32, ctx_lo=65536, ctx_hi=1 << 20, H=64, D=512, HI=64, DI=128,
                          k=1024, W=128, rope_dim=64, layers=("csa", "hca", "csa", "hca")),
 }
@@ -260,3 +263,23 @@ def mixed_decode_inputs_device(device, seed: int = 0, grid: bool = False, batch:
         layers.append(lay)
     q_pos = torch.as_tensor(L - 1, dtype=torch.int64).to(device)
     return layers, q_pos, dict(cfg, batch=B, lengths=L)
+
+
+def out_proj_inputs_device(device, seed: int = 0, S: int | None = None, H: int | None = None,
+                           D: int | None = None, G: int | None = None, d_mid: int | None = None,
+                           d_model: int | None = None):
+    """Inputs of the grouped output projection, drawn on `device`: an attention
+    output o [S, H, D] bf16 ~ N(0, 1/4) (the scale of a softmax-weighted mix of
+    unit rows) and random-init weights w_grp [G, d_mid, (H/G)*D], w_out
+    [d_model, G*d_mid], bf16 ~ N(0, 1/fan_in) (no trained weights exist here)."""
+    cfg = dict(WORKLOADS["out_proj"])
+    for k, v in (("S", S), ("H", H), ("D", D), ("G", G), ("d_mid", d_mid), ("d_model", d_model)):
+        if v is not None:
+            cfg[k] = v
+    g = torch.Generator(device=device).manual_seed(seed)
+    S, H, D, G, dm, dmod = cfg["S"], cfg["H"], cfg["D"], cfg["G"], cfg["d_mid"], cfg["d_model"]
+    d_in = (H // G) * D
+    o = (0.5 * torch.randn(S, H, D, generator=g, device=device)).to(torch.bfloat16)
+    w_grp = (torch.randn(G, dm, d_in, generator=g, device=device) / d_in ** 0.5).to(torch.bfloat16)
+    w_out = (torch.randn(dmod, G * dm, generator=g, device=device) / (G * dm) ** 0.5).to(torch.bfloat16)
+    return dict(o=o, w_grp=w_grp, w_out=w_out), cfg

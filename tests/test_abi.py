@@ -112,3 +112,19 @@ def test_python_binding_refuses_cpu_tensors():
     import long_context_compressed_02_b200 as csa
     with pytest.raises(csa.CsaError):
         csa.csa_compress(torch.zeros(8, 8), torch.zeros(8, 8), torch.zeros(8, 8), 4, True)
+
+
+def test_grouped_out_proj_host_validation(L):
+    null = None
+    p = ctypes.c_void_p(16)
+    # group count must divide the head count
+    assert L.csa_grouped_out_proj(p, p, p, 4, 64, 512, 7, 1024, 4096, p, p, 0, null) == 1
+    assert b"divide" in L.csa_last_error()
+    # widths that are not whole 256-column tiles
+    assert L.csa_grouped_out_proj(p, p, p, 4, 64, 512, 8, 1000, 4096, p, p, 0, null) == 2
+    # misaligned pointer
+    assert L.csa_grouped_out_proj(ctypes.c_void_p(8), p, p, 4, 64, 512, 8, 1024, 4096, p, p, 0, null) == 1
+    # bad output dtype
+    assert L.csa_grouped_out_proj(p, p, p, 4, 64, 512, 8, 1024, 4096, p, p, 2, null) == 1
+    # no rows: nothing to do, null pointers accepted, no device call
+    assert L.csa_grouped_out_proj(null, null, null, 0, 64, 512, 8, 1024, 4096, null, null, 1, null) == 0
