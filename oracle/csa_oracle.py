@@ -45,7 +45,9 @@ argument whose default is the reading):
     intermediate_attn_dim 1024, hidden_size 4096]: consecutive heads form a
     group, each group has its own [d_mid, (H/G)*D] matrix, the concatenated
     group outputs go through one [d_model, G*d_mid] matrix, no bias; the
-    intermediate is stored as bf16 like every other activation of the layer.
+    intermediate is stored as bf16 like every other activation of the layer;
+  * FP4 indexer operands [CS "闪电索引器"]: OCP MX FP4 (E2M1 elements, blocks of
+    32 sharing an E8M0 power-of-two scale), two elements per byte.
 """
 from __future__ import annotations
 
@@ -64,6 +66,8 @@ __all__ = [
     "csa_decode", "hca_decode", "flop_counts",
     "fp8_row_quantize", "stream_append",
     "swa_layer", "grouped_out_proj",
+    "e2m1_decode", "e2m1_encode", "e8m0_decode", "fp4_pack", "fp4_unpack",
+    "mxfp4_quantize", "mxfp4_dequantize",
 ]
 
 # ----------------------------------------------------------------------------
@@ -109,6 +113,101 @@ def e4m3_encode(x) -> np.ndarray:
     code = np.where(a == tab[hi], hi, code).astype(np.uint8)
     neg = (x < 0) & (code != 0)
     return np.where(neg, code | 0x80, code).astype(np.uint8)
+
+
+# ----------------------------------------------------------------------------
+# FP4 for the lightning indexer's QK path ([CS] "闪电索引器": the QK path runs in
+# FP4; "其他辅助设计": the indexer is stored in FP4).  The pages name no block
+# format; the reading taken is the OCP Microscaling (MX) FP4 format: E2M1
+# elements (1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit, subnormal
+# at exponent 0, no infinities or NaN, largest magnitude 6) in blocks of 32
+# consecutive elements sharing one E8M0 scale (an unsigned power of two
+# 2^(byte - 127), byte 0xFF = NaN).  Storage: two elements per byte, the even
+# element in the low nibble.
+# ----------------------------------------------------------------------------
+
+def e2m1_decode(codes) -> np.ndarray:
+    """Exact value of each 4-bit E2M1 code (0..15)."""
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = (c & 0x1).astype(np.float64)
+    mag = np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * np.exp2(e.astype(np.float64) - 1.0))
+    return sign * mag
+
+
+_E2M1_POS = None
+
+
+def _e2m1_table():
+    global _E2M1_POS
+    if _E2M1_POS is None:
+        _E2M1_POS = e2m1_decode(np.arange(8))          # 0, 0.5, 1, 1.5, 2, 3, 4, 6
+    return _E2M1_POS
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """Round to the nearest E2M1 value, ties to the even code (mantissa bit 0),
+    saturating at +-6; returns codes 0..15 (no negative zero)."""
+    x = np.asarray(x, dtype=np.float64)
+    tab = _e2m1_table()
+    a = np.minimum(np.abs(x), 6.0)
+    hi = np.clip(np.searchsorted(tab, a, side="left"), 0, 7)
+    lo = np.clip(hi - 1, 0, 7)
+    dlo = a - tab[lo]
+    dhi = tab[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(a == tab[hi], hi, code)
+    neg = (x < 0) & (code != 0)
+    return np.where(neg, code | 0x8, code).astype(np.uint8)
+
+
+def e8m0_decode(b) -> np.ndarray:
+    """Value of each E8M0 scale byte: 2^(b - 127); 0xFF is NaN."""
+    b = np.asarray(b).astype(np.int64)
+    return np.where(b == 0xFF, np.nan, np.exp2((b - 127).astype(np.float64)))
+
+
+def fp4_pack(codes) -> np.ndarray:
+    """[..., 2n] codes 0..15 -> [..., n] bytes, element 2j in the low nibble."""
+    c = np.asarray(codes).astype(np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def fp4_unpack(packed) -> np.ndarray:
+    """Inverse of fp4_pack: [..., n] bytes -> [..., 2n] codes."""
+    p = np.asarray(packed).astype(np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def mxfp4_quantize(x, block: int = 32):
+    """MX FP4 quantisation of the last axis: for each block of `block`
+    elements the shared scale is 2^(floor(log2(amax)) - 2) (2 = the largest
+    E2M1 exponent), clamped to the E8M0 range, and each element is
+    e2m1_encode(v / scale) (saturating).  An all-zero block gets scale 2^-127.
+    Returns (codes [..., n] 0..15, scale bytes [..., n / block])."""
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[-1]
+    if n % block:
+        raise ValueError("the last axis must be a multiple of the block size")
+    xb = x.reshape(x.shape[:-1] + (n // block, block))
+    amax = np.abs(xb).max(axis=-1)
+    with np.errstate(divide="ignore"):
+        e = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2.0, -127.0)
+    e = np.clip(e, -127.0, 127.0)
+    codes = e2m1_encode(xb / np.exp2(e)[..., None]).reshape(x.shape)
+    return codes, (e + 127.0).astype(np.uint8)
+
+
+def mxfp4_dequantize(codes, scales, block: int = 32) -> np.ndarray:
+    """Values of MX FP4 data: e2m1_decode(code) * e8m0_decode(block scale)."""
+    v = e2m1_decode(codes)
+    s = np.repeat(e8m0_decode(scales), block, axis=-1)
+    return v * s
 
 
 def bf16_round(x) -> np.ndarray:
