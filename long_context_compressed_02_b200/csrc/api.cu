@@ -41,7 +41,8 @@ extern "C" csa_status_t csa_check_device_error(cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess)
     return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: stream sync failed: %s", cudaGetErrorString(e));
-  uint32_t w = csa::read_clear_err_indexer() | csa::read_clear_err_attention() | csa::read_clear_err_proj();
+  uint32_t w = csa::read_clear_err_indexer() | csa::read_clear_err_attention() | csa::read_clear_err_proj() |
+               csa::read_clear_err_compress();
   if (w & 1u) return csa::fail(CSA_ERR_TIMEOUT, "a bounded on-chip wait expired (device error word 0x%x)", w);
   if (w) return csa::fail(CSA_ERR_DEVICE, "a kernel recorded an out-of-range gather index (device error word 0x%x)", w);
   return CSA_OK;

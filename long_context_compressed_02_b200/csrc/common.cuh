@@ -32,6 +32,7 @@ inline int num_sms() {
 uint32_t read_clear_err_indexer();
 uint32_t read_clear_err_attention();
 uint32_t read_clear_err_proj();
+uint32_t read_clear_err_compress();
 
 }  // namespace csa
 

@@ -13,14 +13,26 @@
 // moves them with 16-byte (bf16) or 2 x 16-byte (fp32) vector loads, so a group
 // of D/8 threads reads one row with fully coalesced transactions.  No tensor
 // cores: there is no contraction here.
+#include <algorithm>
 #include <cmath>
 #include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <math_constants.h>
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace csa {
+
+static __device__ uint32_t g_err_compress;
+
+uint32_t read_clear_err_compress() {
+  uint32_t v = 0, z = 0;
+  cudaMemcpyFromSymbol(&v, g_err_compress, sizeof(v));
+  cudaMemcpyToSymbol(g_err_compress, &z, sizeof(z));
+  return v;
+}
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -184,10 +196,6 @@ compress_kernel(const Tin* __restrict__ C, const Tin* __restrict__ Z, const Tin*
   }
   if (owner) Vec8<Tout>::store(out + i * D + ch0, x);
 }
-
-// cos/sin for RoPE pair j at position pos: the angle pos * base^(-2j/r) is formed
-// and reduced modulo 2*pi in double (positions reach 2^20 and beyond), then the
-// reduced angle is evaluated in single precision.
 
 // cos / sin of pos * theta_j with theta_j = ratio^j (ratio = base^(-2/rope_dim),
 // computed on the host in double): the power by squaring and the angle
@@ -376,6 +384,118 @@ rmsnorm_rope_bf16_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int 
   }
 }
 
+// bf16 rows of D = 512 whose position changes every rows_per_pos rows, a
+// multiple of 32 (the per-head query rows of the prefill workloads).  CTAs (two
+// per SM) stream chunks of 32 rows (32 KB) through a 3-stage shared-memory ring:
+// warp 8 issues one bulk asynchronous copy per chunk (completion counted on the
+// stage's mbarrier), so each SM keeps up to 192 KB of reads in flight with few
+// registers.  Warps 0-7 normalise and rotate four rows each: lane l holds
+// channels 8l .. 8l+7 and 256+8l .. 256+8l+7, so every shared-memory read and
+// every global store of a warp covers 512 contiguous bytes; the RoPE dims
+// [448, 512) sit in the second group of lanes 24-31, whose partner lane is l ^ 4.
+constexpr int kBulkRows = 32;
+constexpr int kBulkStages = 3;
+constexpr int kBulkThreads = 288;
+constexpr uint32_t kBulkChunkBytes = kBulkRows * 512 * 2;
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+template <typename Tout>
+__global__ void __launch_bounds__(kBulkThreads, 2)
+rmsnorm_rope_bulk_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows, int rows_per_pos, int64_t pos0,
+                         int norm, int rope_dim, double ratio, float eps, Tout* __restrict__ out) {
+  constexpr int D = 512;
+  extern __shared__ __align__(16) uint8_t smem_ring[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_ring + kBulkStages * kBulkChunkBytes);
+  uint64_t* empty = full + kBulkStages;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t n_chunks = (rows + kBulkRows - 1) / kBulkRows;
+  if (tid == 0) {
+    for (int s = 0; s < kBulkStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 8); }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {
+    // ---------------- producer (lane 0)
+    if (lane == 0) {
+      uint32_t k = 0;
+      for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++k) {
+        const uint32_t s = k % kBulkStages, ph = (k / kBulkStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, &g_err_compress)) break;
+        const int64_t row0 = c * kBulkRows;
+        const uint32_t bytes = (uint32_t)min((int64_t)kBulkRows, rows - row0) * (D * 2);
+        mbar_expect_tx(&full[s], bytes);
+        bulk_load(smem_ring + s * kBulkChunkBytes, x + row0 * D, bytes, &full[s]);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers: warp w takes rows 4w .. 4w+3 of every chunk
+  const bool rope_lane = rope_dim > 0 && lane >= 24;
+  const bool first_half = lane < 28;
+  const int j0 = ((lane - 24) & 3) * 8;
+  float2 cs[8];
+  int64_t cs_pos = -1;
+  uint32_t k = 0;
+  for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x, ++k) {
+    const uint32_t s = k % kBulkStages, ph = (k / kBulkStages) & 1;
+    if (!mbar_wait(&full[s], ph, &g_err_compress)) break;
+    const int64_t row0 = c * kBulkRows;
+    const int rows_in = (int)min((int64_t)kBulkRows, rows - row0);
+    const int64_t pos = pos0 + row0 / rows_per_pos;      // one position per chunk
+    if (rope_dim > 0 && pos != cs_pos) {                // lane j computes pair j, RoPE lanes gather theirs
+      const float2 mine = rope_cs_pow(pos, lane, ratio);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cs[i].x = __shfl_sync(0xffffffffu, mine.x, j0 + i);
+        cs[i].y = __shfl_sync(0xffffffffu, mine.y, j0 + i);
+      }
+      cs_pos = pos;
+    }
+    const uint8_t* chunk = smem_ring + s * kBulkChunkBytes;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rl = warp * 4 + i;
+      if (rl >= rows_in) break;
+      const uint8_t* row = chunk + rl * (D * 2);
+      float v[16];
+      bf16x8_to_float(*reinterpret_cast<const uint4*>(row + lane * 16), v);
+      bf16x8_to_float(*reinterpret_cast<const uint4*>(row + 512 + lane * 16), v + 8);
+      float inv = 1.f;
+      if (norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) ss = fmaf(v[c2], v[c2], ss);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        inv = rsqrtf(ss / (float)D + eps);
+      }
+      float o[16];
+#pragma unroll
+      for (int c2 = 0; c2 < 16; ++c2) o[c2] = v[c2] * inv;
+      if (rope_lane) {
+        float u[8];
+        bf16x8_to_float(*reinterpret_cast<const uint4*>(row + 512 + (lane ^ 4) * 16), u);
+#pragma unroll
+        for (int i2 = 0; i2 < 8; ++i2) {
+          const float a = o[8 + i2], b = u[i2] * inv;
+          o[8 + i2] = first_half ? a * cs[i2].x - b * cs[i2].y : b * cs[i2].y + a * cs[i2].x;
+        }
+      }
+      Tout* dst = out + (row0 + rl) * D;
+      Vec8<Tout>::store(dst + lane * 8, o);
+      Vec8<Tout>::store(dst + 256 + lane * 8, o + 8);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
 template <typename T> __device__ __forceinline__ float to_f(T v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -521,6 +641,15 @@ csa_status_t launch_norm(const void* x, int64_t rows, int D, int rpp, int64_t po
   if (grid > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "csa_rmsnorm_rope: too many rows");
   const double ratio = rope_dim > 0 ? std::pow((double)rope_base, -2.0 / (double)rope_dim) : 1.0;
   if constexpr (std::is_same<Tin, __nv_bfloat16>::value && CPL == 16) {
+    if (rpp % kBulkRows == 0) {
+      const int64_t n_chunks = (rows + kBulkRows - 1) / kBulkRows;
+      const size_t smem = (size_t)kBulkStages * kBulkChunkBytes + 2 * kBulkStages * sizeof(uint64_t);
+      cudaFuncSetAttribute(rmsnorm_rope_bulk_kernel<Tout>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      const int bgrid = (int)std::min<int64_t>(n_chunks, 2 * (int64_t)num_sms());
+      rmsnorm_rope_bulk_kernel<Tout><<<bgrid, kBulkThreads, smem, st>>>(
+          (const __nv_bfloat16*)x, rows, rpp, pos0, norm, rope_dim, ratio, eps, (Tout*)out);
+      return check_launch("csa_rmsnorm_rope");
+    }
     rmsnorm_rope_bf16_kernel<Tout><<<(unsigned)grid, kThreads, 0, st>>>(
         (const __nv_bfloat16*)x, rows, rpp, pos0, ppb, norm, rope_dim, ratio, eps, (Tout*)out);
   } else {

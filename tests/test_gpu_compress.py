@@ -88,3 +88,19 @@ def test_rmsnorm_rope_rows_bf16_out():
     torch.cuda.synchronize()
     ref = O.rope_partial(O.rmsnorm(x), np.arange(1001))
     assert_close(host(out), ref, what="row norm+rope")
+
+
+@pytest.mark.parametrize("norm,out_dtype", [(True, torch.bfloat16), (False, torch.float32), (True, torch.float32)])
+def test_rmsnorm_rope_bulk_path_ragged(norm, out_dtype):
+    """bf16 rows sharing a position in groups of 32 (the chunked bulk-copy
+    path), with a partial last chunk and a position near 2^20."""
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(13)
+    rows, rpp, pos0 = 1000, 32, (1 << 20) - 17
+    x = synth.to_bf16_values(rng.standard_normal((rows, 512)))
+    out = csa.csa_rmsnorm_rope(cuda(x, torch.bfloat16), rows_per_pos=rpp, pos0=pos0, norm=norm, out_dtype=out_dtype)
+    csa.check_device_error()
+    y = O.rmsnorm(x) if norm else x.astype(np.float64)
+    ref = O.rope_partial(y, pos0 + np.arange(rows) // rpp)
+    tol = {} if out_dtype == torch.bfloat16 else dict(max_abs=1e-4, rel_l2=1e-5)
+    assert_close(host(out), ref, what="bulk norm+rope", **tol)
