@@ -128,3 +128,23 @@ def test_grouped_out_proj_host_validation(L):
     assert L.csa_grouped_out_proj(p, p, p, 4, 64, 512, 8, 1024, 4096, p, p, 2, null) == 1
     # no rows: nothing to do, null pointers accepted, no device call
     assert L.csa_grouped_out_proj(null, null, null, 0, 64, 512, 8, 1024, 4096, null, null, 1, null) == 0
+
+
+def test_plain_c_client(L, tmp_path):
+    """The header is C (not only C++): a C99 program includes it, links
+    libcsa.so and runs the host-side checks (no GPU needed)."""
+    import shutil
+    import subprocess
+    from long_context_compressed_02_b200 import LIB_PATH
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    cuda_inc = "/usr/local/cuda/include"
+    src = os.path.join(ROOT, "tests", "abi_c", "check_abi.c")
+    exe = str(tmp_path / "check_abi")
+    lib_dir = os.path.dirname(LIB_PATH)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+                        src, "-o", exe, LIB_PATH, f"-Wl,-rpath,{lib_dir}"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0 and "check_abi: ok" in r.stdout, r.stdout + r.stderr
