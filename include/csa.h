@@ -63,6 +63,8 @@ int csa_abi_version(void);
  * calling thread (empty string if none).  Both pointers stay valid. */
 const char* csa_status_string(csa_status_t s);
 const char* csa_last_error(void);
+/* Same text as csa_last_error(). */
+const char* csa_get_last_error_string(void);
 
 /* Synchronises `stream`, then reads and clears the device error words of the
  * current device.  Returns CSA_ERR_TIMEOUT or CSA_ERR_DEVICE if a kernel
@@ -282,6 +284,12 @@ csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, const void*
  *   stream.
  * ------------------------------------------------------------------------- */
 size_t csa_fused_attention_workspace(int n_seq, int T, int H, int D, int n_split);
+
+/* Workspace for one layer step whose indexer call (csa_index_topk with
+ * n_seq, T, cap, k) and attention call (csa_fused_attention_splitkv with
+ * n_seq, T, H, D, n_split; n_split <= 1 needs none) share one buffer in
+ * stream order: the larger of the two sizes.  Pure host arithmetic. */
+size_t csa_workspace_size(int n_seq, int T, int64_t cap, int k, int H, int D, int n_split);
 csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q_dtype, const void* kv, csa_dtype_t kv_dtype,
                                          const void* kv_rope, const float* kv_scale, int64_t cap,
                                          const int32_t* idx, int k, int m, const void* kv_tok,

@@ -62,6 +62,8 @@ def lib():
                                          I, P, SZ, P, I, P], I),
         "csa_compress_append": ([P, P, I, P, I, I, I, I, P, P, P, P, P, P, I64, I, I, F, F, P], I),
         "csa_grouped_out_proj": ([P, P, P, I, I, I, I, I, I, P, P, I, P], I),
+        "csa_get_last_error_string": ([], ctypes.c_char_p),
+        "csa_workspace_size": ([I, I, I64, I, I, I, I], SZ),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)

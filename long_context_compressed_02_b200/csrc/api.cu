@@ -37,6 +37,14 @@ extern "C" const char* csa_status_string(csa_status_t s) {
 
 extern "C" const char* csa_last_error(void) { return csa::g_last_error.c_str(); }
 
+extern "C" const char* csa_get_last_error_string(void) { return csa_last_error(); }
+
+extern "C" size_t csa_workspace_size(int n_seq, int T, int64_t cap, int k, int H, int D, int n_split) {
+  const size_t a = csa_index_topk_workspace(n_seq, T, cap, k);
+  const size_t b = n_split > 1 ? csa_fused_attention_workspace(n_seq, T, H, D, n_split) : 0;
+  return a > b ? a : b;
+}
+
 extern "C" csa_status_t csa_check_device_error(cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess)

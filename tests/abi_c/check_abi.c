@@ -15,11 +15,13 @@ int main(void) {
 
   /* workspace of the prefill indexer call: the score matrix plus the item counter */
   CHECK(csa_index_topk_workspace(1, 16384, 4096, 512) == (size_t)16384 * 4096 * 4 + 256);
+  CHECK(csa_workspace_size(1, 16384, 4096, 512, 64, 512, 1) == csa_index_topk_workspace(1, 16384, 4096, 512));
 
   /* argument errors are reported before any device work */
   void* p = (void*)(uintptr_t)16;
   CHECK(csa_grouped_out_proj(p, p, p, 4, 64, 512, 7, 1024, 4096, p, p, CSA_BF16, 0) == CSA_ERR_INVALID_ARG);
   CHECK(strstr(csa_last_error(), "divide") != NULL);
+  CHECK(strcmp(csa_get_last_error_string(), csa_last_error()) == 0);
   CHECK(csa_grouped_out_proj(p, p, p, 4, 64, 512, 8, 1000, 4096, p, p, CSA_BF16, 0) == CSA_ERR_UNSUPPORTED);
   CHECK(csa_grouped_out_proj(NULL, NULL, NULL, 0, 64, 512, 8, 1024, 4096, NULL, NULL, CSA_F32, 0) == CSA_OK);
   CHECK(csa_rmsnorm_rope(p, CSA_BF16, 10, 100, 1, 0, 1, 64, 10000.f, 1e-6f, p, CSA_BF16, 0) == CSA_ERR_INVALID_ARG);

@@ -148,3 +148,12 @@ def test_plain_c_client(L, tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([exe], capture_output=True, text=True)
     assert r.returncode == 0 and "check_abi: ok" in r.stdout, r.stdout + r.stderr
+
+
+def test_layer_workspace_is_the_larger_of_the_two(L):
+    a = L.csa_index_topk_workspace(16, 1, 262144, 512)
+    b = L.csa_fused_attention_workspace(16, 1, 64, 512, 5)
+    assert L.csa_workspace_size(16, 1, 262144, 512, 64, 512, 5) == max(a, b)
+    assert L.csa_workspace_size(1, 16384, 4096, 512, 64, 512, 1) == L.csa_index_topk_workspace(1, 16384, 4096, 512)
+    L.csa_compress(None, None, None, None, None, 64, 7, 4, 1, 0, 0, 0, 10000.0, 1e-6, None, 0, None)
+    assert L.csa_get_last_error_string() == L.csa_last_error() != b""
