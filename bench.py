@@ -406,6 +406,41 @@ def out_proj_leg(dev, steps, warmup, csa, synth, torch, seed=0, S=None):
                          "peak_source": f"{src} bf16 burst (the leg runs alone, a few ms)"}}
 
 
+def tiny_leg(dev, steps, warmup, csa, synth, torch):
+    """The tiny fp32 CSA layer (S 2048, 8 heads x 128, indexer 4 x 32, top-k 64):
+    launch-latency bound; reported in microseconds per layer step (4 kernels)."""
+    inp, cfg = synth.prefill_inputs("tiny_csa")
+    S, H, D, m, k, W, HI, DI = (cfg[x] for x in ("S", "H", "D", "m", "k", "W", "HI", "DI"))
+
+    def dv(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+
+    q, C, Z, B, qI, w, kI, sink = (dv(inp[x]) for x in ("q", "C", "Z", "B", "qI_codes", "w", "kI_codes", "sink"))
+    ws = torch.empty(csa.csa_index_topk_workspace(1, S, S // m, k), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        csa.csa_layer_prefill(q, C, Z, B, qI, w, kI, sink, k=k, m=m, W=W, workspace=ws)
+
+    for _ in range(max(3, warmup)):
+        step()
+    csa.check_device_error()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    sparse, window, indexer = _flops(S, H, D, m, k, W, HI, DI)
+    return {"workload": "tiny_csa", "S": S, "H": H, "D": D, "dtype": "f32 storage, bf16 attention operands",
+            "us_per_step": ms * 1e3, "kernels_per_step": 4,
+            "flops_per_step": {"attention": sparse + window, "indexer_fp8": indexer},
+            "bound": "launch latency"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -421,6 +456,7 @@ def main():
     ap.add_argument("--no-hca", action="store_true", help="skip the HCA prefill leg (S 131072)")
     ap.add_argument("--no-mixed", action="store_true", help="skip the 4-layer mixed decode leg")
     ap.add_argument("--no-out-proj", action="store_true", help="skip the grouped output projection leg")
+    ap.add_argument("--no-tiny", action="store_true", help="skip the tiny fp32 layer leg")
     ap.add_argument("--out-proj-only", action="store_true", help="run only the output projection leg (profiling)")
     args = ap.parse_args()
     from long_context_compressed_02_b200 import replicas
@@ -612,7 +648,7 @@ def main():
                "sample": f"{n_rows} evenly spaced query rows of the same S=16384 layer (float64 numpy oracle, "
                          f"{dt:.1f} s including its full-sequence compressor and window-row passes)"}
 
-    hca = mixed = proj = None
+    hca = mixed = proj = tiny = None
     if args.S is None:
         del inp, qn, kt, kv, idx, ws, out
         torch.cuda.empty_cache()
@@ -625,6 +661,8 @@ def main():
         if not args.no_out_proj:
             proj = out_proj_leg(dev, args.steps, args.warmup, csa, synth, torch, seed=replicas.replica_seed(rank))
             torch.cuda.empty_cache()
+        if not args.no_tiny:
+            tiny = tiny_leg(dev, args.steps, args.warmup, csa, synth, torch)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -638,7 +676,7 @@ def main():
                                               "indexer_fp8": fl_index}},
                 "prefill_tokens_per_s": replicas.job_rate(S, world, ms * 1e-3),
                 "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode,
-                "hca_prefill": hca, "decode_mixed": mixed, "out_proj": proj,
+                "hca_prefill": hca, "decode_mixed": mixed, "out_proj": proj, "tiny_csa": tiny,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:
