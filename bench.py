@@ -244,6 +244,63 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1, n_spli
                          "peak_source": f"{src} copy bandwidth"}}
 
 
+def decode_fp4_leg(dev, steps, warmup, csa, synth, torch, seed=1, n_split=None):
+    """The 2^20-context decode step of decode_leg with the indexer's QK path in
+    MX FP4: packed E2M1 keys (64 B) + E8M0 block scales (4 B) per entry, 68 B
+    scanned per entry instead of 132 B."""
+    inp, cfg = synth.decode_inputs_device("csa_decode_1m", dev, seed=seed)
+    Bn, ne, k, W, H, D, HI, DI = (cfg[x] for x in ("batch", "n_e", "k", "W", "H", "D", "HI", "DI"))
+    g = torch.Generator(device=dev).manual_seed(seed + 100)
+    kI4 = torch.randint(0, 256, (Bn, ne, 64), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
+    kI4s = torch.randint(125, 130, (Bn, ne, 4), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
+    qI4 = torch.randint(0, 256, (Bn, 1, HI, 64), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
+    qI4s = torch.randint(125, 130, (Bn, 1, HI, 4), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
+    ws = torch.empty(csa.csa_index_topk_fp4_workspace(Bn, 1, HI, ne, k), dtype=torch.uint8, device=dev)
+    idx = torch.empty(Bn, 1, k, dtype=torch.int32, device=dev)
+    out = torch.empty(Bn, 1, H, D, dtype=torch.bfloat16, device=dev)
+    if n_split is None:
+        n_split = max(1, min(5, csa.num_sms() // Bn))
+    aws = torch.empty(csa.csa_fused_attention_workspace(Bn, 1, H, D, n_split), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        csa.csa_index_topk_fp4(qI4, qI4s, inp["w"], kI4, kI4s, inp["q_pos"], 4, k, workspace=ws, idx=idx)
+        if ev is not None:
+            ev[1].record(stream)
+        csa.csa_fused_attention(inp["q"], inp["kv_nope"], inp["swa"], inp["q_pos"], W, inp["sink"], idx=idx,
+                                kv_rope=inp["kv_rope"], kv_scale=inp["kv_scale"], window_mode=1, inv_rope=True,
+                                rope_dim=64, out=out, n_split=n_split, workspace=aws)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(3, warmup)):
+        step()
+    csa.check_device_error()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    csa.check_device_error()
+    t_idx = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    t_att = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms = float(np.mean([e[0].elapsed_time(e[2]) for e in evs]))
+    scan = Bn * ne * (64 + 4)
+    gather = Bn * k * (D - 64 + 128 + 4)
+    algo = scan + gather + Bn * W * D * 2 + Bn * (H * D * 2 + HI * 68 + HI * 4)
+    hbm, _, _, src = _peaks()
+    ach_idx = scan / (t_idx * 1e-3) / 1e9
+    return {"workload": "csa_decode_1m_fp4_indexer", "batch": Bn, "entries": ne, "top_k": k,
+            "tokens_per_s": Bn / (ms * 1e-3), "ms_per_step": ms,
+            "kernels_ms": {"index_topk_fp4": t_idx, "fused_attention": t_att},
+            "algorithmic_bytes_per_step": algo, "hbm_frac_step": algo / (ms * 1e-3) / 1e9 / hbm,
+            "roofline": {"kernel": "index_topk_fp4", "bound": "hbm", "achieved": ach_idx, "peak": hbm,
+                         "unit": "GB/s", "frac": ach_idx / hbm, "traffic": None,
+                         "peak_source": f"{src} copy bandwidth"}}
+
+
 def mixed_decode_leg(dev, steps, warmup, csa, synth, torch, seed=0, split=None):
     """The 4-layer decode stack (CSA, HCA, CSA, HCA), batch 32, per-sequence
     contexts U[64K, 1M]: one new token per sequence through all four layers."""
@@ -630,9 +687,12 @@ def main():
         roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s", "frac": None,
                 "traffic": None}
 
-    decode = None
+    decode = decode_fp4 = None
     if not args.no_decode and args.S is None:
         decode = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch,
+                                        seed=replicas.replica_seed(rank, base=1))
+        if args.decode_batch is None:
+            decode_fp4 = decode_fp4_leg(dev, args.steps, args.warmup, csa, synth, torch,
                                         seed=replicas.replica_seed(rank, base=1))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -675,7 +735,7 @@ def main():
                            "flops_per_step": {"sparse_mqa": fl_sparse, "swa_window": fl_window,
                                               "indexer_fp8": fl_index}},
                 "prefill_tokens_per_s": replicas.job_rate(S, world, ms * 1e-3),
-                "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode,
+                "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode, "decode_1m_fp4": decode_fp4,
                 "hca_prefill": hca, "decode_mixed": mixed, "out_proj": proj, "tiny_csa": tiny,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)

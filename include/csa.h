@@ -194,6 +194,24 @@ csa_status_t csa_index_topk_noalloc(const uint8_t* qI, const float* qI_scale, co
                                     int32_t* idx, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * csa_index_topk_fp4 — csa_index_topk with the QK path in FP4 ([CS] "闪电索引器":
+ * the indexer's QK path runs in FP4; "其他辅助设计": the indexer is stored in
+ * FP4).  Format (OCP MX FP4): E2M1 codes, two per byte with the even element in
+ * the low nibble, and one E8M0 scale byte (2^(byte - 127)) per 32-element block.
+ *   qI4 [n_seq, T, HI, 64] u8, qI4_scale [n_seq, T, HI, 4] u8,
+ *   kI4 [n_seq, cap, 64] u8,   kI4_scale [n_seq, cap, 4] u8  (DI = 128).
+ * Scores are those of csa_index_topk on the dequantised operands; on the GPU
+ * the blocks are rescaled to each row's largest block scale in e4m3, exact while
+ * a row's block scales span at most 2^8.  cap must be a multiple of 4.
+ * Workspace: csa_index_topk_fp4_workspace(n_seq, T, HI, cap, k) bytes.
+ * ------------------------------------------------------------------------- */
+size_t csa_index_topk_fp4_workspace(int n_seq, int T, int HI, int64_t cap, int k);
+csa_status_t csa_index_topk_fp4(const uint8_t* qI4, const uint8_t* qI4_scale, const float* w,
+                                const uint8_t* kI4, const uint8_t* kI4_scale, const int64_t* q_pos, int n_seq,
+                                int T, int HI, int64_t cap, int m, int k, int32_t* idx, void* workspace,
+                                size_t ws_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Attention over one shared K = V row set per query token ([CS] "共享 KV MQA":
  * the selected compressed entries act as both key and value; one KV head
  * shared by H query heads).  Logits are scale * q_h . row; softmax over the

@@ -64,6 +64,8 @@ def lib():
         "csa_grouped_out_proj": ([P, P, P, I, I, I, I, I, I, P, P, I, P], I),
         "csa_get_last_error_string": ([], ctypes.c_char_p),
         "csa_workspace_size": ([I, I, I64, I, I, I, I], SZ),
+        "csa_index_topk_fp4_workspace": ([I, I, I, I64, I], SZ),
+        "csa_index_topk_fp4": ([P, P, P, P, P, P, I, I, I, I64, I, I, P, P, SZ, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -187,6 +189,30 @@ def csa_index_topk(qI, w, kI, q_pos, m, k, *, qI_scale=None, kI_scale=None, work
     _check(lib().csa_index_topk(_ptr(qI), _ptr(qI_scale), _ptr(w), _ptr(kI), _ptr(kI_scale), _ptr(q_pos),
                                 n_seq, T, HI, DI, cap, m, k, _ptr(idx), _ptr(workspace), workspace.numel(),
                                 _stream(stream)), "csa_index_topk")
+    return idx
+
+
+def csa_index_topk_fp4(qI4, qI4_scale, w, kI4, kI4_scale, q_pos, m, k, *, workspace=None, idx=None, stream=None):
+    """Lightning indexer + top-k on MX FP4 operands: qI4 [n_seq, T, HI, 64] and
+    kI4 [n_seq, cap, 64] uint8 (packed E2M1, the even element in the low
+    nibble), qI4_scale [n_seq, T, HI, 4] and kI4_scale [n_seq, cap, 4] uint8
+    (E8M0 per 32-element block), w [n_seq, T, HI] f32, q_pos [n_seq] int64.
+    Returns idx [n_seq, T, k] int32 (ascending, -1 padded)."""
+    for t, n in ((qI4, "qI4"), (qI4_scale, "qI4_scale"), (w, "w"), (kI4, "kI4"), (kI4_scale, "kI4_scale"),
+                 (q_pos, "q_pos")):
+        _dev(t, n)
+    n_seq, T, HI, _ = qI4.shape
+    cap = kI4.shape[1]
+    if qI4.shape[-1] != 64 or kI4.shape[-1] != 64 or qI4_scale.shape[-1] != 4 or kI4_scale.shape[-1] != 4:
+        raise CsaError("csa_index_topk_fp4: 64 code bytes and 4 scale bytes per 128-element row expected")
+    need = int(lib().csa_index_topk_fp4_workspace(n_seq, T, HI, cap, k))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=qI4.device)
+    if idx is None:
+        idx = torch.empty((n_seq, T, k), dtype=torch.int32, device=qI4.device)
+    _check(lib().csa_index_topk_fp4(_ptr(qI4), _ptr(qI4_scale), _ptr(w), _ptr(kI4), _ptr(kI4_scale), _ptr(q_pos),
+                                    n_seq, T, HI, cap, m, k, _ptr(idx), _ptr(workspace), workspace.numel(),
+                                    _stream(stream)), "csa_index_topk_fp4")
     return idx
 
 

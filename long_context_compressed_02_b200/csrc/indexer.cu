@@ -29,6 +29,7 @@
 // one CTA per row merges the survivors.
 #include <algorithm>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 #include "common.cuh"
@@ -59,7 +60,13 @@ bool make_byte_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t r
 
 // ------------------------------------------------------------------ scores
 constexpr int kIdxThreads = 320;      // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kIdxThreadsFp4 = 448;   // + warps 10..13 convert FP4 key tiles to e4m3
 constexpr int kEpiThreads = 256;
+constexpr int kConvThreads = 128;     // one key row of a 128-key tile per thread
+constexpr int kOpStages = 4;          // converted (e4m3) key tiles in flight (FP4 keys)
+constexpr int kRsSlots = kOpStages + 2;   // key row scales handed from the converter to the epilogue
+constexpr uint32_t kFp4Codes = 128 * 64;  // packed E2M1 codes of a 128-key tile (DI 128)
+constexpr uint32_t kFp4Stage = kFp4Codes + 128 * 4;   // + one E8M0 byte per 32-element block
 constexpr int kStages = 8;           // key-tile ring depth (deeper rings measured slower)
 
 struct IdxParams {
@@ -117,15 +124,100 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return false;
 }
 
+// ------------------------------------------------------------------ FP4 keys
+// MX FP4 operands (E2M1 codes, one E8M0 scale per 32-element block) are turned
+// into e4m3 pre-scaled by 2^(e_block - e_rowmax), so that the row factor
+// 2^(e_rowmax - 127) becomes an ordinary per-row scale and the e4m3 tensor-core
+// path is reused.  For e_block - e_rowmax = d >= -5 every E2M1 magnitude code c
+// maps to one e4m3 byte by (c << 2) + ((6 + d) << 3) (code 1, the value 0.5,
+// to (6 + d) << 3, code 0 to 0): a byte permutation from an 8-entry table; the
+// sign bit moves from bit 3 of the nibble to bit 7 of the byte.  Below d = -5
+// each element is converted through fp32 (exact down to d = -8, the smallest
+// e4m3 subnormal; rounded to nearest even below that).
+__device__ __forceinline__ uint32_t e2m1x4_to_e4m3(uint32_t x, uint32_t lo, uint32_t hi) {
+  const uint32_t mags = __byte_perm(lo, hi, x & 0x7777u);
+  const uint32_t sgn = __byte_perm(0x00008000u, 0u, (x >> 3) & 0x1111u);
+  return mags | sgn;
+}
+
+__device__ __forceinline__ uint32_t e2m1x4_to_e4m3_slow(uint32_t x, int d) {
+  const float scale = ldexpf(1.f, d);
+  uint32_t out = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t c = (x >> (4 * i)) & 0xFu;
+    const uint32_t m = c & 7u;
+    const float mag = m < 2 ? 0.5f * (float)m : (float)(2 + (m & 1)) * ldexpf(1.f, (int)(m >> 1) - 2);
+    const float v = (c & 8u ? -mag : mag) * scale;
+    out |= (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3) << (8 * i);
+  }
+  return out;
+}
+
+// One 128-element row: codes c[b] (16 bytes = 32 elements of block b, even
+// element in the low nibble), scale bytes sc (block b in byte b).  Writes the
+// 128 e4m3 bytes as out[0..7] (16 bytes each, in element order) and returns
+// the row factor 2^(e_rowmax - 127).
+__device__ __forceinline__ float fp4_row_to_e4m3(const uint4 c[4], uint32_t sc, uint4 out[8]) {
+  const int e0 = sc & 0xFF, e1 = (sc >> 8) & 0xFF, e2 = (sc >> 16) & 0xFF, e3 = sc >> 24;
+  const int emax = max(max(e0, e1), max(e2, e3));
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int d = (b == 0 ? e0 : b == 1 ? e1 : b == 2 ? e2 : e3) - emax;
+    const uint32_t w[4] = {c[b].x, c[b].y, c[b].z, c[b].w};
+    uint32_t o[8];
+    if (d >= -5) {
+      const uint32_t K = (uint32_t)((6 + d) << 3);
+      const uint32_t lo = K * 0x01010100u + 0x0C080000u;   // bytes 0, K, 8+K, 12+K
+      const uint32_t hi = K * 0x01010101u + 0x1C181410u;   // bytes 16+K .. 28+K
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[2 * i] = e2m1x4_to_e4m3(w[i] & 0xFFFFu, lo, hi);
+        o[2 * i + 1] = e2m1x4_to_e4m3(w[i] >> 16, lo, hi);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        o[2 * i] = e2m1x4_to_e4m3_slow(w[i] & 0xFFFFu, d);
+        o[2 * i + 1] = e2m1x4_to_e4m3_slow(w[i] >> 16, d);
+      }
+    }
+    out[2 * b] = make_uint4(o[0], o[1], o[2], o[3]);
+    out[2 * b + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  return emax == 255 ? CUDART_NAN_F : ldexpf(1.f, emax - 127);
+}
+
+// Query side: each row (token, head) of FP4 codes [rows, 64 B] + scales
+// [rows, 4 B] becomes an e4m3 row [rows, 128 B] and a per-row scale.
+__global__ void fp4_rows_to_e4m3_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                        int64_t rows, uint8_t* __restrict__ out, float* __restrict__ out_scale) {
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  uint4 c[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) c[b] = __ldg(reinterpret_cast<const uint4*>(codes + r * 64) + b);
+  const uint32_t sc = __ldg(reinterpret_cast<const uint32_t*>(scales + r * 4));
+  uint4 o[8];
+  out_scale[r] = fp4_row_to_e4m3(c, sc, o);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) reinterpret_cast<uint4*>(out + r * 128)[q] = o[q];
+}
+
 __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
   return v;
 }
 
-__global__ void __launch_bounds__(kIdxThreads, 1)
+// FP4: tmap_k covers the packed key codes [rows, 64 B] and tmap_ks their scale
+// bytes viewed as [rows / 4, 16 B]; warps 10-13 convert each staged tile into
+// the e4m3 operand ring, and the key row scales reach the epilogue through
+// shared memory.  FP8: tmap_ks is unused.
+template <bool FP4>
+__global__ void __launch_bounds__(FP4 ? kIdxThreadsFp4 : kIdxThreads, 1)
 indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
-                      IdxParams p) {
+                      const __grid_constant__ CUtensorMap tmap_ks, IdxParams p) {
   extern __shared__ uint8_t smem_raw[];
   // aligned by offsetting the shared array itself, so accesses stay in the shared window
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -135,8 +227,9 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   const uint32_t b_bytes = (uint32_t)p.N * p.DI;
   const uint32_t b_stride = (b_bytes + 1023u) & ~1023u;
   uint8_t* sB = smem;                                         // [2] query tiles (item parity)
-  uint8_t* sA = smem + 2 * b_stride;                          // [kStages] key tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sA + kStages * a_bytes);
+  uint8_t* sA = smem + 2 * b_stride;                          // [kStages] key tiles (FP4: [kOpStages] e4m3 tiles)
+  uint8_t* sP = sA + (FP4 ? kOpStages : kStages) * a_bytes;   // FP4: [kStages] staged packed tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(FP4 ? sP + kStages * kFp4Stage : sP);
   uint64_t* full = bars;                 // [kStages]
   uint64_t* empty = bars + kStages;      // [kStages]
   uint64_t* tfull = bars + 2 * kStages;  // [2]
@@ -145,22 +238,33 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   uint64_t* qempty = qfull + 2;          // [2]
   uint64_t* ifull = qempty + 2;          // [4] claimed-item ring
   uint64_t* iempty = ifull + 4;          // [4]
-  int64_t* s_items = reinterpret_cast<int64_t*>(iempty + 4);   // [4]
+  uint64_t* opfull = iempty + 4;         // [kOpStages] FP4 only
+  uint64_t* opempty = opfull + kOpStages;
+  uint64_t* rsfull = opempty + kOpStages;   // [kRsSlots]
+  int64_t* s_items = reinterpret_cast<int64_t*>(rsfull + kRsSlots);   // [4]
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_items + 4);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
   // per item-ring slot: visible entries per token, column weights w * qs
   int* s_nv = s_abort + 1;                                    // [4][TQ]
   float* s_w = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(s_nv + 4 * p.TQ) + 15) & ~uintptr_t(15));   // [4][N]
+  float* s_rs = s_w + 4 * p.N;                                // FP4: [kRsSlots][128] key row scales
 
   const uint32_t tmem_cols = p.N <= 16 ? 32u : (p.N <= 32 ? 64u : (p.N <= 64 ? 128u : (p.N <= 128 ? 256u : 512u)));
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], FP4 ? kConvThreads : 1); }
+    if (FP4) {
+      for (int o = 0; o < kOpStages; ++o) { mbar_init(&opfull[o], kConvThreads); mbar_init(&opempty[o], 1); }
+      for (int r = 0; r < kRsSlots; ++r) mbar_init(&rsfull[r], kConvThreads);
+    }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1); mbar_init(&tempty[a], kEpiThreads / 2);
       mbar_init(&qfull[a], 1); mbar_init(&qempty[a], 1);
     }
-    for (int i = 0; i < 4; ++i) { mbar_init(&ifull[i], 32); mbar_init(&iempty[i], 1 + kEpiThreads / 32); }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&ifull[i], 32);
+      mbar_init(&iempty[i], 1 + kEpiThreads / 32 + (FP4 ? kConvThreads / 32 : 0));
+    }
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -228,6 +332,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       if (lane == 0) {
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_q);
+        if (FP4) tma_prefetch_desc(&tmap_ks);
       }
       uint32_t gt = 0, ic = 0;
       bool ok = true;
@@ -246,9 +351,15 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             const int s = gt % kStages;
             const uint32_t ph = (gt / kStages) & 1;
             if (!wait_bar(&empty[s], ph ^ 1, abort_flag)) { ok = false; break; }
-            mbar_expect_tx(&full[s], a_bytes);
-            tma_load_2d(sA + s * a_bytes, &tmap_k, 0,
-                        (int32_t)((int64_t)it.b * p.cap + (int64_t)(it.tile0 + j) * 128), &full[s]);
+            const int64_t krow = (int64_t)it.b * p.cap + (int64_t)(it.tile0 + j) * 128;
+            if (FP4) {
+              mbar_expect_tx(&full[s], kFp4Stage);
+              tma_load_2d(sP + s * kFp4Stage, &tmap_k, 0, (int32_t)krow, &full[s]);
+              tma_load_2d(sP + s * kFp4Stage + kFp4Codes, &tmap_ks, 0, (int32_t)(krow / 4), &full[s]);
+            } else {
+              mbar_expect_tx(&full[s], a_bytes);
+              tma_load_2d(sA + s * a_bytes, &tmap_k, 0, (int32_t)krow, &full[s]);
+            }
           }
           ++ic;
         }
@@ -278,10 +389,12 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
           const uint32_t ph = (gt / kStages) & 1;
           const int acc = gt & 1;
           const uint32_t aph = (gt >> 1) & 1;
-          if (!wait_bar(&full[s], ph, abort_flag)) { ok = false; break; }
+          const int o = gt % kOpStages;
+          const uint32_t oph = (gt / kOpStages) & 1;
+          if (!wait_bar(FP4 ? &opfull[o] : &full[s], FP4 ? oph : ph, abort_flag)) { ok = false; break; }
           if (!wait_bar(&tempty[acc], aph ^ 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t dAs = dA + ((s * a_bytes) >> 4);
+          const uint64_t dAs = dA + (((FP4 ? o : s) * a_bytes) >> 4);
           const uint32_t d = tmem + acc * p.N;
           mma_f8(d, dAs, dB, idesc, 0);
           if (nk > 1) mma_f8(d, dAs + 2, dB + 2, idesc, 1);
@@ -289,7 +402,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             mma_f8(d, dAs + 4, dB + 4, idesc, 1);
             mma_f8(d, dAs + 6, dB + 6, idesc, 1);
           }
-          mma_commit(&empty[s]);
+          mma_commit(FP4 ? &opempty[o] : &empty[s]);
           mma_commit(&tfull[acc]);
         }
         if (!ok) break;
@@ -297,7 +410,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         ++ic;
       }
     }
-  } else {
+  } else if (!FP4 || warp < 10) {
     // ---------------- epilogue: 8 warps in two groups of four; group h owns
     // TMEM accumulator h and therefore every other tile, so two tiles'
     // epilogues run at once.  Each thread owns one key (TMEM lane) of a tile.
@@ -336,6 +449,12 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         ksc_next = key_scale(j + 2);          // issued a tile ahead: off the critical path
         if (!wait_bar(&tfull[acc], aph, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        float ksc_use = ksc;
+        if (FP4) {
+          const int r = g % kRsSlots;
+          if (!wait_bar(&rsfull[r], (g / kRsSlots) & 1, abort_flag)) { ok = false; break; }
+          ksc_use = s_rs[r * 128 + key_in_tile];
+        }
         const uint32_t tb = tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N;
         float run = 0.f;
         for (int cc = 0; cc < p.N; cc += 32) {
@@ -364,7 +483,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             run += pr[0];
             if (((cc + 32) & (p.HI - 1)) == 0) {
               const int tq = (cc + 31) >> log2hi;
-              if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = run * ksc;
+              if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = run * ksc_use;
               run = 0.f;
             }
           } else {
@@ -372,7 +491,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             for (int jj = 0; jj < 32; ++jj) {
               if ((jj & (p.HI - 1)) == 0) {
                 const int tq = (cc + jj) >> log2hi;
-                if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = pr[jj] * ksc;
+                if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = pr[jj] * ksc_use;
               }
             }
           }
@@ -383,6 +502,45 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       __syncwarp();
       if (lane == 0) release_item(kk);       // this warp is done with the slot's weights
       gt += it.n_tiles;
+    }
+  } else {
+    // ---------------- FP4 converter (warps 10-13): thread ct owns key row ct of
+    // every tile; staged packed tile -> e4m3 operand tile (128-byte swizzle, the
+    // layout TMA gives the FP8 path) + the row scale for the epilogue
+    const int ct = tid - kIdxThreads;
+    uint32_t gt = 0;
+    bool ok = true;
+    for (uint32_t kk = 0; ok; ++kk) {
+      const int64_t item = read_item(kk);
+      if (item >= p.n_items) {
+        __syncwarp();
+        if (lane == 0) release_item(kk);
+        break;
+      }
+      const IdxItem it = idx_item(p, item);
+      for (int j = 0; j < it.n_tiles; ++j, ++gt) {
+        const int s = gt % kStages, o = gt % kOpStages, r = gt % kRsSlots;
+        if (!wait_bar(&full[s], (gt / kStages) & 1, abort_flag)) { ok = false; break; }
+        if (!wait_bar(&opempty[o], ((gt / kOpStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        const uint8_t* st = sP + s * kFp4Stage;
+        uint4 c[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) c[b] = *reinterpret_cast<const uint4*>(st + ct * 64 + b * 16);
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(st + kFp4Codes + ct * 4);
+        uint4 out[8];
+        const float rs = fp4_row_to_e4m3(c, sc, out);
+        uint8_t* dst = sA + o * a_bytes;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(dst + swz128(ct, q)) = out[q];
+        s_rs[r * 128 + ct] = rs;
+        fence_proxy_async_smem();            // generic-proxy writes -> visible to the tensor core
+        mbar_arrive(&opfull[o]);
+        mbar_arrive(&empty[s]);
+        mbar_arrive(&rsfull[r]);
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) release_item(kk);
     }
   }
   __syncwarp();                 // reconverge role warps before the CTA barrier
@@ -780,37 +938,23 @@ extern "C" size_t csa_index_topk_workspace(int n_seq, int T, int64_t cap, int k)
   return ws_layout(n_seq, T, cap, k).total;
 }
 
-extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale, const float* w,
-                                       const uint8_t* kI, const float* kI_scale, const int64_t* q_pos,
-                                       int n_seq, int T, int HI, int DI, int64_t cap, int m, int k,
-                                       int32_t* idx, void* workspace, size_t ws_bytes, cudaStream_t stream) {
-  clear_error();
-  CSA_REQUIRE(n_seq >= 1 && T >= 1 && cap >= 1 && m >= 1, "csa_index_topk: n_seq, T, cap, m must be >= 1");
-  CSA_REQUIRE(DI == 32 || DI == 64 || DI == 128, "csa_index_topk: DI must be 32, 64 or 128");
-  CSA_REQUIRE(HI >= 1 && HI <= 64 && (HI & (HI - 1)) == 0, "csa_index_topk: HI must be a power of two <= 64");
-  CSA_REQUIRE(k >= 1 && k <= 2048, "csa_index_topk: k must be in [1, 2048]");
-  CSA_REQUIRE(qI && w && kI && q_pos && idx, "csa_index_topk: null pointer");
-  CSA_REQUIRE(aligned16(qI) && aligned16(kI) && aligned16(w) && aligned16(idx) && aligned16(q_pos) &&
-              (!qI_scale || aligned16(qI_scale)) && (!kI_scale || aligned16(kI_scale)),
-              "csa_index_topk: pointers must be 16-byte aligned");
-  CSA_REQUIRE((int64_t)n_seq * cap < (int64_t)1 << 31 && (int64_t)n_seq * T * HI < (int64_t)1 << 31,
-              "csa_index_topk: tensor too large for 32-bit TMA coordinates");
-  const WsLayout L = ws_layout(n_seq, T, cap, k);
-  if (!workspace || ws_bytes < L.total)
-    return fail(CSA_ERR_WORKSPACE, "csa_index_topk: workspace of %zu bytes needed, %zu given", L.total, ws_bytes);
-  CSA_REQUIRE(aligned16(workspace), "csa_index_topk: workspace must be 16-byte aligned");
-  if (L.n_chunks > 1 && (int64_t)L.n_chunks * k > kMergeCap)
-    return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: ceil(cap/%d) * k = %lld exceeds %d merge candidates",
-                kChunk, (long long)L.n_chunks * k, kMergeCap);
-  CSA_REQUIRE(L.n_chunks <= 64, "csa_index_topk: cap too large");
+namespace csa {
+namespace {
 
+// Scores kernel + top-k for both key formats.  FP8: kI e4m3 [rows, DI] with an
+// optional fp32 row scale kI_scale.  FP4 (kI_e8m0 != NULL): kI holds packed
+// E2M1 codes [rows, 64 B] and kI_e8m0 the block scale bytes [rows, 4]; DI 128.
+csa_status_t index_topk_run(const uint8_t* qI, const float* qI_scale, const float* w, const uint8_t* kI,
+                            const float* kI_scale, const uint8_t* kI_e8m0, const int64_t* q_pos, int n_seq, int T,
+                            int HI, int DI, int64_t cap, int m, int k, int32_t* idx, const WsLayout& L, uint8_t* ws,
+                            cudaStream_t stream) {
+  const bool fp4 = kI_e8m0 != nullptr;
   // token block: N = TQ * HI columns, a multiple of 32 and at most 256
   int TQ = 256 / HI;
   while (TQ > 1 && (TQ / 2) * HI >= 32 && TQ / 2 >= T) TQ /= 2;
   const int N = TQ * HI;
   if (N % 32 != 0) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: HI=%d gives no valid MMA width", HI);
 
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   IdxParams ip{};
   ip.qs = qI_scale; ip.w = w; ip.ks = kI_scale; ip.q_pos = q_pos;
   ip.scores = reinterpret_cast<float*>(ws + L.scores);
@@ -830,21 +974,38 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
   const int64_t n_kchunks = (tiles + chunk_tiles - 1) / chunk_tiles;
   ip.n_seq = n_seq; ip.n_qblocks = n_qblocks;
   ip.n_items = rows_blocks * n_kchunks;
-  CUtensorMap mk, mq;
-  if (!make_byte_map(&mk, kI, (uint64_t)n_seq * cap, DI, 128) ||
-      !make_byte_map(&mq, qI, (uint64_t)n_seq * T * HI, DI, N))
-    return fail(CSA_ERR_CUDA, "csa_index_topk: cuTensorMapEncodeTiled failed");
+  CUtensorMap mk, mq, mks;
+  bool maps_ok = make_byte_map(&mq, qI, (uint64_t)n_seq * T * HI, DI, N);
+  if (fp4) {
+    maps_ok = maps_ok &&
+              encode_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kI, 64, (uint64_t)n_seq * cap, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              encode_2d(&mks, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kI_e8m0, 16, (uint64_t)n_seq * cap / 4, 16, 32,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  } else {
+    maps_ok = maps_ok && make_byte_map(&mk, kI, (uint64_t)n_seq * cap, DI, 128);
+    mks = mk;
+  }
+  if (!maps_ok) return fail(CSA_ERR_CUDA, "csa_index_topk: cuTensorMapEncodeTiled failed");
 
-  const size_t smem = 1024 + 2 * (((size_t)N * DI + 1023) / 1024) * 1024 + (size_t)kStages * 128 * DI +
-                      (2 * kStages + 16) * 8 + 4 * 8 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4;
+  const size_t tiles_bytes = fp4 ? (size_t)kOpStages * 128 * DI + (size_t)kStages * kFp4Stage
+                                 : (size_t)kStages * 128 * DI;
+  const size_t smem = 1024 + 2 * (((size_t)N * DI + 1023) / 1024) * 1024 + tiles_bytes +
+                      (2 * kStages + 16 + 2 * kOpStages + kRsSlots) * 8 + 4 * 8 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4 +
+                      (fp4 ? (size_t)kRsSlots * 128 * 4 : 0);
   ip.item_counter = reinterpret_cast<uint32_t*>(ws + L.counter);
   {
     cudaError_t e = cudaMemsetAsync(ip.item_counter, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_index_topk: counter reset failed: %s", cudaGetErrorString(e));
   }
-  cudaFuncSetAttribute(indexer_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int grid = (int)std::min<int64_t>(ip.n_items, sms);
-  indexer_scores_kernel<<<grid, kIdxThreads, smem, stream>>>(mk, mq, ip);
+  if (fp4) {
+    cudaFuncSetAttribute(indexer_scores_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    indexer_scores_kernel<true><<<grid, kIdxThreadsFp4, smem, stream>>>(mk, mq, mks, ip);
+  } else {
+    cudaFuncSetAttribute(indexer_scores_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    indexer_scores_kernel<false><<<grid, kIdxThreads, smem, stream>>>(mk, mq, mks, ip);
+  }
   csa_status_t st = check_launch("csa_index_topk(scores)");
   if (st != CSA_OK) return st;
 
@@ -881,6 +1042,78 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
     st = check_launch("csa_index_topk(merge)");
   }
   return st;
+}
+
+}  // namespace
+}  // namespace csa
+
+extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale, const float* w,
+                                       const uint8_t* kI, const float* kI_scale, const int64_t* q_pos,
+                                       int n_seq, int T, int HI, int DI, int64_t cap, int m, int k,
+                                       int32_t* idx, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(n_seq >= 1 && T >= 1 && cap >= 1 && m >= 1, "csa_index_topk: n_seq, T, cap, m must be >= 1");
+  CSA_REQUIRE(DI == 32 || DI == 64 || DI == 128, "csa_index_topk: DI must be 32, 64 or 128");
+  CSA_REQUIRE(HI >= 1 && HI <= 64 && (HI & (HI - 1)) == 0, "csa_index_topk: HI must be a power of two <= 64");
+  CSA_REQUIRE(k >= 1 && k <= 2048, "csa_index_topk: k must be in [1, 2048]");
+  CSA_REQUIRE(qI && w && kI && q_pos && idx, "csa_index_topk: null pointer");
+  CSA_REQUIRE(aligned16(qI) && aligned16(kI) && aligned16(w) && aligned16(idx) && aligned16(q_pos) &&
+              (!qI_scale || aligned16(qI_scale)) && (!kI_scale || aligned16(kI_scale)),
+              "csa_index_topk: pointers must be 16-byte aligned");
+  CSA_REQUIRE((int64_t)n_seq * cap < (int64_t)1 << 31 && (int64_t)n_seq * T * HI < (int64_t)1 << 31,
+              "csa_index_topk: tensor too large for 32-bit TMA coordinates");
+  const WsLayout L = ws_layout(n_seq, T, cap, k);
+  if (!workspace || ws_bytes < L.total)
+    return fail(CSA_ERR_WORKSPACE, "csa_index_topk: workspace of %zu bytes needed, %zu given", L.total, ws_bytes);
+  CSA_REQUIRE(aligned16(workspace), "csa_index_topk: workspace must be 16-byte aligned");
+  if (L.n_chunks > 1 && (int64_t)L.n_chunks * k > kMergeCap)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: ceil(cap/%d) * k = %lld exceeds %d merge candidates",
+                kChunk, (long long)L.n_chunks * k, kMergeCap);
+  CSA_REQUIRE(L.n_chunks <= 64, "csa_index_topk: cap too large");
+
+  return index_topk_run(qI, qI_scale, w, kI, kI_scale, nullptr, q_pos, n_seq, T, HI, DI, cap, m, k, idx, L,
+                        static_cast<uint8_t*>(workspace), stream);
+}
+
+namespace {
+inline size_t fp4_query_bytes(int n_seq, int T, int HI) {
+  const size_t rows = (size_t)n_seq * T * HI;
+  return align_up(rows * 128, 256) + align_up(rows * 4, 256);
+}
+}  // namespace
+
+extern "C" size_t csa_index_topk_fp4_workspace(int n_seq, int T, int HI, int64_t cap, int k) {
+  if (n_seq <= 0 || T <= 0 || HI <= 0 || cap <= 0 || k <= 0) return 0;
+  return ws_layout(n_seq, T, cap, k).total + fp4_query_bytes(n_seq, T, HI);
+}
+
+extern "C" csa_status_t csa_index_topk_fp4(const uint8_t* qI4, const uint8_t* qI4_scale, const float* w,
+                                           const uint8_t* kI4, const uint8_t* kI4_scale, const int64_t* q_pos,
+                                           int n_seq, int T, int HI, int64_t cap, int m, int k, int32_t* idx,
+                                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(n_seq >= 1 && T >= 1 && cap >= 1 && m >= 1, "csa_index_topk_fp4: n_seq, T, cap, m must be >= 1");
+  CSA_REQUIRE(cap % 4 == 0, "csa_index_topk_fp4: cap must be a multiple of 4");
+  CSA_REQUIRE(HI >= 1 && HI <= 64 && (HI & (HI - 1)) == 0, "csa_index_topk_fp4: HI must be a power of two <= 64");
+  CSA_REQUIRE(k >= 1 && k <= 2048, "csa_index_topk_fp4: k must be in [1, 2048]");
+  CSA_REQUIRE(qI4 && qI4_scale && w && kI4 && kI4_scale && q_pos && idx, "csa_index_topk_fp4: null pointer");
+  CSA_REQUIRE(aligned16(qI4) && aligned16(qI4_scale) && aligned16(kI4) && aligned16(kI4_scale) && aligned16(w) &&
+              aligned16(idx) && aligned16(q_pos), "csa_index_topk_fp4: pointers must be 16-byte aligned");
+  CSA_REQUIRE((int64_t)n_seq * cap < (int64_t)1 << 31 && (int64_t)n_seq * T * HI < (int64_t)1 << 31,
+              "csa_index_topk_fp4: tensor too large for 32-bit TMA coordinates");
+  const WsLayout L = ws_layout(n_seq, T, cap, k);
+  const size_t need = L.total + fp4_query_bytes(n_seq, T, HI);
+  if (!workspace || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "csa_index_topk_fp4: workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  CSA_REQUIRE(aligned16(workspace), "csa_index_topk_fp4: workspace must be 16-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t qrows = (int64_t)n_seq * T * HI;
+  uint8_t* q8 = ws + L.total;
+  float* qs = reinterpret_cast<float*>(q8 + align_up((size_t)qrows * 128, 256));
+  fp4_rows_to_e4m3_kernel<<<(unsigned)((qrows + 127) / 128), 128, 0, stream>>>(qI4, qI4_scale, qrows, q8, qs);
+  csa_status_t st = check_launch("csa_index_topk_fp4(query)");
+  if (st != CSA_OK) return st;
+  return index_topk_run(q8, qs, w, kI4, nullptr, kI4_scale, q_pos, n_seq, T, HI, 128, cap, m, k, idx, L, ws, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -157,3 +157,15 @@ def test_layer_workspace_is_the_larger_of_the_two(L):
     assert L.csa_workspace_size(1, 16384, 4096, 512, 64, 512, 1) == L.csa_index_topk_workspace(1, 16384, 4096, 512)
     L.csa_compress(None, None, None, None, None, 64, 7, 4, 1, 0, 0, 0, 10000.0, 1e-6, None, 0, None)
     assert L.csa_get_last_error_string() == L.csa_last_error() != b""
+
+
+def test_fp4_indexer_host_validation(L):
+    p = ctypes.c_void_p(16)
+    base = L.csa_index_topk_workspace(2, 1, 4096, 512)
+    assert L.csa_index_topk_fp4_workspace(2, 1, 64, 4096, 512) == base + 2 * 64 * 128 + 512
+    # cap not a multiple of 4
+    st = L.csa_index_topk_fp4(p, p, p, p, p, p, 2, 1, 64, 4095, 4, 512, p, p, 1 << 30, None)
+    assert st == 1 and b"multiple of 4" in L.csa_last_error()
+    # workspace too small
+    st = L.csa_index_topk_fp4(p, p, p, p, p, p, 2, 1, 64, 4096, 4, 512, p, p, 16, None)
+    assert st == 3
