@@ -141,6 +141,56 @@ def test_decode_matches_prefill_last_row():
     np.testing.assert_allclose(Od, Og[t], rtol=1e-13)
 
 
+def _decode_operands(x, t, m, overlap, W, norm_rope):
+    """The decode functions' inputs at position t, built from the prefill
+    definitions: the query row, every cache entry, and the raw window rows
+    [max(0, t - W + 1), t], each normalised and rotated when norm_rope."""
+    kv = O.compress(x["C"], x["Z"], x["B"], m, overlap)
+    lo = max(0, t - W + 1)
+    q, swa = x["q"][t], x["C"][lo:t + 1]
+    if norm_rope:
+        q = O.rope_partial(O.rmsnorm(q), np.full(q.shape[0], t))
+        kv = O.rope_partial(O.rmsnorm(kv), np.arange(kv.shape[0]) * m)
+        swa = O.rope_partial(O.rmsnorm(swa), np.arange(lo, t + 1))
+    return q, kv, swa
+
+
+@pytest.mark.parametrize("norm_rope", [False, True])
+@pytest.mark.parametrize("t", [255, 128, 129, 20])
+def test_hca_decode_matches_prefill_row(norm_rope, t):
+    """[CS] "HCA": dense attention over every complete 128-token entry; [LD]:
+    plus the 128-token raw window and the sink in one softmax, inverse RoPE on
+    the output.  Decoding the token at position t against caches that hold the
+    prefill's entries and the last W raw rows must reproduce row t of the
+    prefill layer: at the last position, at the first token after a block
+    boundary (a newly visible entry), one token later, and before any entry is
+    complete (window only)."""
+    m, W, S = 32, 40, 256
+    x = _layer_inputs(S, 3, 128, m, nb=m, seed=7)
+    Og = O.hca_layer(x["q"], x["C"], x["Z"], x["B"], x["sink"], m=m, W=W, norm_rope=norm_rope,
+                     inv_rope=norm_rope)
+    q, kv, swa = _decode_operands(x, t, m, False, W, norm_rope)
+    Od = O.hca_decode(q, kv, swa, x["sink"], t, m=m, inv_rope=norm_rope)
+    np.testing.assert_allclose(Od, Og[t], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("norm_rope", [False, True])
+@pytest.mark.parametrize("t", [255, 128, 129])
+def test_csa_decode_matches_prefill_row_with_rope(norm_rope, t):
+    """As test_decode_matches_prefill_last_row, with the QK normalisation, the
+    partial RoPE of queries, entries and window rows, and the inverse RoPE of
+    the output ([CS] "其他辅助设计"; [LD]), at a block boundary as well."""
+    m, W, S = 4, 40, 256
+    x = _layer_inputs(S, 3, 128, m, seed=8)
+    Og, idx = O.csa_layer(x["q"], x["C"], x["Z"], x["B"], x["qI"], x["w"], x["kI"], x["sink"], k=9, m=m, W=W,
+                          norm_rope=norm_rope, inv_rope=norm_rope)
+    q, kv, swa = _decode_operands(x, t, m, True, W, norm_rope)
+    Od, idd = O.csa_decode(q, x["qI"][t], x["w"][t], x["kI"], kv, swa, x["sink"], t, k=9, m=m,
+                           inv_rope=norm_rope)
+    np.testing.assert_array_equal(idd, idx[t])
+    np.testing.assert_allclose(Od, Og[t], rtol=1e-12, atol=1e-13)
+
+
 def test_flop_counts_match_workload_table():
     a, i = O.flop_counts(16384, 64, 512, 4, k=512, HI=64, DI=128)
     assert abs(a / 1e12 - 1.305) < 0.01 and abs(i / 1e12 - 0.550) < 0.01
