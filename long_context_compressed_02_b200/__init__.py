@@ -192,6 +192,10 @@ def csa_index_topk(qI, w, kI, q_pos, m, k, *, qI_scale=None, kI_scale=None, work
     return idx
 
 
+def csa_index_topk_fp4_workspace(n_seq, T, HI, cap, k):
+    return int(lib().csa_index_topk_fp4_workspace(n_seq, T, HI, cap, k))
+
+
 def csa_index_topk_fp4(qI4, qI4_scale, w, kI4, kI4_scale, q_pos, m, k, *, workspace=None, idx=None, stream=None):
     """Lightning indexer + top-k on MX FP4 operands: qI4 [n_seq, T, HI, 64] and
     kI4 [n_seq, cap, 64] uint8 (packed E2M1, the even element in the low
