@@ -19,10 +19,7 @@ import argparse
 import json
 import math
 import os
-import signal
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -51,6 +48,29 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def fp8_peak_tflops(torch, dev, n=8192, reps=10):
+    """Dense e4m3 tensor throughput of this GPU, measured here with the library
+    FP8 GEMM (torch._scaled_mm, cuBLASLt) on n^3, best of `reps` by CUDA events:
+    the roofline denominator of the FP8 indexer (no FP8 figure is recorded with
+    the measured HBM and BF16 peaks).  None if the library call is unavailable."""
+    try:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev)
+        best = None
+        for _ in range(reps + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1) * 1e-3
+            best = t if best is None else min(best, t)
+        return 2.0 * n ** 3 / best / 1e12
+    except Exception:
+        return None
+
+
 def _flops(S, H, D, m, k, W, HI, DI):
     t = np.arange(S, dtype=np.int64)
     nv = (t + 1) // m
@@ -61,53 +81,81 @@ def _flops(S, H, D, m, k, W, HI, DI):
 
 
 class Clocks:
-    """Samples nvidia-smi during the timed region."""
+    """Samples the GPU's SM clock, power and clock-event reasons every 10 ms
+    from a background thread (NVML, read-only queries) while the benchmark
+    runs; summary() reports the samples taken between mark_start() and
+    mark_end().  Falls back to nothing if NVML is unavailable."""
 
-    def __init__(self, index):
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, torch, device):
+        import threading
+        self.samples, self.t0, self.t1 = [], None, None
+        self.stop_ev = threading.Event()
+        self.h = None
         try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.p = None
+            self.h = None
+            return
+        self.th = threading.Thread(target=self._run, daemon=True)
+        self.th.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.h),
+                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
+            except Exception:
+                pass
+            self.stop_ev.wait(0.01)
+
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
-        if self.p is None:
+        if self.h is None:
             return None
-        self.p.send_signal(signal.SIGTERM)
-        try:
-            self.p.wait(timeout=5)
-        except Exception:
-            self.p.kill()
-        self.f.flush()
-        rows = []
-        with open(self.f.name) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.f.name)
+        self.stop_ev.set()
+        self.th.join(timeout=2)
+        rows = [r for r in self.samples if self.t0 is not None and self.t0 <= r[0] <= (self.t1 or r[0])]
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows)}
+        reasons = sorted({n for r in rows for n, bit in self.REASONS if r[2] & bit})
+        return {"sm_mhz": float(np.median([r[1] for r in rows])), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(r[3] for r in rows),
+                "source": "NVML every 10 ms during the timed region"}
+
+
+# Query rows per oracle sample: the reference arm times one such sample per
+# step and the cpu_baseline leg one sample, so both rates are the same
+# measurement (each sample also runs the oracle's full-sequence compressor
+# and window-row passes, whose cost is spread over these rows).
+ORACLE_ROWS = 2048
+
+
+def oracle_rows(S, shift=0):
+    """ORACLE_ROWS evenly spaced query rows of an S-token layer, moved by
+    `shift` (different samples for different reference-arm steps)."""
+    base = np.linspace(0, S - 1, min(S, ORACLE_ROWS)).astype(np.int64)
+    return np.unique(np.minimum(S - 1, base + shift))
 
 
 def cpu_oracle_sample(inp_host, cfg, rows):
     """Times the float64 oracle on the given query rows of the workload."""
     import oracle as O
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    except Exception:
-        cores = len(os.sched_getaffinity(0))
+    cores = _blas_threads()
     t0 = time.perf_counter()
     O.csa_layer(inp_host["q"][rows], inp_host["C"], inp_host["Z"], inp_host["B"],
                 O.e4m3_decode(inp_host["qI_codes"][rows]), inp_host["w"][rows],
@@ -135,11 +183,10 @@ def run_reference(args, rank, world):
     from long_context_compressed_02_b200 import synth
     inp, cfg = synth.prefill_inputs_device(WORKLOAD, "cpu", seed=0)
     host = host_inputs(inp)
-    rng = np.random.default_rng(0)
     times, flops = [], []
     cores = 1
     for step in range(args.warmup + args.steps):
-        rows = np.sort(rng.choice(cfg["S"], 8, replace=False))
+        rows = oracle_rows(cfg["S"], shift=step)
         fl, dt, cores = cpu_oracle_sample(host, cfg, rows)
         if step >= args.warmup:
             times.append(dt)
@@ -149,15 +196,52 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "S": cfg["S"], "H": cfg["H"], "D": cfg["D"], "m": cfg["m"],
-                       "top_k": cfg["k"], "window": cfg["W"], "sample": "8 random query rows per step"},
+                       "top_k": cfg["k"], "window": cfg["W"],
+                       "sample": f"{ORACLE_ROWS} evenly spaced query rows per step (shifted by the step index)"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": "8 random query rows of the S=16384 layer per step (oracle recomputes the "
-                                       "compressor and window rows each call)"},
+                             "sample": f"{ORACLE_ROWS} evenly spaced query rows of the S=16384 layer per step, "
+                                       "including the oracle's full-sequence compressor and window-row passes "
+                                       "(the same sample as the native arm's cpu_baseline)"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1, n_split=None):
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def decode_oracle_sample(inp, cfg, b=0):
+    """Times the float64 oracle's whole decode step (indexer over every visible
+    entry, top-k, attention over the selected entries + SWA cache + sink) for
+    sequence b of the batch.  Its inputs, the caches decoded exactly to float64
+    through the e4m3 code table, are prepared before the clock starts."""
+    import oracle as O
+    tab = O.e4m3_decode(np.arange(256, dtype=np.uint8))
+    D, ne = cfg["D"], cfg["n_e"]
+    kI = tab[inp["kI"][b].cpu().numpy()] * inp["kI_scale"][b].double().cpu().numpy()[:, None]
+    qI = tab[inp["qI"][b, 0].cpu().numpy()] * inp["qI_scale"][b, 0].double().cpu().numpy()[:, None]
+    kv = np.empty((ne, D))
+    kv[:, :D - 64] = tab[inp["kv_nope"][b].cpu().numpy()]
+    kv[:, :D - 64] *= inp["kv_scale"][b].double().cpu().numpy()[:, None]
+    kv[:, D - 64:] = inp["kv_rope"][b].double().cpu().numpy()
+    q = inp["q"][b, 0].double().cpu().numpy()
+    w = inp["w"][b, 0].double().cpu().numpy()
+    swa = inp["swa"][b].double().cpu().numpy()
+    sink = inp["sink"].double().cpu().numpy()
+    t = int(inp["q_pos"][b].item())
+    t0 = time.perf_counter()
+    O.csa_decode(q, qI, w, kI, kv, swa, sink, t, k=cfg["k"], m=4, inv_rope=True)
+    dt = time.perf_counter() - t0
+    return {"value": 1.0 / dt, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"one whole decode step of sequence {b} ({ne} entries, top-k {cfg['k']}), {dt:.2f} s; "
+                      "caches decoded to float64 beforehand"}
+
+
+def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1, n_split=None, cpu_baseline=False):
     """CSA decode at 2^20 context, batch 16 (one new token per sequence): indexer
     scan over the e4m3 key cache + top-k, then the fused attention over the 512
     selected e4m3 entries, the 128-row bf16 SWA cache and the sink."""
@@ -230,7 +314,8 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1, n_spli
     algo = scan + gather + swa + qbytes
     hbm, _, _, src = _peaks()
     ach_idx = scan / (t_idx * 1e-3) / 1e9
-    return {"workload": "csa_decode_1m", "batch": Bn, "attention_splits": n_split, "context": cfg["ctx"], "entries": ne, "top_k": k,
+    cpu = decode_oracle_sample(inp, cfg) if cpu_baseline else None
+    return {"workload": "csa_decode_1m", "batch": Bn, "cpu_baseline": cpu, "attention_splits": n_split, "context": cfg["ctx"], "entries": ne, "top_k": k,
             "tokens_per_s": Bn / (ms * 1e-3), "ms_per_step": ms, "kernels_ms": {"index_topk": t_idx,
                                                                                  "fused_attention": t_att},
             "algorithmic_bytes_per_step": algo,
@@ -413,15 +498,15 @@ def hca_prefill_leg(dev, steps, warmup, csa, synth, torch, seed=0):
     t = np.arange(S, dtype=np.int64)
     fl_dense = 4 * D * H * int(((t + 1) // m).sum())
     fl_window = 4 * D * H * int(np.minimum(W, t + 1).sum())
-    _, _, bf16_sus, src = _peaks()
+    _, bf16_burst, _, src = _peaks()
     ach = (fl_dense + fl_window) / (per["fused_attention"] * 1e-3) / 1e12
     return {"workload": "hca_prefill", "S": S, "H": H, "D": D, "m": m, "entries": ne, "window": W,
             "tflops": (fl_dense + fl_window) / (ms * 1e-3) / 1e12, "ms_per_step": ms,
             "prefill_tokens_per_s": S / (ms * 1e-3), "kernels_ms": per,
             "flops_per_step": {"hca_dense": fl_dense, "swa_window": fl_window},
-            "roofline": {"kernel": "fused_attention", "bound": "tensor", "achieved": ach, "peak": bf16_sus,
-                         "unit": "TFLOP/s", "frac": ach / bf16_sus, "traffic": None,
-                         "peak_source": f"{src} bf16 sustained"}}
+            "roofline": {"kernel": "fused_attention", "bound": "tensor", "achieved": ach, "peak": bf16_burst,
+                         "unit": "TFLOP/s", "frac": ach / bf16_burst, "traffic": None,
+                         "peak_source": f"{src} bf16 burst (timed region well under a second)"}}
 
 
 def out_proj_leg(dev, steps, warmup, csa, synth, torch, seed=0, S=None):
@@ -492,7 +577,7 @@ def tiny_leg(dev, steps, warmup, csa, synth, torch):
     csa.check_device_error()
     ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
     sparse, window, indexer = _flops(S, H, D, m, k, W, HI, DI)
-    return {"workload": "tiny_csa", "S": S, "H": H, "D": D, "dtype": "f32 storage, bf16 attention operands",
+    return {"workload": "tiny_csa", "S": S, "H": H, "D": D, "dtype": "f32 storage and fp32 attention arithmetic",
             "us_per_step": ms * 1e3, "kernels_per_step": 4,
             "flops_per_step": {"attention": sparse + window, "indexer_fp8": indexer},
             "bound": "launch latency"}
@@ -588,6 +673,7 @@ def main():
         mark(5)
 
     launches_per_step = 6      # 2 norm/rope, compress, indexer scores, top-k, fused attention
+    clocks = Clocks(torch, dev) if rank == 0 else None
     for _ in range(max(3, args.warmup)):
         step()
     csa.check_device_error()
@@ -597,16 +683,19 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    clocks = Clocks(torch.cuda.current_device()) if rank == 0 else None
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     barrier()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    if clocks:
+        clocks.mark_start()
     t_start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t_end.record(stream)
     barrier()
+    if clocks:
+        clocks.mark_end()
     clk = clocks.stop() if clocks else None
     csa.check_device_error()
     ms = t_start.elapsed_time(t_end) / args.steps
@@ -671,42 +760,47 @@ def main():
                "steps": n_e2e, "pipelined": "uploads / compute / downloads of consecutive steps overlap"}
         del dev_in, dev_out
 
-    # ---- roofline of the dominant call
+    # ---- roofline of the dominant call.  The timed region lasts a fraction of
+    # a second at the maximum SM clock, so the BF16 denominator is the measured
+    # burst figure; the FP8 one is measured in this run (fp8_peak_tflops).
     hbm, bf16_burst, bf16_sus, src = _peaks()
-    algo = {"fused_attention": (fl_sparse + fl_window, "tensor", bf16_sus),
-            "index_topk": (fl_index, "tensor", 2 * bf16_sus)}
+    fp8_peak = fp8_peak_tflops(torch, dev)
+    algo = {"fused_attention": (fl_sparse + fl_window, "tensor", bf16_burst, f"{src} bf16 burst"),
+            "index_topk": (fl_index, "tensor", fp8_peak,
+                           "e4m3 GEMM measured in this run (torch._scaled_mm 8192^3, best of 10)")}
     dom = max(per, key=per.get)
-    if dom in algo:
-        fl, bound, peak = algo[dom]
+    if dom in algo and algo[dom][2]:
+        fl, bound, peak, psrc = algo[dom]
         ach = fl / (per[dom] * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": bound, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak,
                 "traffic": PROFILED_TRAFFIC.get(dom) if args.S is None else None,
-                "peak_source": f"{src} bf16 sustained" + (" x2 (fp8 nominal ratio)" if dom == "index_topk" else "")}
+                "peak_source": psrc}
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s", "frac": None,
                 "traffic": None}
+    idx_ach = fl_index / (per["index_topk"] * 1e-3) / 1e12
+    indexer_roof = {"kernel": "index_topk", "bound": "tensor", "achieved": idx_ach, "peak": fp8_peak,
+                    "unit": "TFLOP/s", "frac": idx_ach / fp8_peak if fp8_peak else None,
+                    "peak_source": algo["index_topk"][3]}
 
     decode = decode_fp4 = None
     if not args.no_decode and args.S is None:
         decode = decode_leg(dev, args.steps, args.warmup, csa, synth, torch, batch=args.decode_batch,
-                                        seed=replicas.replica_seed(rank, base=1))
+                            seed=replicas.replica_seed(rank, base=1),
+                            cpu_baseline=rank == 0 and world == 1 and not args.no_cpu_baseline)
         if args.decode_batch is None:
             decode_fp4 = decode_fp4_leg(dev, args.steps, args.warmup, csa, synth, torch,
                                         seed=replicas.replica_seed(rank, base=1))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = host_inputs(inp)
-        n_rows, fl, dt = 32, 0.0, 0.0
-        while True:
-            rows = np.linspace(0, S - 1, n_rows).astype(np.int64)
-            fl, dt, cores = cpu_oracle_sample(host, cfg, rows)
-            if dt >= 8.0 or n_rows >= S:
-                break
-            n_rows = min(S, int(n_rows * max(2.0, 10.0 / max(dt, 1e-3))))
+        rows = oracle_rows(S)
+        fl, dt, cores = cpu_oracle_sample(host, cfg, rows)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n_rows} evenly spaced query rows of the same S=16384 layer (float64 numpy oracle, "
-                         f"{dt:.1f} s including its full-sequence compressor and window-row passes)"}
+               "sample": f"{len(rows)} evenly spaced query rows of the same S={S} layer (float64 numpy oracle, "
+                         f"{dt:.1f} s including its full-sequence compressor and window-row passes; the "
+                         f"reference arm times the same sample per step)"}
 
     hca = mixed = proj = tiny = None
     if args.S is None:
@@ -735,7 +829,7 @@ def main():
                            "flops_per_step": {"sparse_mqa": fl_sparse, "swa_window": fl_window,
                                               "indexer_fp8": fl_index}},
                 "prefill_tokens_per_s": replicas.job_rate(S, world, ms * 1e-3),
-                "kernels_ms": per, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode, "decode_1m_fp4": decode_fp4,
+                "kernels_ms": per, "roofline": roof, "indexer_roofline": indexer_roof, "cpu_baseline": cpu, "e2e": e2e, "decode_1m": decode, "decode_1m_fp4": decode_fp4,
                 "hca_prefill": hca, "decode_mixed": mixed, "out_proj": proj, "tiny_csa": tiny,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)

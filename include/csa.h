@@ -162,6 +162,11 @@ csa_status_t csa_compress_append(const void* c_tok, const void* z_tok, csa_dtype
  *            calls sharing one workspace must be ordered on one stream.
  * Requires DI in {32, 64, 128}; HI in {1,2,4,...,64} (power of two <= 64 whose
  * product with the token block is a multiple of 16); 1 <= k <= 2048; cap >= 1.
+ * Rows longer than 16384 entries are cut into chunks of 16384 whose candidates
+ * are merged: ceil(cap / 16384) * k must not exceed 16384 (CSA_ERR_UNSUPPORTED
+ * otherwise), which allows cap = 262144 entries (a 2^20-token context at
+ * m = 4) at k = 1024 and cap = 131072 at k = 2048.
+ * csa_index_topk_workspace returns 0 when n_seq * T * cap * 4 overflows size_t.
  * ------------------------------------------------------------------------- */
 size_t csa_index_topk_workspace(int n_seq, int T, int64_t cap, int k);
 csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale, const float* w,
@@ -180,13 +185,16 @@ csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale, const floa
  * and results are those of csa_index_topk; a call whose scratch would exceed
  * 32 MiB (csa_index_topk_workspace(n_seq, T, cap, k), dominated by
  * n_seq * T * cap * 4 bytes of scores) returns CSA_ERR_UNSUPPORTED.
- * The first call on each device looks up the array's device address (a CUDA
- * runtime query), so make that first call before any stream capture.  Every
- * call on a device shares the same array and it keeps the previous call's
- * contents (each kernel overwrites every scratch byte before reading it, so
- * nothing needs clearing); calls that may overlap on the GPU (different
- * streams, or host threads racing) must be serialised by the caller.  No
- * memory is allocated or freed.
+ * The first call in each CUDA context looks up the array's device address (a
+ * CUDA runtime query, cached per context, so a context created after
+ * cudaDeviceReset gets a fresh lookup); make that first call before any stream
+ * capture.  Every call on a device shares the same array, which keeps the
+ * previous call's contents: the call resets, with stream-ordered memsets inside
+ * the array, the work-item counter and (rows longer than 16384 entries) the
+ * key histograms it uses, and it reads only score entries it has written
+ * itself, so earlier contents never reach the result.  Calls that may overlap
+ * on the GPU (different streams, or host threads racing) race on the array and
+ * must be serialised by the caller.  No memory is allocated or freed.
  * ------------------------------------------------------------------------- */
 csa_status_t csa_index_topk_noalloc(const uint8_t* qI, const float* qI_scale, const float* w,
                                     const uint8_t* kI, const float* kI_scale, const int64_t* q_pos,
@@ -224,9 +232,12 @@ csa_status_t csa_index_topk_fp4(const uint8_t* qI4, const uint8_t* qI4_scale, co
  * Outputs of the two partial calls: O_part [n_seq, T, H, D] fp32 normalised by
  * the branch's own softmax sum, lse_part [n_seq, T, H] fp32 natural-log
  * log-sum-exp of the branch logits (-inf and O = 0 when the set is empty).
- * Computation: BF16 tensor-core products (F32 inputs are rounded to BF16),
- * fp32 accumulation and softmax.  Requires D in {128, 512}, H <= 64,
- * rope_dim in {0, 64} (E4M3 needs 64).
+ * Computation: when q, the entries and the window rows are all F32 (the
+ * float32 workloads), fp32 arithmetic throughout on CUDA cores (fused
+ * multiply-add dot products, expf); otherwise BF16 tensor-core products (an
+ * F32 operand next to a BF16 one is rounded to BF16) with fp32 accumulation
+ * and softmax.  Requires D in {128, 512}, H <= 64, rope_dim in {0, 64} (E4M3
+ * needs 64).
  * ------------------------------------------------------------------------- */
 
 /* csa_sparse_mqa — CSA main branch: rows kv[b, idx[b,t,j]] for idx >= 0.

@@ -92,7 +92,8 @@ struct AttnParams {
   int src2, W;
   const int64_t* q_pos;     // [n_seq] (null: 0)
   int n_seq, T, H;
-  float scale_log2;
+  float scale;              // softmax scale of the logits
+  float scale_log2;         // the same times log2(e)
   float* O_part;            // partial outputs
   float* lse_part;
   const float* O_in;        // combine inputs (may be null)
@@ -975,6 +976,177 @@ attn_merge_kernel(const float* __restrict__ Os, const float* __restrict__ Ls, co
   }
 }
 
+// ---------------------------------------------------------------------------
+// float32 attention on CUDA cores: the path of calls whose queries, entries
+// and window rows are all fp32 (the tiny float32 layer).  The same row set,
+// softmax, sink merge and inverse RoPE as attn_kernel, in fp32 arithmetic
+// throughout (fused multiply-add dot products, expf), so the result is an
+// fp32-rounded evaluation of the definition instead of one on bf16 operands.
+// One CTA per (work item, group of heads); TPH threads per head, thread
+// (head hl, index li) owning dims li + TPH j (j < 16) of its head, so a dim d
+// and its RoPE partner d + 32 belong to the same thread.  A CTA holds
+// min(H, 4096 / D) heads (blockDim.x / TPH), so few-head calls use small CTAs
+// and more of them fit on an SM.  Rows are staged 32 at a time in shared memory.
+constexpr int kF32MaxThreads = 256;
+constexpr int kF32Rows = 32;
+
+template <int D>
+__global__ void __launch_bounds__(kF32MaxThreads)
+attn_f32_kernel(const __grid_constant__ AttnParams p, int epi) {
+  constexpr int TPH = D == 128 ? 8 : 32;      // threads per head
+  constexpr int NJ = D / TPH;                 // dims per thread: 16
+  const int HG = blockDim.x / TPH;            // heads per CTA
+  extern __shared__ float4 s_rows4[];         // [kF32Rows][D]
+  float* s_rows = reinterpret_cast<float*>(s_rows4);
+  __shared__ RowSet s_rs;
+  const int tid = threadIdx.x, hl = tid / TPH, li = tid % TPH;
+  const int64_t item = blockIdx.x;
+  const int64_t bt = item / p.n_split;
+  const int sp = (int)(item % p.n_split);
+  const int b = (int)(bt / p.T), t = (int)(bt % p.T);
+  const int h = blockIdx.y * HG + hl;
+  const bool hv = h < p.H;
+  if (tid < 32) {
+    const RowSet r = row_set_warp(p, b, t, sp, tid);
+    if (tid == 0) s_rs = r;
+  }
+  __syncthreads();
+  const RowSet rs = s_rs;
+  const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
+  const float scale = p.scale;
+  float q[NJ], o[NJ];
+  {
+    const float* qr = reinterpret_cast<const float*>(p.q) + (bt * p.H + (hv ? h : 0)) * D;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) { q[j] = hv ? qr[li + TPH * j] : 0.f; o[j] = 0.f; }
+  }
+  float m = -CUDART_INF_F, l = 0.f;
+  for (int c = rs.c0; c < rs.c1; ++c) {
+    const bool win = c < rs.nh2;
+    const int base = (win ? c : c - rs.nh2) * kRows;
+    const int nset = win ? rs.n2 : rs.n1;
+    for (int r0 = base; r0 < base + kRows && r0 < nset; r0 += kF32Rows) {
+      const int nr = min(kF32Rows, nset - r0);
+      // stage the rows (whole warps per row segment, 16-byte loads)
+      for (int u = tid; u < nr * (D / 4); u += blockDim.x) {
+        const int rr = u / (D / 4), c4 = u % (D / 4);
+        const int r = r0 + rr;
+        int64_t row = r;
+        bool ok = true;
+        if (win) {
+          row = rs.lo2 + r;
+        } else if (rs.idx) {
+          row = rs.idx[r];
+          if (row < 0 || row >= p.cap) { ok = false; if (c4 == 0) atomicOr(&g_err_attn, DEV_ERR_BAD_INDEX); }
+        }
+        const float* src = win ? reinterpret_cast<const float*>(p.kv2) + ((int64_t)b * p.cap2 + row) * D
+                               : reinterpret_cast<const float*>(p.kv) + ((int64_t)b * p.cap + (ok ? row : 0)) * D;
+        s_rows4[rr * (D / 4) + c4] = ok ? __ldg(reinterpret_cast<const float4*>(src) + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      __syncthreads();
+      float s[kF32Rows];
+#pragma unroll
+      for (int rr = 0; rr < kF32Rows; ++rr) {
+        float acc = 0.f;
+        if (rr < nr) {
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) acc = fmaf(q[j], s_rows[rr * D + li + TPH * j], acc);
+        }
+#pragma unroll
+        for (int off = TPH / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        s[rr] = rr < nr ? acc * scale : -CUDART_INF_F;
+      }
+      float mx = m;
+#pragma unroll
+      for (int rr = 0; rr < kF32Rows; ++rr) mx = fmaxf(mx, s[rr]);
+      const float alpha = (m == -CUDART_INF_F) ? 0.f : expf(m - mx);
+      l *= alpha;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) o[j] *= alpha;
+#pragma unroll
+      for (int rr = 0; rr < kF32Rows; ++rr) {
+        if (rr < nr) {
+          const float pr = expf(s[rr] - mx);
+          l += pr;
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) o[j] = fmaf(pr, s_rows[rr * D + li + TPH * j], o[j]);
+        }
+      }
+      m = mx;
+      __syncthreads();
+    }
+  }
+  if (!hv) return;
+  const float lse_w = l > 0.f ? m + logf(l) : -CUDART_INF_F;
+  if (epi == EPI_PARTIAL) {
+    const int64_t orow = (bt * p.n_split + sp) * p.H + h;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) p.O_part[orow * D + li + TPH * j] = o[j] * inv;
+    if (li == 0) p.lse_part[orow] = lse_w;
+    return;
+  }
+  const int64_t orow = bt * p.H + h;
+  const float lse_p = p.O_in ? p.lse_in[orow] : -CUDART_INF_F;
+  const float sk = p.sink ? p.sink[h] : -CUDART_INF_F;
+  float M = fmaxf(fmaxf(lse_w, lse_p), sk);
+  if (M == -CUDART_INF_F) M = 0.f;
+  const float ew = expf(lse_w - M), ep = expf(lse_p - M), es = expf(sk - M);
+  const float den = ew + ep + es;
+  const float cw = l > 0.f ? ew / (den * l) : 0.f, cp = den > 0.f ? ep / den : 0.f;
+  float v[NJ];
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    v[j] = cw * o[j];
+    if (p.O_in) v[j] = fmaf(cp, p.O_in[orow * D + li + TPH * j], v[j]);
+  }
+  if (p.inv_rope) {
+    // rotation by -pos of the pairs (d, d + half) of the last rope_dim dims
+    constexpr int JH = 32 / TPH;              // j offset of the partner dim d + 32
+    const int r0 = D - p.rope_dim, half = p.rope_dim / 2;
+    float w[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int d = li + TPH * j;
+      w[j] = v[j];
+      if (d >= r0) {
+        const bool first = d < r0 + half;
+        const int jj = first ? d - r0 : d - r0 - half;
+        const double inv_freq = exp(-2.0 * (double)jj / (double)p.rope_dim * log((double)p.rope_base));
+        const double ang = fmod((double)pos * inv_freq, 6.283185307179586476925286766559);
+        double sd, cd;
+        sincos(ang, &sd, &cd);
+        const float other = first ? v[min(NJ - 1, j + JH)] : v[max(0, j - JH)];
+        w[j] = first ? v[j] * (float)cd + other * (float)sd : v[j] * (float)cd - other * (float)sd;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) v[j] = w[j];
+  }
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int64_t o_i = orow * D + li + TPH * j;
+    if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[o_i] = __float2bfloat16_rn(v[j]);
+    else reinterpret_cast<float*>(p.out)[o_i] = v[j];
+  }
+}
+
+template <int D>
+csa_status_t launch_attn_f32(const AttnParams& p, int epi, cudaStream_t st) {
+  const int64_t items = (int64_t)p.n_seq * p.T * p.n_split;
+  if (items == 0) return CSA_OK;
+  if (items > 0x7fffffff) return fail(CSA_ERR_UNSUPPORTED, "attention (fp32): too many work items");
+  constexpr int TPH = D == 128 ? 8 : 32;
+  // whole warps: heads per CTA rounded up to a multiple of 32 / TPH (masked heads idle)
+  const int per_warp = 32 / TPH;
+  const int HG = std::min(kF32MaxThreads / TPH, (p.H + per_warp - 1) / per_warp * per_warp);
+  const size_t smem = (size_t)kF32Rows * D * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attention (fp32): cannot reserve shared memory: %s", cudaGetErrorString(e));
+  attn_f32_kernel<D><<<dim3((unsigned)items, (unsigned)((p.H + HG - 1) / HG)), HG * TPH, smem, st>>>(p, epi);
+  return check_launch("attention (fp32)");
+}
+
 struct AttnMaps {
   CUtensorMap q, kv, tok;
 };
@@ -1024,6 +1196,8 @@ template <int EPI>
 csa_status_t dispatch(AttnParams& p, int D, csa_dtype_t q_dtype, csa_dtype_t kv_dtype, csa_dtype_t tok_dtype,
                       cudaStream_t st) {
   if (p.n_split < 1) p.n_split = 1;
+  if (q_dtype == CSA_F32 && kv_dtype == CSA_F32 && (p.src2 == SRC2_NONE || tok_dtype == CSA_F32))
+    return D == 512 ? launch_attn_f32<512>(p, EPI, st) : launch_attn_f32<128>(p, EPI, st);
   AttnMaps m;
   csa_status_t s = build_maps(p, m, D, q_dtype, kv_dtype, tok_dtype);
   if (s != CSA_OK) return s;
@@ -1072,7 +1246,7 @@ extern "C" csa_status_t csa_sparse_mqa(const void* q, csa_dtype_t q_dtype, const
   AttnParams p{};
   p.q = q; p.q_f32 = q_dtype == CSA_F32; p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale;
   p.cap = cap; p.src1 = SRC1_GATHER; p.idx = idx; p.k = k; p.m = 1; p.src2 = SRC2_NONE;
-  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = O_part; p.lse_part = lse_part; p.rope_dim = rope_dim;
   return dispatch<EPI_PARTIAL>(p, D, q_dtype, kv_dtype, kv_dtype, stream);
 }
@@ -1090,7 +1264,7 @@ extern "C" csa_status_t hca_dense_attn(const void* q, csa_dtype_t q_dtype, const
   AttnParams p{};
   p.q = q; p.q_f32 = q_dtype == CSA_F32; p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale;
   p.cap = cap; p.q_pos = q_pos; p.src1 = SRC1_DENSE; p.m = m; p.src2 = SRC2_NONE;
-  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = O_part; p.lse_part = lse_part; p.rope_dim = rope_dim;
   return dispatch<EPI_PARTIAL>(p, D, q_dtype, kv_dtype, kv_dtype, stream);
 }
@@ -1115,7 +1289,7 @@ extern "C" csa_status_t swa_sink_combine(const void* q, csa_dtype_t q_dtype, con
   p.q = q; p.q_f32 = q_dtype == CSA_F32; p.q_pos = q_pos;
   p.kv = kv_tok; p.cap = cap; p.src1 = SRC1_NONE; p.m = 1;
   p.kv2 = kv_tok; p.cap2 = cap; p.src2 = window_mode == 0 ? SRC2_WINDOW : SRC2_CACHE; p.W = W;
-  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_in = O_part; p.lse_in = lse_part; p.sink = sink; p.out = out; p.out_bf16 = out_dtype == CSA_BF16;
   p.inv_rope = inv_rope; p.rope_dim = rope_dim; p.rope_base = rope_base;
   return dispatch<EPI_COMBINE>(p, D, q_dtype, kv_dtype, kv_dtype, stream);
@@ -1144,7 +1318,7 @@ extern "C" csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, 
   p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale; p.cap = cap;
   p.src1 = idx ? SRC1_GATHER : SRC1_DENSE; p.idx = idx; p.k = k; p.m = m;
   p.kv2 = kv_tok; p.cap2 = tok_cap; p.src2 = window_mode == 0 ? SRC2_WINDOW : SRC2_CACHE; p.W = W;
-  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f;
   p.sink = sink; p.out = out; p.out_bf16 = out_dtype == CSA_BF16;
   p.inv_rope = inv_rope; p.rope_dim = rope_dim; p.rope_base = rope_base;
   return dispatch<EPI_COMBINE>(p, D, q_dtype, kv_dtype, tok_dtype, stream);
@@ -1190,7 +1364,7 @@ extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q
   p.kv = kv; p.kv_rope = (const __nv_bfloat16*)kv_rope; p.kv_scale = kv_scale; p.cap = cap;
   p.src1 = idx ? SRC1_GATHER : SRC1_DENSE; p.idx = idx; p.k = k; p.m = m;
   p.kv2 = kv_tok; p.cap2 = tok_cap; p.src2 = window_mode == 0 ? SRC2_WINDOW : SRC2_CACHE; p.W = W;
-  p.n_seq = n_seq; p.T = T; p.H = H; p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_seq = n_seq; p.T = T; p.H = H; p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = Os; p.lse_part = Ls; p.rope_dim = rope_dim; p.n_split = n_split;
   p.item_counter = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(Ls) + ((parts * 4 + 255) / 256) * 256);
   cudaError_t ce = cudaMemsetAsync(p.item_counter, 0, sizeof(uint32_t), stream);

@@ -2,8 +2,10 @@
 through the C ABI, returns exactly what csa_index_topk returns with a caller
 workspace, on two calls in a row.  It serves callers that cannot allocate
 device memory; its scratch is a fixed 32 MiB array inside libcsa.so, shared
-by every call, so the second call also checks that stale contents from the
-first do not leak into the result.  Collected last on purpose."""
+by every call, so the second call, whose rows are shorter than the first
+call's (fewer visible entries, more -1 padding), also checks that scores left
+in the array by the first call do not leak into the result.  Collected last on
+purpose."""
 import ctypes
 
 import numpy as np
@@ -38,9 +40,14 @@ def _case(seed, n_seq, T, cap, HI, DI, k, q_pos, grid):
     return cuda(qI), cuda(w), cuda(kI), cuda(ks), cuda(np.asarray(q_pos, np.int64))
 
 
+# q_pos per call: the second call's rows are shorter than the first call's
 @pytest.mark.parametrize("shape", [
-    dict(n_seq=1, T=600, cap=150, HI=64, DI=128, k=64, q_pos=[0], grid=True),          # prefill-like
-    dict(n_seq=3, T=1, cap=40000, HI=64, DI=128, k=512, q_pos=[159999, 70001, 5], grid=False),  # chunked decode
+    dict(n_seq=1, T=600, cap=150, HI=64, DI=128, k=64, q_pos=([0], [0]), grid=True),          # prefill-like
+    dict(n_seq=3, T=1, cap=40000, HI=64, DI=128, k=512, q_pos=([159999, 70001, 5], [159999, 70001, 5]),
+         grid=False),                                                                             # chunked decode
+    dict(n_seq=3, T=1, cap=40000, HI=64, DI=128, k=512, q_pos=([159999, 70001, 4000], [60003, 1000, 2]),
+         grid=False),                                                                             # rows shrink
+    dict(n_seq=1, T=300, cap=150, HI=64, DI=128, k=64, q_pos=([300], [0]), grid=True),        # prefill, shorter
 ])
 def test_noalloc_matches_workspace_entry_point_on_two_calls(shape):
     import long_context_compressed_02_b200 as csa
@@ -50,7 +57,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(shape):
     n_seq, T, k = shape["n_seq"], shape["T"], shape["k"]
     for call in range(2):
         qI, w, kI, ks, pos = _case(100 + call, shape["n_seq"], shape["T"], shape["cap"], shape["HI"],
-                                   shape["DI"], shape["k"], shape["q_pos"], shape["grid"])
+                                   shape["DI"], shape["k"], shape["q_pos"][call], shape["grid"])
         ref = csa.csa_index_topk(qI, w, kI, pos, 4, k, kI_scale=ks)
         got = torch.full((n_seq, T, k), -7, dtype=torch.int32, device="cuda")
         st = fn(ctypes.c_void_p(qI.data_ptr()), None, ctypes.c_void_p(w.data_ptr()), ctypes.c_void_p(kI.data_ptr()),
