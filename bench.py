@@ -280,23 +280,35 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1, n_spli
     torch.cuda.synchronize()
     csa.check_device_error()
     # the decode-time cache writer for the same batch: append one token per
-    # sequence (at a block boundary, so every call emits an e4m3 cache row)
+    # sequence (at a block boundary, so every call emits an e4m3 KV row and the
+    # block's e4m3 indexer key)
     m_c = 4
     ring_C = torch.zeros(Bn, 2 * m_c, D, dtype=torch.bfloat16, device=dev)
     ring_Z = torch.zeros_like(ring_C)
+    ring_CI = torch.zeros(Bn, 2 * m_c, DI, dtype=torch.bfloat16, device=dev)
+    ring_ZI = torch.zeros_like(ring_CI)
     c_tok = torch.randn(Bn, D, device=dev).to(torch.bfloat16)
     z_tok = torch.randn(Bn, D, device=dev).to(torch.bfloat16)
+    ci_tok = torch.randn(Bn, DI, device=dev).to(torch.bfloat16)
+    zi_tok = torch.randn(Bn, DI, device=dev).to(torch.bfloat16)
     B_c = torch.zeros(2 * m_c, D, device=dev)
+    B_i = torch.zeros(2 * m_c, DI, device=dev)
     pos_c = torch.full((Bn,), 4 * 1000 - 1, dtype=torch.int64, device=dev)
     row_nope = torch.empty(Bn, 1024, D - 64, dtype=torch.uint8, device=dev)
     row_rope = torch.empty(Bn, 1024, 64, dtype=torch.bfloat16, device=dev)
     row_scale = torch.empty(Bn, 1024, device=dev)
+    key_codes = torch.empty(Bn, 1024, DI, dtype=torch.uint8, device=dev)
+    key_scale = torch.empty(Bn, 1024, device=dev)
+
+    def append():
+        csa.csa_cache_append(c_tok, z_tok, B_c, m_c, True, pos_c, ring_C, ring_Z, row_nope, row_rope, row_scale,
+                             ci_tok, zi_tok, B_i, ring_CI, ring_ZI, key_codes, key_scale)
     for _ in range(3):
-        csa.csa_compress_append(c_tok, z_tok, B_c, m_c, True, pos_c, ring_C, ring_Z, row_nope, row_rope, row_scale)
+        append()
     wa, wb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     wa.record(stream)
     for _ in range(steps):
-        csa.csa_compress_append(c_tok, z_tok, B_c, m_c, True, pos_c, ring_C, ring_Z, row_nope, row_rope, row_scale)
+        append()
     wb.record(stream)
     torch.cuda.synchronize()
     csa.check_device_error()
@@ -320,8 +332,9 @@ def decode_leg(dev, steps, warmup, csa, synth, torch, batch=None, seed=1, n_spli
                                                                                  "fused_attention": t_att},
             "algorithmic_bytes_per_step": algo,
             "cache_append": {"ms": t_app, "rows_per_call": Bn,
-                             "note": "new token appended to the 2m-token ring, block entry pooled, normalised, "
-                                     "rotated and written as an e4m3 cache row (not part of ms_per_step)"},
+                             "note": "new token appended to the 2m-token rings, the block's KV entry pooled, "
+                                     "normalised, rotated and written as an e4m3 cache row, and its indexer key "
+                                     "pooled and written as an e4m3 key row, one launch (not part of ms_per_step)"},
             "hbm_frac_step": algo / (ms * 1e-3) / 1e9 / hbm,
             "roofline": {"kernel": "index_topk", "bound": "hbm", "achieved": ach_idx, "peak": hbm, "unit": "GB/s",
                          "frac": ach_idx / hbm,

@@ -71,6 +71,15 @@ const char* csa_get_last_error_string(void);
  * recorded an expired wait or a bad gather index since the last check. */
 csa_status_t csa_check_device_error(cudaStream_t stream);
 
+/* Self-test of the failure path (no counterpart on the pages): launches one
+ * thread that waits, through the same bounded on-chip wait the kernels use, on
+ * a barrier phase that nothing completes, with a limit of limit_ns (1 us to
+ * 100 ms) instead of the kernels' 2 s.  The wait expires, the expiry is
+ * recorded in the device error word and the kernel returns, so the next
+ * csa_check_device_error on the stream reports CSA_ERR_TIMEOUT and the context
+ * stays usable.  No memory is touched besides the error word. */
+csa_status_t csa_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------------
  * csa_compress — softmax-gated KV compressor ([CS] "KV 压缩": an entry is the
  * per-channel Softmax(Z + B)-weighted sum of the content C over its block; CSA
@@ -138,6 +147,28 @@ csa_status_t csa_compress_append(const void* c_tok, const void* z_tok, csa_dtype
                                  int n_seq, int D, int m, int overlap, const int64_t* q_pos, void* ring_C,
                                  void* ring_Z, uint8_t* kv_nope, void* kv_rope, float* kv_scale, int64_t cap,
                                  int norm, int rope_dim, float rope_base, float eps, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * csa_cache_append — the whole decode-time cache write of a CSA layer in one
+ * launch: the KV row as csa_compress_append (norm on) AND the lightning
+ * indexer's key of the same block ([CS] "闪电索引器": the indexer scores the
+ * compressed entries, so each entry has an index key; "KV 压缩": entries are
+ * pooled block by block).  Reading taken where the pages are silent: the key
+ * is pooled by the same per-channel softmax over its own stream (ci_tok,
+ * zi_tok [n_seq, DI], bias B_I [2m or m, DI] fp32, ring_CI / ring_ZI
+ * [n_seq, 2m, DI]) with no RMSNorm and no RoPE, and stored like a KV row with
+ * rope_dim 0:  kI[b, i, :] = e4m3(key / s_I), kI_scale[b, i] = s_I =
+ * max|key| / 448 (1 for an all-zero key) -- the layout csa_index_topk reads.
+ * Other arguments, requirements and the ring contract are those of
+ * csa_compress_append; DI a multiple of 16 in [16, 2048].  Grid: one CTA per
+ * (sequence, stream).
+ * ------------------------------------------------------------------------- */
+csa_status_t csa_cache_append(const void* c_tok, const void* z_tok, csa_dtype_t in_dtype, const float* B, int n_seq,
+                              int D, int m, int overlap, const int64_t* q_pos, void* ring_C, void* ring_Z,
+                              uint8_t* kv_nope, void* kv_rope, float* kv_scale, int64_t cap, int rope_dim,
+                              float rope_base, float eps, const void* ci_tok, const void* zi_tok, const float* B_I,
+                              int DI, void* ring_CI, void* ring_ZI, uint8_t* kI, float* kI_scale,
+                              cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * csa_index_topk — lightning indexer + top-k ([CS] "闪电索引器": index heads,

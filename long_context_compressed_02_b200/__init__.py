@@ -8,6 +8,7 @@ fails, an exception is raised.
 Entry points (same names as the C ABI):
   csa_compress, csa_compress_append, csa_rmsnorm_rope, csa_index_topk,
   csa_sparse_mqa, hca_dense_attn, swa_sink_combine, csa_fused_attention,
+  csa_fused_attention_splitkv (n_split > 1), csa_index_topk_fp4, csa_cache_append,
   csa_grouped_out_proj
 and compositions of them: csa_layer_prefill, hca_layer_prefill,
 swa_layer_prefill, csa_layer_decode, hca_layer_decode, swa_layer_decode.
@@ -64,6 +65,8 @@ def lib():
         "csa_grouped_out_proj": ([P, P, P, I, I, I, I, I, I, P, P, I, P], I),
         "csa_get_last_error_string": ([], ctypes.c_char_p),
         "csa_workspace_size": ([I, I, I64, I, I, I, I], SZ),
+        "csa_selftest_wait_timeout": ([ctypes.c_uint64, P], I),
+        "csa_cache_append": ([P, P, I, P, I, I, I, I, P, P, P, P, P, P, I64, I, F, F, P, P, P, I, P, P, P, P, P], I),
         "csa_index_topk_fp4_workspace": ([I, I, I, I64, I], SZ),
         "csa_index_topk_fp4": ([P, P, P, P, P, P, I, I, I, I64, I, I, P, P, SZ, P], I),
     }
@@ -106,6 +109,12 @@ def num_sms(device=None):
 
 def csa_fused_attention_workspace(n_seq, T, H, D, n_split):
     return int(lib().csa_fused_attention_workspace(n_seq, T, H, D, n_split))
+
+
+def selftest_wait_timeout(limit_ns=1_000_000, stream=None):
+    """Launches the bounded-wait self-test (a wait that nothing completes,
+    limit limit_ns); the next check_device_error reports the expiry."""
+    _check(lib().csa_selftest_wait_timeout(int(limit_ns), _stream(stream)), "csa_selftest_wait_timeout")
 
 
 def check_device_error(stream=None):
@@ -152,6 +161,33 @@ def csa_compress_append(c_tok, z_tok, B, m, overlap, q_pos, ring_C, ring_Z, kv_n
                                      _ptr(q_pos), _ptr(ring_C), _ptr(ring_Z), _ptr(kv_nope), _ptr(kv_rope),
                                      _ptr(kv_scale), kv_nope.shape[1], int(norm), rope_dim, rope_base, eps,
                                      _stream(stream)), "csa_compress_append")
+
+
+def csa_cache_append(c_tok, z_tok, B, m, overlap, q_pos, ring_C, ring_Z, kv_nope, kv_rope, kv_scale,
+                     ci_tok, zi_tok, B_I, ring_CI, ring_ZI, kI, kI_scale, *, rope_dim=64, rope_base=10000.0,
+                     eps=1e-6, stream=None):
+    """Decode-time cache write of a CSA layer in one launch: the KV row (as
+    csa_compress_append with norm on) and the indexer key of the same block,
+    pooled from its own stream (ci_tok, zi_tok [n_seq, DI], B_I, rings
+    [n_seq, 2m, DI]) and stored as e4m3 kI [n_seq, cap, DI] + kI_scale [n_seq, cap]."""
+    for t, n in ((c_tok, "c_tok"), (z_tok, "z_tok"), (B, "B"), (q_pos, "q_pos"), (ring_C, "ring_C"),
+                 (ring_Z, "ring_Z"), (kv_nope, "kv_nope"), (kv_rope, "kv_rope"), (kv_scale, "kv_scale"),
+                 (ci_tok, "ci_tok"), (zi_tok, "zi_tok"), (B_I, "B_I"), (ring_CI, "ring_CI"), (ring_ZI, "ring_ZI"),
+                 (kI, "kI"), (kI_scale, "kI_scale")):
+        _dev(t, n)
+    n_seq, D = c_tok.shape
+    DI = ci_tok.shape[1]
+    cap = kv_nope.shape[1]
+    if tuple(ring_C.shape) != (n_seq, 2 * m, D) or tuple(ring_CI.shape) != (n_seq, 2 * m, DI) or \
+            tuple(kI.shape) != (n_seq, cap, DI) or tuple(kI_scale.shape) != (n_seq, cap) or \
+            ci_tok.dtype != c_tok.dtype or ring_CI.dtype != c_tok.dtype or ring_C.dtype != c_tok.dtype:
+        raise CsaError("csa_cache_append: rings [n_seq, 2m, D|DI], kI [n_seq, cap, DI], kI_scale [n_seq, cap] of "
+                       "the token dtype expected")
+    _check(lib().csa_cache_append(_ptr(c_tok), _ptr(z_tok), _DT[c_tok.dtype], _ptr(B), n_seq, D, m, int(overlap),
+                                  _ptr(q_pos), _ptr(ring_C), _ptr(ring_Z), _ptr(kv_nope), _ptr(kv_rope),
+                                  _ptr(kv_scale), cap, rope_dim, rope_base, eps, _ptr(ci_tok), _ptr(zi_tok),
+                                  _ptr(B_I), DI, _ptr(ring_CI), _ptr(ring_ZI), _ptr(kI), _ptr(kI_scale),
+                                  _stream(stream)), "csa_cache_append")
 
 
 def csa_rmsnorm_rope(x, rows_per_pos=1, pos0=0, *, norm=True, rope_dim=64, rope_base=10000.0, eps=1e-6,

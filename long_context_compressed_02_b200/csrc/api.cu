@@ -1,6 +1,8 @@
-// Status reporting shared by all entry points of libcsa.so.
+// Status reporting shared by all entry points of libcsa.so, and the self-test
+// of the bounded on-chip waits.
 #include <string>
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace csa {
 
@@ -17,6 +19,25 @@ csa_status_t fail(csa_status_t s, const char* fmt, ...) {
 }
 
 void clear_error() { g_last_error.clear(); }
+
+static __device__ uint32_t g_err_selftest;
+
+uint32_t read_clear_err_selftest() {
+  uint32_t v = 0, z = 0;
+  cudaMemcpyFromSymbol(&v, g_err_selftest, sizeof(v));
+  cudaMemcpyToSymbol(g_err_selftest, &z, sizeof(z));
+  return v;
+}
+
+// One thread waits on an mbarrier phase that nothing completes, through the
+// same bounded wait the kernels use, with the given limit; the expiry is
+// recorded in the device error word and the kernel returns.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0, &g_err_selftest, limit_ns);
+}
 
 }  // namespace csa
 
@@ -50,8 +71,15 @@ extern "C" csa_status_t csa_check_device_error(cudaStream_t stream) {
   if (e != cudaSuccess)
     return csa::fail(CSA_ERR_CUDA, "csa_check_device_error: stream sync failed: %s", cudaGetErrorString(e));
   uint32_t w = csa::read_clear_err_indexer() | csa::read_clear_err_attention() | csa::read_clear_err_proj() |
-               csa::read_clear_err_compress();
+               csa::read_clear_err_compress() | csa::read_clear_err_selftest();
   if (w & 1u) return csa::fail(CSA_ERR_TIMEOUT, "a bounded on-chip wait expired (device error word 0x%x)", w);
   if (w) return csa::fail(CSA_ERR_DEVICE, "a kernel recorded an out-of-range gather index (device error word 0x%x)", w);
   return CSA_OK;
+}
+
+extern "C" csa_status_t csa_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
+  csa::clear_error();
+  CSA_REQUIRE(limit_ns >= 1000 && limit_ns <= 100000000ull, "csa_selftest_wait_timeout: limit_ns must be in [1 us, 100 ms]");
+  csa::selftest_wait_kernel<<<1, 1, 0, stream>>>(limit_ns);
+  return csa::check_launch("csa_selftest_wait_timeout");
 }

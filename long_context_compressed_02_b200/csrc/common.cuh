@@ -33,6 +33,7 @@ uint32_t read_clear_err_indexer();
 uint32_t read_clear_err_attention();
 uint32_t read_clear_err_proj();
 uint32_t read_clear_err_compress();
+uint32_t read_clear_err_selftest();
 
 }  // namespace csa
 

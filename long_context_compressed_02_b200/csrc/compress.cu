@@ -525,14 +525,47 @@ __device__ __forceinline__ float block_reduce(float v, float* s_red) {
 // previous one when overlapping), RMS-normalised, rotated at position i * m,
 // and written as cache row i: the first D - rope_dim dims as e4m3 codes under
 // the row scale amax / 448, the RoPE dims as bf16, the scale as fp32.
+// One pooled stream of the writer: the KV cache (RMSNorm + RoPE, e4m3 + bf16
+// RoPE dims) or the indexer key cache (no norm or RoPE, all dims e4m3).
+struct AppendStream {
+  const void* c_tok;
+  const void* z_tok;
+  const float* B;
+  void* ring_C;
+  void* ring_Z;
+  uint8_t* kv_nope;
+  __nv_bfloat16* kv_rope;
+  float* kv_scale;
+  int D, norm, rope_dim;
+  double ratio;
+};
+struct AppendParams {
+  AppendStream st[2];       // blockIdx.y selects the stream
+  const int64_t* q_pos;
+  int m, overlap;
+  int64_t cap;
+  float eps;
+};
+
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads)
-compress_append_kernel(const Tin* __restrict__ c_tok, const Tin* __restrict__ z_tok, const float* __restrict__ B,
-                       int D, int m, int overlap, const int64_t* __restrict__ q_pos, Tin* __restrict__ ring_C,
-                       Tin* __restrict__ ring_Z, uint8_t* __restrict__ kv_nope, __nv_bfloat16* __restrict__ kv_rope,
-                       float* __restrict__ kv_scale, int64_t cap, int norm, int rope_dim, double ratio, float eps) {
+compress_append_kernel(const __grid_constant__ AppendParams P) {
   extern __shared__ float s_row[];          // [D] the pooled entry
   __shared__ float s_red[kThreads / 32];
+  const AppendStream& S = P.st[blockIdx.y];
+  const Tin* __restrict__ c_tok = static_cast<const Tin*>(S.c_tok);
+  const Tin* __restrict__ z_tok = static_cast<const Tin*>(S.z_tok);
+  const float* __restrict__ B = S.B;
+  Tin* __restrict__ ring_C = static_cast<Tin*>(S.ring_C);
+  Tin* __restrict__ ring_Z = static_cast<Tin*>(S.ring_Z);
+  uint8_t* __restrict__ kv_nope = S.kv_nope;
+  __nv_bfloat16* __restrict__ kv_rope = S.kv_rope;
+  float* __restrict__ kv_scale = S.kv_scale;
+  const int D = S.D, norm = S.norm, rope_dim = S.rope_dim, m = P.m, overlap = P.overlap;
+  const int64_t* __restrict__ q_pos = P.q_pos;
+  const int64_t cap = P.cap;
+  const double ratio = S.ratio;
+  const float eps = P.eps;
   const int b = blockIdx.x, tid = threadIdx.x;
   const int64_t pos = q_pos[b];
   const int L = 2 * m;
@@ -659,6 +692,16 @@ csa_status_t launch_norm(const void* x, int64_t rows, int D, int rpp, int64_t po
   return check_launch("csa_rmsnorm_rope");
 }
 
+csa_status_t launch_append(const AppendParams& P, csa_dtype_t in_dtype, int n_seq, int n_streams, cudaStream_t st,
+                           const char* what) {
+  const int dmax = n_streams > 1 ? std::max(P.st[0].D, P.st[1].D) : P.st[0].D;
+  const size_t smem = (size_t)dmax * sizeof(float);
+  const dim3 grid((unsigned)n_seq, (unsigned)n_streams);
+  if (in_dtype == CSA_F32) compress_append_kernel<float><<<grid, kThreads, smem, st>>>(P);
+  else compress_append_kernel<__nv_bfloat16><<<grid, kThreads, smem, st>>>(P);
+  return check_launch(what);
+}
+
 }  // namespace
 }  // namespace csa
 
@@ -735,16 +778,39 @@ extern "C" csa_status_t csa_compress_append(const void* c_tok, const void* z_tok
   CSA_REQUIRE(aligned16(c_tok) && aligned16(z_tok) && aligned16(B) && aligned16(q_pos) && aligned16(ring_C) &&
               aligned16(ring_Z) && aligned16(kv_nope) && aligned16(kv_scale) && (!kv_rope || aligned16(kv_rope)),
               "csa_compress_append: pointers must be 16-byte aligned");
-  const double ratio = rope_dim > 0 ? std::pow((double)rope_base, -2.0 / (double)rope_dim) : 1.0;
-  const size_t smem = (size_t)D * sizeof(float);
-  if (in_dtype == CSA_F32) {
-    compress_append_kernel<float><<<n_seq, kThreads, smem, stream>>>(
-        (const float*)c_tok, (const float*)z_tok, B, D, m, overlap, q_pos, (float*)ring_C, (float*)ring_Z, kv_nope,
-        (__nv_bfloat16*)kv_rope, kv_scale, cap, norm, rope_dim, ratio, eps);
-  } else {
-    compress_append_kernel<__nv_bfloat16><<<n_seq, kThreads, smem, stream>>>(
-        (const __nv_bfloat16*)c_tok, (const __nv_bfloat16*)z_tok, B, D, m, overlap, q_pos, (__nv_bfloat16*)ring_C,
-        (__nv_bfloat16*)ring_Z, kv_nope, (__nv_bfloat16*)kv_rope, kv_scale, cap, norm, rope_dim, ratio, eps);
-  }
-  return check_launch("csa_compress_append");
+  AppendParams P{};
+  P.st[0] = AppendStream{c_tok, z_tok, B, ring_C, ring_Z, kv_nope, (__nv_bfloat16*)kv_rope, kv_scale, D, norm, rope_dim,
+                         rope_dim > 0 ? std::pow((double)rope_base, -2.0 / (double)rope_dim) : 1.0};
+  P.q_pos = q_pos; P.m = m; P.overlap = overlap; P.cap = cap; P.eps = eps;
+  return launch_append(P, in_dtype, n_seq, 1, stream, "csa_compress_append");
+}
+
+extern "C" csa_status_t csa_cache_append(const void* c_tok, const void* z_tok, csa_dtype_t in_dtype, const float* B,
+                                         int n_seq, int D, int m, int overlap, const int64_t* q_pos, void* ring_C,
+                                         void* ring_Z, uint8_t* kv_nope, void* kv_rope, float* kv_scale, int64_t cap,
+                                         int rope_dim, float rope_base, float eps, const void* ci_tok,
+                                         const void* zi_tok, const float* B_I, int DI, void* ring_CI, void* ring_ZI,
+                                         uint8_t* kI, float* kI_scale, cudaStream_t stream) {
+  clear_error();
+  CSA_REQUIRE(n_seq >= 0 && cap >= 1, "csa_cache_append: n_seq >= 0 and cap >= 1 required");
+  CSA_REQUIRE(D % 8 == 0 && D >= 64 && D <= 2048, "csa_cache_append: D must be a multiple of 8 in [64, 2048]");
+  CSA_REQUIRE(DI % 16 == 0 && DI >= 16 && DI <= 2048, "csa_cache_append: DI must be a multiple of 16 in [16, 2048]");
+  CSA_REQUIRE(m >= 1 && m <= 1024, "csa_cache_append: m must be in [1, 1024]");
+  CSA_REQUIRE(overlap == 0 || overlap == 1, "csa_cache_append: overlap must be 0 or 1");
+  CSA_REQUIRE(rope_dim == 0 || (rope_dim == 64 && D > 64), "csa_cache_append: rope_dim must be 0 or 64 (< D)");
+  CSA_REQUIRE(in_dtype == CSA_F32 || in_dtype == CSA_BF16, "csa_cache_append: in_dtype must be F32 or BF16");
+  if (n_seq == 0) return CSA_OK;
+  CSA_REQUIRE(c_tok && z_tok && B && q_pos && ring_C && ring_Z && kv_nope && kv_scale && (rope_dim == 0 || kv_rope) &&
+              ci_tok && zi_tok && B_I && ring_CI && ring_ZI && kI && kI_scale, "csa_cache_append: null pointer");
+  CSA_REQUIRE(aligned16(c_tok) && aligned16(z_tok) && aligned16(B) && aligned16(q_pos) && aligned16(ring_C) &&
+              aligned16(ring_Z) && aligned16(kv_nope) && aligned16(kv_scale) && (!kv_rope || aligned16(kv_rope)) &&
+              aligned16(ci_tok) && aligned16(zi_tok) && aligned16(B_I) && aligned16(ring_CI) && aligned16(ring_ZI) &&
+              aligned16(kI) && aligned16(kI_scale), "csa_cache_append: pointers must be 16-byte aligned");
+  AppendParams P{};
+  P.st[0] = AppendStream{c_tok, z_tok, B, ring_C, ring_Z, kv_nope, (__nv_bfloat16*)kv_rope, kv_scale, D, 1, rope_dim,
+                         rope_dim > 0 ? std::pow((double)rope_base, -2.0 / (double)rope_dim) : 1.0};
+  // the indexer key: the same pooling over its own stream, no norm or RoPE
+  P.st[1] = AppendStream{ci_tok, zi_tok, B_I, ring_CI, ring_ZI, kI, nullptr, kI_scale, DI, 0, 0, 1.0};
+  P.q_pos = q_pos; P.m = m; P.overlap = overlap; P.cap = cap; P.eps = eps;
+  return launch_append(P, in_dtype, n_seq, 2, stream, "csa_cache_append");
 }

@@ -907,6 +907,7 @@ topk_merge_kernel(TopkParams p) {
 struct WsLayout {
   size_t scores, cand_key, cand_idx, cand_cnt, hist, counter, total;
   int n_chunks;
+  bool ok;                 // false: the sizes overflow size_t (total is then 0)
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -915,8 +916,17 @@ WsLayout ws_layout(int n_seq, int T, int64_t cap, int k) {
   WsLayout L{};
   const size_t rows = (size_t)n_seq * (size_t)T;
   L.n_chunks = (int)((cap + kChunk - 1) / kChunk);
+  // the score matrix dominates; every later term is smaller than it, so one
+  // overflow-checked product bounds the whole layout
+  size_t score_bytes = 0;
+  if (__builtin_mul_overflow(rows, (size_t)cap, &score_bytes) ||
+      __builtin_mul_overflow(score_bytes, (size_t)4, &score_bytes) || score_bytes > (SIZE_MAX >> 2)) {
+    L.ok = false;
+    return L;
+  }
+  L.ok = true;
   size_t off = 0;
-  L.scores = off; off = align_up(off + rows * (size_t)cap * 4, 256);
+  L.scores = off; off = align_up(off + score_bytes, 256);
   if (L.n_chunks > 1) {
     L.cand_key = off; off = align_up(off + rows * L.n_chunks * (size_t)k * 4, 256);
     L.cand_idx = off; off = align_up(off + rows * L.n_chunks * (size_t)k * 4, 256);
@@ -935,7 +945,7 @@ using namespace csa;
 
 extern "C" size_t csa_index_topk_workspace(int n_seq, int T, int64_t cap, int k) {
   if (n_seq <= 0 || T <= 0 || cap <= 0 || k <= 0) return 0;
-  return ws_layout(n_seq, T, cap, k).total;
+  return ws_layout(n_seq, T, cap, k).total;   // 0 when the sizes overflow
 }
 
 namespace csa {
@@ -1063,6 +1073,8 @@ extern "C" csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale,
   CSA_REQUIRE((int64_t)n_seq * cap < (int64_t)1 << 31 && (int64_t)n_seq * T * HI < (int64_t)1 << 31,
               "csa_index_topk: tensor too large for 32-bit TMA coordinates");
   const WsLayout L = ws_layout(n_seq, T, cap, k);
+  if (!L.ok)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: n_seq * T * cap * 4 bytes of scores overflow size_t");
   if (!workspace || ws_bytes < L.total)
     return fail(CSA_ERR_WORKSPACE, "csa_index_topk: workspace of %zu bytes needed, %zu given", L.total, ws_bytes);
   CSA_REQUIRE(aligned16(workspace), "csa_index_topk: workspace must be 16-byte aligned");
@@ -1084,7 +1096,8 @@ inline size_t fp4_query_bytes(int n_seq, int T, int HI) {
 
 extern "C" size_t csa_index_topk_fp4_workspace(int n_seq, int T, int HI, int64_t cap, int k) {
   if (n_seq <= 0 || T <= 0 || HI <= 0 || cap <= 0 || k <= 0) return 0;
-  return ws_layout(n_seq, T, cap, k).total + fp4_query_bytes(n_seq, T, HI);
+  const WsLayout L = ws_layout(n_seq, T, cap, k);
+  return L.ok ? L.total + fp4_query_bytes(n_seq, T, HI) : 0;
 }
 
 extern "C" csa_status_t csa_index_topk_fp4(const uint8_t* qI4, const uint8_t* qI4_scale, const float* w,
@@ -1102,6 +1115,8 @@ extern "C" csa_status_t csa_index_topk_fp4(const uint8_t* qI4, const uint8_t* qI
   CSA_REQUIRE((int64_t)n_seq * cap < (int64_t)1 << 31 && (int64_t)n_seq * T * HI < (int64_t)1 << 31,
               "csa_index_topk_fp4: tensor too large for 32-bit TMA coordinates");
   const WsLayout L = ws_layout(n_seq, T, cap, k);
+  if (!L.ok)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk_fp4: n_seq * T * cap * 4 bytes of scores overflow size_t");
   const size_t need = L.total + fp4_query_bytes(n_seq, T, HI);
   if (!workspace || ws_bytes < need)
     return fail(CSA_ERR_WORKSPACE, "csa_index_topk_fp4: workspace of %zu bytes needed, %zu given", need, ws_bytes);
@@ -1129,9 +1144,41 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB, held by every GPU that loads the library
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
+// The array's device address, looked up per CUDA context: a context created
+// after cudaDeviceReset, or a driver-API context other than the device's
+// primary one, loads the module again at another address.  Contexts are told
+// apart by their unique id (cuCtxGetId), which is never reused.
+struct NoAllocAddr {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+constexpr int kMaxContexts = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+NoAllocAddr g_noalloc_addr[kMaxContexts] = {};
+int g_noalloc_n = 0;
+
+typedef CUresult (*PFN_ctx_get_current)(CUcontext*);
+typedef CUresult (*PFN_ctx_get_id)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(p);
+}
+
+// Id of the calling thread's current context (0 if there is none yet).
+bool current_ctx_id(unsigned long long* id) {
+  static PFN_ctx_get_current get_cur = driver_fn<PFN_ctx_get_current>("cuCtxGetCurrent");
+  static PFN_ctx_get_id get_id = driver_fn<PFN_ctx_get_id>("cuCtxGetId");
+  if (!get_cur || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS) return false;
+  *id = 0;
+  return ctx == nullptr || get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 }  // namespace
 }  // namespace csa
@@ -1144,7 +1191,7 @@ extern "C" csa_status_t csa_index_topk_noalloc(const uint8_t* qI, const float* q
   CSA_REQUIRE(n_seq >= 1 && T >= 1 && cap >= 1 && k >= 1,
               "csa_index_topk_noalloc: n_seq, T, cap and k must be >= 1");
   const size_t need = csa_index_topk_workspace(n_seq, T, cap, k);
-  if (need > kNoAllocScratchBytes)
+  if (need == 0 || need > kNoAllocScratchBytes)
     return fail(CSA_ERR_UNSUPPORTED,
                 "csa_index_topk_noalloc: this call needs %zu bytes of scratch but the built-in array holds %zu "
                 "(n_seq * T * cap * 4 bytes of scores must fit); use csa_index_topk with a workspace",
@@ -1152,20 +1199,26 @@ extern "C" csa_status_t csa_index_topk_noalloc(const uint8_t* qI, const float* q
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_index_topk_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk_noalloc: device %d out of range", dev);
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    unsigned long long ctx = 0;
+    if (!current_ctx_id(&ctx))
+      return fail(CSA_ERR_CUDA, "csa_index_topk_noalloc: cannot identify the current CUDA context");
+    for (int i = 0; i < g_noalloc_n && ctx != 0; ++i)
+      if (g_noalloc_addr[i].ctx_id == ctx) scratch = g_noalloc_addr[i].ptr;
+    if (!scratch) {
       // Host code only sees a stand-in for the array: its device address is
-      // looked up once per device, with that device current.
-      void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      // looked up once per context, with the caller's device current (the
+      // lookup also creates the device's primary context if there is none).
+      e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
       if (e != cudaSuccess)
         return fail(CSA_ERR_CUDA, "csa_index_topk_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-      g_noalloc_ptr[dev] = p;
+      if ((ctx != 0 || current_ctx_id(&ctx)) && ctx != 0) {
+        if (g_noalloc_n < kMaxContexts) g_noalloc_addr[g_noalloc_n++] = {ctx, scratch};
+        else g_noalloc_addr[ctx % kMaxContexts] = {ctx, scratch};
+      }
     }
-    scratch = g_noalloc_ptr[dev];
   }
   return csa_index_topk(qI, qI_scale, w, kI, kI_scale, q_pos, n_seq, T, HI, DI, cap, m, k, idx, scratch,
                         kNoAllocScratchBytes, stream);

@@ -56,14 +56,15 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                          uint64_t limit_ns = kWaitNs) {
   uint64_t start = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0) {
       const uint64_t now = global_ns();
       if (start == 0) start = now;
-      else if (now - start > kWaitNs) break;
+      else if (now - start > limit_ns) break;
     }
   }
   if (err) atomicOr(err, DEV_ERR_TIMEOUT_MBAR);

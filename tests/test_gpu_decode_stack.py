@@ -66,7 +66,7 @@ def _check_layer(lay, res, b, t, k, W, D, what):
     assert_close(host(out)[b, 0], ref, what=what)
 
 
-@pytest.mark.parametrize("n_split", [(1, 1), (4, 16)])
+@pytest.mark.parametrize("n_split", [(1, 1), (4, 16), (8, 8)])
 def test_mixed_stack_small_contexts(n_split):
     """Four sequences with short, unequal contexts (one below top-k entries,
     one below a single HCA entry's worth of window): every sequence, every layer."""

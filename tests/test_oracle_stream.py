@@ -73,3 +73,28 @@ def test_fp8_row_quantize_definition():
     assert np.array_equal(rope, O.bf16_round(x[:, 448:]))
     z_codes, _, z_scale = O.fp8_row_quantize(np.zeros((1, 512)), 64)
     assert z_scale[0] == 1.0 and not z_codes.any()
+
+
+def test_index_key_stream_equals_batch_and_quantises_whole_row():
+    """The indexer key of each block ([CS] "闪电索引器" scores compressed
+    entries; reading taken: the key is pooled by the same per-channel softmax
+    over its own (C_I, Z_I) stream, with no norm or RoPE) streamed one token at
+    a time equals the batch compressor of that stream, and its e4m3 row has no
+    bf16 part: every dim is a code under the row scale amax / 448."""
+    rng = np.random.default_rng(14)
+    m, DI, S = 4, 128, 45
+    CI, ZI = rng.standard_normal((S, DI)), rng.standard_normal((S, DI))
+    BI = 0.1 * rng.standard_normal((2 * m, DI))
+    ref = O.compress(CI, ZI, BI, m, True)
+    ring_c, ring_z = np.zeros((2 * m, DI)), np.zeros((2 * m, DI))
+    for t in range(S):
+        r = O.stream_append(ring_c, ring_z, CI[t], ZI[t], t, BI, m, True, norm_rope=False)
+        if r is None:
+            continue
+        i, key = r
+        assert np.array_equal(key, ref[i])
+        codes, rope, scale = O.fp8_row_quantize(key, 0)
+        assert codes.shape == (DI,) and rope.shape == (0,)
+        assert scale == np.abs(key).max() / 448.0
+        deq = O.e4m3_decode(codes) * scale
+        assert np.all(np.abs(deq - key) <= np.maximum(np.abs(key) * 2.0 ** -4, scale * 2.0 ** -10) * (1 + 1e-12))
