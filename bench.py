@@ -409,7 +409,7 @@ def mixed_decode_leg(dev, steps, warmup, csa, synth, torch, seed=0, split=None):
     # split-KV ranges per sequence (items are claimed dynamically, so unequal
     # sequence lengths balance across CTAs)
     if split is None:
-        split = {"csa": max(1, min(9, sms // Bn)), "hca": 16}
+        split = {"csa": max(1, min(9, sms // Bn)), "hca": 12}
     bufs = []
     for lay in layers:
         b = {"out": torch.empty(Bn, 1, H, D, dtype=torch.bfloat16, device=dev)}

@@ -335,9 +335,13 @@ csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, const void*
  * in parallel (more CTAs when there are few query tokens, e.g. decode), followed
  * by a merge of the n_split partial results and the sink in one softmax and the
  * optional inverse RoPE.  Same result as csa_fused_attention up to rounding.
- * CTAs claim (token, range) items from a counter in the workspace, so ranges of
- * unequal length (sequences of unequal context) balance across the GPU.
- *   n_split in [1, 16]; workspace of csa_fused_attention_workspace(n_seq, T, H, D,
+ * Every token's rows are cut into ranges of one common length: the longest
+ * possible row set (k gathered or cap dense entries, plus the window) divided
+ * by n_split, so a short token takes fewer, fuller ranges and its remaining
+ * ranges are empty (lse -inf, output not written, skipped by the merge).  CTAs
+ * claim (token, range) items from a counter in the workspace, so ranges of
+ * sequences of unequal context balance across the GPU.
+ *   n_split in [1, 32]; workspace of csa_fused_attention_workspace(n_seq, T, H, D,
  *   n_split) bytes, 16-byte aligned, owned by the caller (partials: fp32
  *   [n_seq*T*n_split, H, D] + lse, then the item counter, reset by the call with a
  *   stream-ordered memset); calls sharing one workspace must be ordered on one

@@ -69,6 +69,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 enum KvKind { KV_BF16 = 0, KV_F32 = 1, KV_FP8 = 2 };
 enum EpiMode { EPI_PARTIAL = 0, EPI_COMBINE = 1 };
+constexpr int kMaxSplit = 32;      // ranges per query token in split-KV calls
 // Row set of a query token: source 1 (compressed entries: a gathered top-k
 // list or the dense prefix of complete entries) followed by source 2 (raw
 // window rows).  Either may be absent.  All rows share one softmax.
@@ -104,6 +105,8 @@ struct AttnParams {
   float rope_base;
   int tma_q, tma_kv, tma_tok;   // TMA tile loads for bf16 queries / dense entries / window rows
   int n_split;                  // ranges of half chunks per query token (partials merged afterwards)
+  int per_item;                 // > 0: half chunks per range, the same for every token (ranges past a
+                                // token's rows are empty); 0: each token's rows cut into n_split ranges
   uint32_t* item_counter;       // non-null: items are claimed dynamically from this zeroed counter
 };
 
@@ -158,7 +161,7 @@ __device__ __forceinline__ RowSet row_set_warp(const AttnParams& p, int b, int t
   r.n = r.n1 + r.n2;
   r.nh2 = (r.n2 + kRows - 1) / kRows;
   r.nh = r.nh2 + (r.n1 + kRows - 1) / kRows;
-  const int per = (r.nh + p.n_split - 1) / p.n_split;
+  const int per = p.per_item > 0 ? p.per_item : (r.nh + p.n_split - 1) / p.n_split;
   r.c0 = min(r.nh, sp * per);
   r.c1 = min(r.nh, r.c0 + per);
   return r;
@@ -827,7 +830,11 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
       // last tile's upper half: those 64 threads exchange through shared memory.
       const int64_t obase = (bt * p.n_split + sp) * p.H;   // n_split = 1: token row
       float* xs = reinterpret_cast<float*>(sP);            // [64 heads][64 lanes] exchange
-      for (int tt = 0; tt < NT; ++tt) {
+      // an empty range of a split token leaves its partial output unwritten: its
+      // lse is -inf and the merge does not read it (a plain partial call still
+      // writes O = 0 for an empty row set)
+      const int n_out_tiles = (EPI == EPI_PARTIAL && !any && p.per_item > 0) ? 0 : NT;
+      for (int tt = 0; tt < n_out_tiles; ++tt) {
         float o[64];
         if (any) {
           tmem_ld32(tmem + lane_base + kOCol + 64 * tt, o);
@@ -906,7 +913,7 @@ attn_merge_kernel(const float* __restrict__ Os, const float* __restrict__ Ls, co
                   const int64_t* __restrict__ q_pos, int T, int n_split, int H, int D, int inv_rope, int rope_dim,
                   float rope_base, void* __restrict__ out, int out_bf16) {
   constexpr int kHeads = 8;                       // heads per CTA (blockIdx.y selects the group)
-  __shared__ float s_coef[kHeads][16];
+  __shared__ float s_coef[kHeads][kMaxSplit];
   __shared__ float2 s_cs[32];
   const int64_t bt = blockIdx.x;
   const int h0 = blockIdx.y * kHeads;
@@ -944,6 +951,7 @@ attn_merge_kernel(const float* __restrict__ Os, const float* __restrict__ Ls, co
     const int pd = first ? d0 + half : d0 - half;
     for (int sp = 0; sp < n_split; ++sp) {
       const float c = s_coef[hl][sp];
+      if (c == 0.f) continue;                     // an empty range (lse -inf): its output was not written
       const float* src = Os + ((bt * n_split + sp) * H + h) * (int64_t)D;
       const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + d0));
       const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + d0) + 1);
@@ -1340,7 +1348,7 @@ extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q
                                                     int n_split, void* workspace, size_t ws_bytes, void* out,
                                                     csa_dtype_t out_dtype, cudaStream_t stream) {
   clear_error();
-  CSA_REQUIRE(n_split >= 1 && n_split <= 16, "csa_fused_attention_splitkv: n_split must be in [1, 16]");
+  CSA_REQUIRE(n_split >= 1 && n_split <= kMaxSplit, "csa_fused_attention_splitkv: n_split must be in [1, 32]");
   csa_status_t s = check_common("csa_fused_attention_splitkv", q, q_dtype, kv, kv_dtype, kv_rope, kv_scale, cap,
                                 n_seq, T, H, D, rope_dim);
   if (s != CSA_OK) return s;
@@ -1366,6 +1374,15 @@ extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q
   p.kv2 = kv_tok; p.cap2 = tok_cap; p.src2 = window_mode == 0 ? SRC2_WINDOW : SRC2_CACHE; p.W = W;
   p.n_seq = n_seq; p.T = T; p.H = H; p.scale = scale; p.scale_log2 = scale * 1.4426950408889634f;
   p.O_part = Os; p.lse_part = Ls; p.rope_dim = rope_dim; p.n_split = n_split;
+  {
+    // one range length for every token: the longest possible row set (k
+    // gathered or cap dense entries, plus the window) cut into n_split ranges,
+    // so short tokens take fewer, fuller ranges instead of n_split tiny ones
+    const int64_t rows1 = idx ? (int64_t)k : cap;
+    const int64_t rows2 = std::min<int64_t>(W, tok_cap);
+    const int64_t nh_max = (rows1 + kRows - 1) / kRows + (rows2 + kRows - 1) / kRows;
+    p.per_item = (int)std::max<int64_t>(1, (nh_max + n_split - 1) / n_split);
+  }
   p.item_counter = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(Ls) + ((parts * 4 + 255) / 256) * 256);
   cudaError_t ce = cudaMemsetAsync(p.item_counter, 0, sizeof(uint32_t), stream);
   if (ce != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_fused_attention_splitkv: counter reset failed: %s", cudaGetErrorString(ce));
