@@ -286,6 +286,10 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
   constexpr int KV2 = (KV == KV_F32) ? KV_F32 : KV_BF16;   // window rows: bf16 unless the store is fp32
 
   extern __shared__ uint8_t smem_raw[];
+  // launched as a dependent of the previous kernel: wait for its results (the
+  // queries, index lists and caches), then let the next kernel begin launching
+  pdl_wait();
+  pdl_trigger();
   // aligned by offsetting the shared array itself, so accesses stay in the shared window
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem;
@@ -915,6 +919,7 @@ attn_merge_kernel(const float* __restrict__ Os, const float* __restrict__ Ls, co
   constexpr int kHeads = 8;                       // heads per CTA (blockIdx.y selects the group)
   __shared__ float s_coef[kHeads][kMaxSplit];
   __shared__ float2 s_cs[32];
+  pdl_wait();                                     // the partials of the attention kernel are complete
   const int64_t bt = blockIdx.x;
   const int h0 = blockIdx.y * kHeads;
   const int b = (int)(bt / T), t = (int)(bt % T);
@@ -1170,7 +1175,8 @@ csa_status_t launch_attn(const AttnParams& p, const AttnMaps& m, cudaStream_t st
   const int64_t items = (int64_t)p.n_seq * p.T * p.n_split;
   if (items == 0) return CSA_OK;
   const int grid = (int)std::min<int64_t>(items, num_sms());
-  kern<<<grid, kThreads, smem, st>>>(p, m.q, m.kv, m.tok);
+  e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, p, m.q, m.kv, m.tok);
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attention: launch failed: %s", cudaGetErrorString(e));
   return check_launch("attention");
 }
 
@@ -1391,7 +1397,10 @@ extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q
   const int64_t toks = (int64_t)n_seq * T;
   if (toks == 0) return CSA_OK;
   CSA_REQUIRE(toks <= 0x7fffffff, "csa_fused_attention_splitkv: too many tokens");
-  attn_merge_kernel<<<dim3((unsigned)toks, (unsigned)((H + 7) / 8)), 256, 0, stream>>>(
-      Os, Ls, sink, q_pos, T, n_split, H, D, inv_rope, rope_dim, rope_base, out, out_dtype == CSA_BF16);
+  cudaError_t le = launch_pdl(attn_merge_kernel, dim3((unsigned)toks, (unsigned)((H + 7) / 8)), dim3(256), 0, stream,
+                              (const float*)Os, (const float*)Ls, sink, q_pos, T, n_split, H, D, inv_rope, rope_dim,
+                              rope_base, out, (int)(out_dtype == CSA_BF16));
+  if (le != cudaSuccess)
+    return fail(CSA_ERR_CUDA, "csa_fused_attention_splitkv(merge): launch failed: %s", cudaGetErrorString(le));
   return check_launch("csa_fused_attention_splitkv(merge)");
 }

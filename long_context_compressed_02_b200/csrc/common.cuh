@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <utility>
 #include <cuda_runtime.h>
 #include "../../include/csa.h"
 
@@ -18,6 +19,26 @@ inline csa_status_t check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
   return CSA_OK;
+}
+
+// Programmatic dependent launch: a kernel launched this way may start while
+// the previous kernel on the stream finishes; it must call pdl_wait() before
+// touching anything that kernel (or an earlier one) writes, and does so first
+// thing, which also keeps the chain of completions transitive.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 inline int num_sms() {

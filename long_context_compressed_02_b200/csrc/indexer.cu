@@ -81,6 +81,8 @@ struct IdxParams {
   int n_seq, n_qblocks;
   int64_t n_items;        // n_seq x n_qblocks x key chunks
   uint32_t* item_counter; // zeroed before the launch: items are claimed dynamically
+  uint32_t* hist_zero;    // non-null: [hist_words] histogram words this grid zeroes
+  int64_t hist_words;
 };
 
 // One work item of the persistent scores kernel: a key chunk of one token
@@ -223,6 +225,14 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   // aligned by offsetting the shared array itself, so accesses stay in the shared window
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the selection kernels may start launching; they wait for this grid's end.
+  // Rows split into chunks: this grid zeroes their key histograms (filled by
+  // the next kernel), in place of a separate memset.
+  pdl_trigger();
+  if (p.hist_zero) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < p.hist_words; i += (int64_t)gridDim.x * blockDim.x)
+      p.hist_zero[i] = 0u;
+  }
 
   const uint32_t a_bytes = 128u * p.DI;
   const uint32_t b_bytes = (uint32_t)p.N * p.DI;
@@ -739,6 +749,8 @@ struct TopkParams {
 __global__ void __launch_bounds__(kTopkThreads)
 topk_hist_kernel(TopkParams p) {
   __shared__ uint32_t h[kHistBins];
+  pdl_wait();                              // the scores (and the zeroed histograms) are complete
+  pdl_trigger();
   const int64_t row = blockIdx.x;
   const int chunk = blockIdx.y;
   const int b = (int)(row / p.T), t = (int)(row % p.T);
@@ -795,6 +807,8 @@ template <bool FILTERED>
 __global__ void __launch_bounds__(FILTERED ? kTopkThreads : kTopkThreadsSmall, FILTERED ? 2 : 8)
 topk_chunk_kernel(TopkParams p) {
   extern __shared__ uint32_t s_keys[];   // kChunk keys (or kChunk / 2 keys + kChunk / 2 ids)
+  pdl_wait();                            // scores (and histograms) of the previous kernels are complete
+  pdl_trigger();
   constexpr int NTH = FILTERED ? kTopkThreads : kTopkThreadsSmall;
   __shared__ SelectSmem<NTH> ss;
   __shared__ uint32_t s_B;
@@ -885,6 +899,8 @@ topk_chunk_kernel(TopkParams p) {
 // candidates in ascending entry order).
 __global__ void __launch_bounds__(kTopkThreads)
 topk_merge_kernel(TopkParams p) {
+  pdl_wait();                            // every chunk's candidates are written
+  pdl_trigger();
   extern __shared__ uint32_t s_mem[];
   uint32_t* s_keys = s_mem;                                   // kMergeCap
   int32_t* s_ids = reinterpret_cast<int32_t*>(s_mem + kMergeCap);
@@ -1046,6 +1062,10 @@ csa_status_t index_topk_run(const uint8_t* qI, const float* qI_scale, const floa
     cudaError_t e = cudaMemsetAsync(ip.item_counter, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_index_topk: counter reset failed: %s", cudaGetErrorString(e));
   }
+  if (L.n_chunks > 1) {
+    ip.hist_zero = reinterpret_cast<uint32_t*>(ws + L.hist);
+    ip.hist_words = (int64_t)n_seq * T * kHistBins;
+  }
   if (fp4) {
     const size_t smem = smem_for(kStages);
     const int grid = (int)std::min<int64_t>(ip.n_items, sms);
@@ -1097,21 +1117,23 @@ csa_status_t index_topk_run(const uint8_t* qI, const float* qI_scale, const floa
   auto chunk_kernel = L.n_chunks > 1 ? topk_chunk_kernel<true> : topk_chunk_kernel<false>;
   cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   dim3 g1((unsigned)rows, (unsigned)L.n_chunks);
+  // the selection kernels follow by dependent launch (each waits for the one before)
+  auto launched = [&](cudaError_t e, const char* what) -> csa_status_t {
+    if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+    return check_launch(what);
+  };
   if (L.n_chunks > 1) {
-    cudaError_t e = cudaMemsetAsync(tp.hist, 0, (size_t)rows * kHistBins * sizeof(uint32_t), stream);
-    if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_index_topk: histogram reset failed: %s", cudaGetErrorString(e));
-    topk_hist_kernel<<<g1, kTopkThreads, 0, stream>>>(tp);
-    st = check_launch("csa_index_topk(histogram)");
+    st = launched(launch_pdl(topk_hist_kernel, g1, dim3(kTopkThreads), 0, stream, tp), "csa_index_topk(histogram)");
     if (st != CSA_OK) return st;
   }
-  chunk_kernel<<<g1, L.n_chunks > 1 ? kTopkThreads : kTopkThreadsSmall, smem1, stream>>>(tp);
-  st = check_launch("csa_index_topk(select)");
+  st = launched(launch_pdl(chunk_kernel, g1, dim3(L.n_chunks > 1 ? kTopkThreads : kTopkThreadsSmall), smem1, stream, tp),
+                "csa_index_topk(select)");
   if (st != CSA_OK) return st;
   if (L.n_chunks > 1) {
     const size_t smem2 = kMergeCap * 8;
     cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
-    topk_merge_kernel<<<(unsigned)rows, kTopkThreads, smem2, stream>>>(tp);
-    st = check_launch("csa_index_topk(merge)");
+    st = launched(launch_pdl(topk_merge_kernel, dim3((unsigned)rows), dim3(kTopkThreads), smem2, stream, tp),
+                  "csa_index_topk(merge)");
   }
   return st;
 }
