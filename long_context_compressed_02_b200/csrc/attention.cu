@@ -410,6 +410,8 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
         mbar_arrive(q_full);
       }
       // ---- KV half chunks into the two-slot ring
+      int pre_c = -1;                    // half chunk whose gathered row index pre_row holds
+      int32_t pre_row = 0;
       for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
         const int slot = g & 1;
         const uint32_t fpar = ((g >> 1) & 1) ^ 1;     // completion of PV(g - 2), which read this slot
@@ -481,6 +483,116 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
           mbar_arrive(&full[NT - 1]);
           continue;
         }
+        if (KV == KV_FP8 && !win) {
+          // e4m3 rows: nope part (D - 64 bytes), bf16 RoPE part (64 dims), fp32
+          // row scale.  Loader warp lw owns rows 16 lw .. 16 lw + 15 of the half
+          // chunk; lane l looks up row 16 lw + (l & 15).  The loads are
+          // coalesced: in slab pair tt (e4m3 bytes 128 tt .. 128 tt + 127 of a
+          // row) lane l takes 16-byte piece l & 7 of row 4 i + (l >> 3), so one
+          // load instruction reads whole 128-byte segments of four rows.  The last
+          // pair holds the row's last 64 e4m3 bytes (lane l: piece l & 3 of row
+          // 8 i + (l >> 2)) and its RoPE part (piece l & 7 of row 4 i + (l >> 3)).
+          // Every load of the half chunk is issued before the slot is free.
+          constexpr int kNope = D - 64;
+          const int rl = lane & 15;
+          const uint8_t* kvn = reinterpret_cast<const uint8_t*>(p.kv);
+          const uint8_t* kvr = reinterpret_cast<const uint8_t*>(p.kv_rope);
+          // Issues the loads of (source-1) half chunk cc: this lane's pieces and
+          // the scale of its own row.
+          auto issue = [&](int cc, uint4 (&rw)[NT][4], uint4 (&rp)[4], float& scv) {
+            const int r1 = (cc - rs.nh2) * kRows + 16 * lw + rl;
+            bool vld = r1 < rs.n1;
+            int64_t row1 = 0;
+            if (vld) {
+              if (rs.idx) {
+                row1 = pre_c == cc ? pre_row : __ldg(rs.idx + r1);
+                if (row1 < 0 || row1 >= p.cap) { atomicOr(&g_err_attn, DEV_ERR_BAD_INDEX); vld = false; row1 = 0; }
+              } else {
+                row1 = r1;
+              }
+            }
+            const long long gr0 = (long long)b * p.cap + row1;
+            scv = vld ? __ldg(p.kv_scale + gr0) : 0.f;
+            const uint4 zero = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int src = 4 * i + (lane >> 3);
+              const long long gr = __shfl_sync(0xffffffffu, gr0, src);
+              const bool v = __shfl_sync(0xffffffffu, vld, src);
+#pragma unroll
+              for (int tt = 0; tt < NT - 1; ++tt)
+                rw[tt][i] = v ? __ldg(reinterpret_cast<const uint4*>(kvn + gr * kNope + 128 * tt + 16 * (lane & 7)))
+                              : zero;
+              rp[i] = v ? __ldg(reinterpret_cast<const uint4*>(kvr + gr * 128 + 16 * (lane & 7))) : zero;
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int src = 8 * i + (lane >> 2);
+              const long long gr = __shfl_sync(0xffffffffu, gr0, src);
+              const bool v = __shfl_sync(0xffffffffu, vld, src);
+              rw[NT - 1][i] =
+                  v ? __ldg(reinterpret_cast<const uint4*>(kvn + gr * kNope + 128 * (NT - 1) + 16 * (lane & 3)))
+                    : zero;
+            }
+          };
+          uint4 raw[NT][4], rope[4];
+          float sc;
+          issue(c, raw, rope, sc);
+          // While these loads are in flight: the next half chunk's gathered row
+          // indices (kept in pre_row), or its contiguous rows' bytes bulk-prefetched
+          // into L2, so that its loads are served from L2.
+          if (c + 1 < rs.c1) {
+            const int r0 = (c + 1 - rs.nh2) * kRows;
+            const int nr = min(kRows, rs.n1 - r0);
+            if (rs.idx == nullptr) {
+              const long long g0 = (long long)b * p.cap + r0;
+              if (lt == 0) prefetch_l2_bulk(kvn + g0 * kNope, (uint32_t)(nr * kNope));
+              else if (lt == 1) prefetch_l2_bulk(kvr + g0 * 128, (uint32_t)(nr * 128));
+              else if (lt == 2 && ((g0 | nr) & 3) == 0) prefetch_l2_bulk(p.kv_scale + g0, (uint32_t)(nr * 4));
+            } else if (16 * lw + rl < nr) {
+              pre_row = __ldg(rs.idx + r0 + 16 * lw + rl);
+              pre_c = c + 1;
+            }
+          }
+          // row scales to the converting lanes (waits for the scale loads only now)
+          float sc4[4], sc2[2];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sc4[i] = __shfl_sync(0xffffffffu, sc, 4 * i + (lane >> 3));
+#pragma unroll
+          for (int i = 0; i < 2; ++i) sc2[i] = __shfl_sync(0xffffffffu, sc, 8 * i + (lane >> 2));
+#pragma unroll
+          for (int tt = 0; tt < NT; ++tt) {
+            if (!wait_bar(&done[tt], fpar, abort_flag)) { ok = false; break; }
+            if (tt < NT - 1) {
+              // piece l & 7 of the pair: slab 2 tt + (l & 7) / 4, 16-byte chunks 2 (l & 3), 2 (l & 3) + 1
+              uint8_t* dst = sl_base + (2 * tt + ((lane & 7) >> 2)) * kSlab;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int rr = 16 * lw + 4 * i + (lane >> 3);
+                float v[16];
+                e4m3x16_to_float(raw[tt][i], sc4[i], v);
+                st_shared16(dst + swz128(rr, 2 * (lane & 3)), to_bf16x8(v));
+                st_shared16(dst + swz128(rr, 2 * (lane & 3) + 1), to_bf16x8(v + 8));
+              }
+            } else {
+              uint8_t* dst = sl_base + (2 * tt) * kSlab;
+#pragma unroll
+              for (int i = 0; i < 2; ++i) {
+                const int rr = 16 * lw + 8 * i + (lane >> 2);
+                float v[16];
+                e4m3x16_to_float(raw[tt][i], sc2[i], v);
+                st_shared16(dst + swz128(rr, 2 * (lane & 3)), to_bf16x8(v));
+                st_shared16(dst + swz128(rr, 2 * (lane & 3) + 1), to_bf16x8(v + 8));
+              }
+              uint8_t* dr = sl_base + (NS - 1) * kSlab;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) st_shared16(dr + swz128(16 * lw + 4 * i + (lane >> 3), lane & 7), rope[i]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&full[tt]);
+          }
+          continue;
+        }
         // converting loads: thread (my_r, part) converts slabs 2 tt + part of row my_r
         const int r = cl * kRows + my_r;
         bool valid = r < nset;
@@ -494,47 +606,6 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
           } else {
             row = r;
           }
-        }
-        if (KV == KV_FP8 && !win) {
-          // e4m3 row: nope part (D - 64 bytes) + bf16 RoPE part + scale.  The raw
-          // bytes of this thread's slabs are fetched before the slot is free.
-          constexpr int kNope = D - 64;
-          const uint8_t* srcn = reinterpret_cast<const uint8_t*>(p.kv) + ((int64_t)b * p.cap + row) * kNope;
-          const uint4* srcr = reinterpret_cast<const uint4*>(p.kv_rope + ((int64_t)b * p.cap + row) * 64);
-          const float sc = valid ? __ldg(p.kv_scale + (int64_t)b * p.cap + row) : 0.f;
-          uint4 raw[NT][4];
-          uint4 rp8[8];
-#pragma unroll
-          for (int tt = 0; tt < NT; ++tt) {
-            const int s = 2 * tt + part;
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              raw[tt][i] = (valid && s < NS - 1) ? __ldg(reinterpret_cast<const uint4*>(srcn + 64 * s) + i)
-                                                  : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) rp8[i] = (valid && part == 1) ? __ldg(srcr + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-          for (int tt = 0; tt < NT; ++tt) {
-            if (!wait_bar(&done[tt], fpar, abort_flag)) { ok = false; break; }
-            const int s = 2 * tt + part;
-            uint8_t* dst = sl_base + s * kSlab;
-            if (s < NS - 1) {
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                float v[16];
-                e4m3x16_to_float(raw[tt][q4], sc, v);
-                st_shared16(dst + swz128(my_r, 2 * q4), to_bf16x8(v));
-                st_shared16(dst + swz128(my_r, 2 * q4 + 1), to_bf16x8(v + 8));
-              }
-            } else {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) st_shared16(dst + swz128(my_r, q), rp8[q]);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&full[tt]);
-          }
-          continue;
         }
         // fp32 rows (an fp32 store and its window rows)
         const float* src = win ? reinterpret_cast<const float*>(p.kv2) + ((int64_t)b * p.cap2 + row) * D
@@ -918,22 +989,34 @@ attn_merge_kernel(const float* __restrict__ Os, const float* __restrict__ Ls, co
                   float rope_base, void* __restrict__ out, int out_bf16) {
   constexpr int kHeads = 8;                       // heads per CTA (blockIdx.y selects the group)
   __shared__ float s_coef[kHeads][kMaxSplit];
+  __shared__ int s_act[kMaxSplit];                // splits with a nonzero weight for some head of the group
+  __shared__ int s_nact;
   __shared__ float2 s_cs[32];
   pdl_wait();                                     // the partials of the attention kernel are complete
   const int64_t bt = blockIdx.x;
   const int h0 = blockIdx.y * kHeads;
   const int b = (int)(bt / T), t = (int)(bt % T);
   const int64_t pos = (q_pos ? q_pos[b] : 0) + t;
-  const int tid = threadIdx.x;
-  if (tid < kHeads && h0 + tid < H) {
-    const int h = h0 + tid;
-    float M = sink ? sink[h] : -CUDART_INF_F;
-    for (int sp = 0; sp < n_split; ++sp) M = fmaxf(M, Ls[(bt * n_split + sp) * H + h]);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  {
+    // warp w: head h0 + w; lane: split (n_split <= 32), one softmax over the
+    // partials' lse and the sink
+    const int h = h0 + warp;
+    const bool hv = warp < kHeads && h < H;
+    const float l = (hv && lane < n_split) ? Ls[(bt * n_split + lane) * H + h] : -CUDART_INF_F;
+    const float sk = (hv && sink) ? sink[h] : -CUDART_INF_F;
+    float M = l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    M = fmaxf(M, sk);
     if (M == -CUDART_INF_F) M = 0.f;
-    float den = sink ? __expf(sink[h] - M) : 0.f;
-    for (int sp = 0; sp < n_split; ++sp) den += __expf(Ls[(bt * n_split + sp) * H + h] - M);
+    const float e = __expf(l - M);
+    float den = e;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (sink) den += __expf(sk - M);
     const float inv = den > 0.f ? 1.f / den : 0.f;
-    for (int sp = 0; sp < n_split; ++sp) s_coef[tid][sp] = __expf(Ls[(bt * n_split + sp) * H + h] - M) * inv;
+    if (warp < kHeads) s_coef[warp][lane] = (hv && lane < n_split) ? e * inv : 0.f;
   }
   const int half = rope_dim / 2;
   if (inv_rope && tid >= 32 && tid < 32 + half) {
@@ -945,28 +1028,48 @@ attn_merge_kernel(const float* __restrict__ Os, const float* __restrict__ Ls, co
     s_cs[j] = make_float2((float)cd, (float)sd);
   }
   __syncthreads();
+  if (warp == 0) {
+    // an empty range (lse -inf) has weight 0 and its output was not written
+    bool any = false;
+#pragma unroll
+    for (int hl = 0; hl < kHeads; ++hl) any |= s_coef[hl][lane] != 0.f;
+    const unsigned act = __ballot_sync(0xffffffffu, any);
+    if (any) s_act[__popc(act & ((1u << lane) - 1u))] = lane;
+    if (lane == 0) s_nact = __popc(act);
+  }
+  __syncthreads();
+  const int n_act = s_nact;
   const int r0 = D - rope_dim;
   const int per_row = D / 8;
   const int nh = min(kHeads, H - h0);
+  constexpr int kU = 4;                           // partials loaded together
   for (int idx = tid; idx < nh * per_row; idx += blockDim.x) {
     const int hl = idx / per_row, h = h0 + hl, d0 = (idx % per_row) * 8;
     float v[8] = {0, 0, 0, 0, 0, 0, 0, 0}, w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const bool rot = inv_rope && d0 >= r0;
     const bool first = d0 < r0 + half;
     const int pd = first ? d0 + half : d0 - half;
-    for (int sp = 0; sp < n_split; ++sp) {
-      const float c = s_coef[hl][sp];
-      if (c == 0.f) continue;                     // an empty range (lse -inf): its output was not written
-      const float* src = Os + ((bt * n_split + sp) * H + h) * (int64_t)D;
-      const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + d0));
-      const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + d0) + 1);
-      v[0] += c * a0.x; v[1] += c * a0.y; v[2] += c * a0.z; v[3] += c * a0.w;
-      v[4] += c * a1.x; v[5] += c * a1.y; v[6] += c * a1.z; v[7] += c * a1.w;
-      if (rot) {
-        const float4 b0 = __ldg(reinterpret_cast<const float4*>(src + pd));
-        const float4 b1 = __ldg(reinterpret_cast<const float4*>(src + pd) + 1);
-        w[0] += c * b0.x; w[1] += c * b0.y; w[2] += c * b0.z; w[3] += c * b0.w;
-        w[4] += c * b1.x; w[5] += c * b1.y; w[6] += c * b1.z; w[7] += c * b1.w;
+    for (int i0 = 0; i0 < n_act; i0 += kU) {
+      float4 a[kU][2], q[kU][2];
+      float c[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const bool in = i0 + u < n_act;
+        const int sp = in ? s_act[i0 + u] : 0;
+        c[u] = in ? s_coef[hl][sp] : 0.f;
+        const float* src = Os + ((bt * n_split + sp) * H + h) * (int64_t)D;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        a[u][0] = in ? __ldg(reinterpret_cast<const float4*>(src + d0)) : z;
+        a[u][1] = in ? __ldg(reinterpret_cast<const float4*>(src + d0) + 1) : z;
+        q[u][0] = (in && rot) ? __ldg(reinterpret_cast<const float4*>(src + pd)) : z;
+        q[u][1] = (in && rot) ? __ldg(reinterpret_cast<const float4*>(src + pd) + 1) : z;
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        v[0] += c[u] * a[u][0].x; v[1] += c[u] * a[u][0].y; v[2] += c[u] * a[u][0].z; v[3] += c[u] * a[u][0].w;
+        v[4] += c[u] * a[u][1].x; v[5] += c[u] * a[u][1].y; v[6] += c[u] * a[u][1].z; v[7] += c[u] * a[u][1].w;
+        w[0] += c[u] * q[u][0].x; w[1] += c[u] * q[u][0].y; w[2] += c[u] * q[u][0].z; w[3] += c[u] * q[u][0].w;
+        w[4] += c[u] * q[u][1].x; w[5] += c[u] * q[u][1].y; w[6] += c[u] * q[u][1].z; w[7] += c[u] * q[u][1].w;
       }
     }
     if (rot) {

@@ -233,6 +233,11 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 }
 
 // 16-byte global -> shared async copy (L2 only); src_bytes < 16 zero-fills the rest.
+// Bulk prefetch of [src, src + bytes) into L2 (no destination, no completion
+// to wait for); src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
