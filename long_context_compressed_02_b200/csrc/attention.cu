@@ -19,8 +19,8 @@
 // K-major A operand of the first product and, read through an MN-major
 // descriptor, the A operand of the second; nothing is transposed or copied.
 // Rows stream through a ring of two 64-row slots (half chunks), so the loads
-// of half chunk h+1 overlap the S, softmax and PV work of half chunk h; S(h+1)
-// is issued before PV(h), so the softmax of h overlaps the S products of h+1.
+// of half chunk h+1 overlap the S, softmax and PV work of half chunk h, and the
+// S products of h+1 overlap the softmax of h.
 // S goes to two TMEM accumulators (even / odd slabs, alternating MMA by MMA,
 // since an MMA into the accumulator of the one before waits for it), summed by
 // the softmax.  Softmax runs per column (head) over TMEM lanes (rows): the
@@ -31,10 +31,13 @@
 // global memory (the RoPE dimension pairs d, d+32 sit in different warps and
 // are exchanged through shared memory for the inverse rotation).
 //
-// Roles (288 threads): warps 0-3 softmax + epilogue, warps 4-7 loaders
+// Roles (352 threads): warps 0-3 softmax + epilogue, warps 4-7 loaders
 // (gathers through cp.async, fenced and signalled per slab pair by the
 // producer, TMA boxes for contiguous rows, or load-convert for fp32 / e4m3
-// stores), warp 8 TMEM allocation + MMA issue.  Each slot is refilled slab
+// stores), warp 8 TMEM allocation + the even-slab S MMAs, warp 10 the odd-slab
+// S MMAs, warp 9 the PV MMAs (one issuing thread each: an MMA instruction
+// holds its thread for tens of cycles, so a single issuer starves the tensor
+// pipe on products this small).  Each slot is refilled slab
 // pair by slab pair as the PV tile pair that read it retires, and S MMAs start
 // on a slab pair as soon as it lands.  Work items (query token, range of half
 // chunks) are taken grid-stride, or, for split-KV calls, claimed from a
@@ -61,7 +64,7 @@ uint32_t read_clear_err_attention() {
 
 namespace {
 
-constexpr int kThreads = 288;
+constexpr int kThreads = 352;      // 11 warps: 4 softmax + epilogue, 4 loaders, 3 MMA issuers
 constexpr int kNQ = 64;            // query rows (heads) per tile = MMA N
 constexpr int kRows = 64;          // KV rows per ring slot (a half chunk) = M of the S MMA
 constexpr float kTau = 8.0f;       // lazy-rescale threshold (log2 units)
@@ -315,12 +318,12 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(q_full, 128); mbar_init(q_free, 1); mbar_init(epi_done, 128);
+    mbar_init(q_full, 128); mbar_init(q_free, 2); mbar_init(epi_done, 128);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128); mbar_init(&p_full[i], 128);
+      mbar_init(&s_full[i], 2); mbar_init(&s_free[i], 128); mbar_init(&p_full[i], 128);
       for (int t = 0; t < NT; ++t) { mbar_init(&kv_full[i * NT + t], 128); mbar_init(&pv_done[i * NT + t], 1); }
     }
-    for (int i = 0; i < 4; ++i) { mbar_init(&item_full[i], 1); mbar_init(&item_empty[i], 9); }
+    for (int i = 0; i < 4; ++i) { mbar_init(&item_full[i], 1); mbar_init(&item_empty[i], 11); }
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -334,7 +337,7 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
   // Item sequence k = 0, 1, ... of this CTA: grid-stride, or (with a counter)
   // claimed by one loader thread with an atomic and handed to every role warp
   // through a 4-slot ring, so CTAs that drew short items take more of them.
-  // Whole-warp call; every role warp (9 of them) releases each slot once.
+  // Whole-warp call; every role warp (11 of them) releases each slot once.
   auto get_item = [&](uint32_t k, bool fetcher) -> int64_t {
     if (p.item_counter == nullptr) return (int64_t)blockIdx.x + (int64_t)k * gridDim.x;
     const uint32_t slot = k & 3, par = (k >> 2) & 1;
@@ -625,12 +628,16 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
         }
       }
     }
-  } else if (warp == 8) {
-    // ============================ MMA issuer (lane 0; the warp computes row sets)
+  } else if (warp >= 8) {
+    // ============================ MMA issuers (lane 0; each warp computes row sets)
     // S^T(h) = KV_h[64 rows, D] . Q^T        M 64, N 64, into TMEM columns 64 (h % 2)
+    //          (+ 128 for the odd slabs' accumulator)
     // O^T   += KV_h^T[128 d, 64 rows] . P_h^T  M 128, N 64, per 128-d tile
-    // S(h + 1) is issued before PV(h), so the softmax of half chunk h overlaps
-    // the S products of the next one.
+    // An MMA instruction holds its issuing thread for tens of cycles whatever its
+    // shape, so one thread cannot keep the tensor pipe fed with these small
+    // products: warp 8 issues the even slabs of S, warp 10 the odd slabs (the
+    // two accumulators of h's S buffer, side by side), warp 9 the PV products.
+    const int role = warp - 8;                 // 0: S even slabs, 1: PV, 2: S odd slabs
     const uint32_t idesc_s = make_idesc(64, kNQ, 1, 1, 0, 0);
     const uint32_t idesc_o = make_idesc(128, kNQ, 1, 1, 1, 1);
     // Descriptors differ only in the start-address field (bits 0..13, address >> 4):
@@ -642,8 +649,8 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
     uint32_t g = 0, qcount = 0, pv_items = 0;
     bool ok = true;
     // PV(h): the 4 K-steps of a tile pair alternate between the pair's two
-    // accumulators (an MMA into the accumulator of the previous one waits for
-    // it); each pair commits its two tiles' barriers, which free their slabs.
+    // accumulators; each pair commits its two tiles' barriers, which free their
+    // slabs for the next loads.
     auto issue_pv = [&](uint32_t h, bool first) -> bool {
       if (!wait_bar(&p_full[h & 1], (h >> 1) & 1, abort_flag)) return false;
       if (first) {
@@ -680,43 +687,30 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
       const RowSet rs = row_set_warp(p, b, t, sp, lane);
       if (rs.c1 <= rs.c0) continue;
       if (lane == 0) {
-        if (!wait_bar(q_full, qcount & 1, abort_flag)) ok = false;
-        ++qcount;
-        // Order: S(h), then PV(h - 1) (its softmax overlapped S(h)); the item's
-        // last PV follows its S at once, so the epilogue does not wait for the
-        // next item's loads.
-        bool pend = false;
-        uint32_t pend_g = 0;
-        bool pend_first = false;
-        for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
-          const uint32_t slot = g & 1;
-          if (!wait_bar(&s_free[slot], ((g >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          // S^T(g): even slabs into accumulator a (columns 64 slot), odd slabs into
-          // accumulator b (columns 128 + 64 slot), alternating MMA by MMA
-#pragma unroll 1
-          for (int tt = 0; tt < NT; ++tt) {
-            if (!wait_bar(&kv_full[slot * NT + tt], (g >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (role == 1) {
+          for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g)
+            if (!issue_pv(g, c == rs.c0)) ok = false;
+        } else {
+          if (!wait_bar(q_full, qcount & 1, abort_flag)) ok = false;
+          ++qcount;
+          const int hh = role == 0 ? 0 : 1;    // this issuer's slabs: 2 tt + hh
+          for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
+            const uint32_t slot = g & 1;
+            if (!wait_bar(&s_free[slot], ((g >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
+#pragma unroll 1
+            for (int tt = 0; tt < NT; ++tt) {
+              if (!wait_bar(&kv_full[slot * NT + tt], (g >> 1) & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              const int s = 2 * tt + hh;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                const int s = 2 * tt + hh;
-                mma_bf16(tmem + 64 * slot + 128 * hh, dS_A + ((slot * kSlot + s * kSlab + kk * 32) >> 4),
-                         dS_B + ((s * kQSlab + kk * 32) >> 4), idesc_s, (tt | kk) != 0);
-              }
+              for (int kq = 0; kq < 4; ++kq)
+                mma_bf16(tmem + 64 * slot + 128 * hh, dS_A + ((slot * kSlot + s * kSlab + kq * 32) >> 4),
+                         dS_B + ((s * kQSlab + kq * 32) >> 4), idesc_s, (tt | kq) != 0);
             }
-          }
-          if (!ok) break;
-          mma_commit(&s_full[slot]);
-          const bool last = c == rs.c1 - 1;
-          if (last) mma_commit(q_free);
-          if (pend && !issue_pv(pend_g, pend_first)) { ok = false; break; }
-          pend = true; pend_g = g; pend_first = (c == rs.c0);
-          if (last) {
-            if (!issue_pv(pend_g, pend_first)) { ok = false; break; }
-            pend = false;
+            if (!ok) break;
+            mma_commit(&s_full[slot]);
+            if (c == rs.c1 - 1) mma_commit(q_free);
           }
         }
       }
