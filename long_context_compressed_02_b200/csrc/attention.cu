@@ -317,6 +317,10 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // inverse RoPE frequencies, once per CTA: inv_freq_j = base^(-2j / rope_dim)
+  __shared__ double s_invf[32];
+  if (EPI == EPI_COMBINE && p.inv_rope && tid < 32)
+    s_invf[tid] = exp(-2.0 * (double)tid / (double)p.rope_dim * log((double)p.rope_base));
   if (tid == 0) {
     mbar_init(q_full, 128); mbar_init(q_free, 2); mbar_init(epi_done, 128);
     for (int i = 0; i < 2; ++i) {
@@ -741,15 +745,20 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
       const int64_t pos = (p.q_pos ? p.q_pos[b] : 0) + t;
       float2* cs = s_cs + (icount & 1) * 32;
       if (EPI == EPI_COMBINE && p.inv_rope && tid < 32) {
-        const int j = tid;
-        double inv_freq = exp(-2.0 * (double)j / (double)p.rope_dim * log((double)p.rope_base));
-        double ang = fmod((double)pos * inv_freq, 6.283185307179586476925286766559);
-        double sd, cd;
-        sincos(ang, &sd, &cd);
-        cs[j] = make_float2((float)cd, (float)sd);
+        // angle pos * inv_freq_j reduced to [0, 2 pi) in double (pos reaches 2^20
+        // and more), then cos / sin in float of the reduced angle
+        const double ang = (double)pos * s_invf[tid];
+        const double r = ang - 6.283185307179586476925286766559 * floor(ang * 0.15915494309189533576888376337251);
+        float sf, cf;
+        sincosf((float)r, &sf, &cf);
+        cs[tid] = make_float2(cf, sf);
       }
       float m_own[2] = {-CUDART_INF_F, -CUDART_INF_F};   // running max of columns 2 lane, 2 lane + 1
-      float l_own[2] = {0.f, 0.f};                       // this warp's rows' sums of the same columns
+      // this thread's rows' running sums of its 16 columns (v16 layout), reduced
+      // over the rows once, in the epilogue
+      float l_part[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) l_part[i] = 0.f;
       for (int c = rs.c0; c < rs.c1 && ok; ++c, ++g) {
         const uint32_t sb = g & 1;
         if (!wait_bar(&s_full[sb], (g >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -771,25 +780,40 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
           if (!vA) { x[4 * cc] = -CUDART_INF_F; x[4 * cc + 1] = -CUDART_INF_F; }
           if (!vB) { x[4 * cc + 2] = -CUDART_INF_F; x[4 * cc + 3] = -CUDART_INF_F; }
         }
-        float v16[16];
+        // The running maxima stay unless a logit of this half chunk exceeds its
+        // column's maximum by more than kTau (lazy rescaling): one barrier
+        // reduction over the 128 threads decides; only then are the column
+        // maxima reduced and the maxima and their rescale factors updated.
+        const float sl2 = p.scale_log2;
+        bool exceed = c == rs.c0;
+        if (!exceed) {
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          v16[2 * cc] = fmaxf(x[4 * cc], x[4 * cc + 2]);
-          v16[2 * cc + 1] = fmaxf(x[4 * cc + 1], x[4 * cc + 3]);
+          for (int cc = 0; cc < 8; ++cc) {
+            const float2 mm = *reinterpret_cast<const float2*>(bc_m + 8 * cc + 2 * (lane & 3));
+            exceed |= fmaxf(x[4 * cc], x[4 * cc + 2]) * sl2 > mm.x + kTau;
+            exceed |= fmaxf(x[4 * cc + 1], x[4 * cc + 3]) * sl2 > mm.y + kTau;
+          }
         }
-        const float2 cm = col_reduce16<true>(v16, lane);
-        float* red = s_red + (g & 1) * 256;
-        *reinterpret_cast<float2*>(red + warp * 64 + 2 * lane) = cm;
-        named_bar_sync(1, 128);
+        exceed = named_bar_or(2, 128, exceed);
         bool need_rescale = false;
-        float alpha[2];
-        {
+        if (exceed) {
+          float v16[16];
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            v16[2 * cc] = fmaxf(x[4 * cc], x[4 * cc + 2]);
+            v16[2 * cc + 1] = fmaxf(x[4 * cc + 1], x[4 * cc + 3]);
+          }
+          const float2 cm = col_reduce16<true>(v16, lane);
+          float* red = s_red + (g & 1) * 256;
+          *reinterpret_cast<float2*>(red + warp * 64 + 2 * lane) = cm;
+          named_bar_sync(1, 128);
+          float alpha[2];
           const float2 r0 = *reinterpret_cast<const float2*>(red + 2 * lane);
           const float2 r1 = *reinterpret_cast<const float2*>(red + 64 + 2 * lane);
           const float2 r2 = *reinterpret_cast<const float2*>(red + 128 + 2 * lane);
           const float2 r3 = *reinterpret_cast<const float2*>(red + 192 + 2 * lane);
-          const float mx[2] = {fmaxf(fmaxf(r0.x, r1.x), fmaxf(r2.x, r3.x)) * p.scale_log2,
-                               fmaxf(fmaxf(r0.y, r1.y), fmaxf(r2.y, r3.y)) * p.scale_log2};
+          const float mx[2] = {fmaxf(fmaxf(r0.x, r1.x), fmaxf(r2.x, r3.x)) * sl2,
+                               fmaxf(fmaxf(r0.y, r1.y), fmaxf(r2.y, r3.y)) * sl2};
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const float mn = (mx[j] > m_own[j] + kTau) ? mx[j] : m_own[j];
@@ -800,10 +824,16 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
           __syncwarp();
           *reinterpret_cast<float2*>(bc_m + 2 * lane) = make_float2(m_own[0], m_own[1]);
           *reinterpret_cast<float2*>(bc_m + 64 + 2 * lane) = make_float2(alpha[0], alpha[1]);
+          need_rescale = __any_sync(0xffffffffu, need_rescale);
+          __syncwarp();
+          // the running sums of this thread's columns scale by the same factors
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const float2 al = *reinterpret_cast<const float2*>(bc_m + 64 + 8 * cc + 2 * (lane & 3));
+            l_part[2 * cc] *= al.x;
+            l_part[2 * cc + 1] *= al.y;
+          }
         }
-        need_rescale = __any_sync(0xffffffffu, need_rescale);
-        __syncwarp();
-        const float sl2 = p.scale_log2;
         float pr[32];
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
@@ -822,15 +852,11 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
           st_shared4(pb + swz128(rA, cc), pack_bf16(pr[4 * cc], pr[4 * cc + 1]));
           st_shared4(pb + swz128(rB, cc), pack_bf16(pr[4 * cc + 2], pr[4 * cc + 3]));
         }
-        // column sums of this half chunk (same ownership as the maxima)
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
-          v16[2 * cc] = pr[4 * cc] + pr[4 * cc + 2];
-          v16[2 * cc + 1] = pr[4 * cc + 1] + pr[4 * cc + 3];
+          l_part[2 * cc] += pr[4 * cc] + pr[4 * cc + 2];
+          l_part[2 * cc + 1] += pr[4 * cc + 1] + pr[4 * cc + 3];
         }
-        const float2 csum = col_reduce16<false>(v16, lane);
-        l_own[0] = l_own[0] * alpha[0] + csum.x;
-        l_own[1] = l_own[1] * alpha[1] + csum.y;
         if (need_rescale) {
           // O^T columns scale by alpha once PV(g - 1) has retired (this thread is
           // TMEM lane e of every tile)
@@ -857,9 +883,9 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
       }
       if (!ok) break;
       // ---------------- epilogue
-      // column sums over the 4 warps
+      // column sums over this warp's rows (lane l: columns 2 l, 2 l + 1), then over the 4 warps
       float* red = s_red + (g & 1) * 256;
-      *reinterpret_cast<float2*>(red + warp * 64 + 2 * lane) = make_float2(l_own[0], l_own[1]);
+      *reinterpret_cast<float2*>(red + warp * 64 + 2 * lane) = col_reduce16<false>(l_part, lane);
       named_bar_sync(1, 128);
       __syncwarp();
 #pragma unroll
@@ -942,23 +968,44 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
             o[h] = first ? o[h] * csj.x + w * csj.y : o[h] * csj.x - w * csj.y;
           }
         }
-        if (EPI == EPI_COMBINE) {
-          if (p.out_bf16) {
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + obase * D + d;
+        // Out through shared memory: thread e puts its 64 heads' values of dim d
+        // into a [head][dim] staging tile in the P buffers (free: the item's last
+        // PV has retired), then the 128 threads store whole 16-byte pieces of the
+        // head rows (fp32 tiles in two 64-dim halves).
+        if (EPI == EPI_COMBINE && p.out_bf16) {
+          __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sP);          // [64][128]
+          named_bar_sync(1, 128);             // exchange reads / previous tile's stores done
 #pragma unroll
-            for (int h = 0; h < 64; ++h)
-              if (h < p.H) dst[(int64_t)h * D] = __float2bfloat16_rn(o[h]);
-          } else {
-            float* dst = reinterpret_cast<float*>(p.out) + obase * D + d;
-#pragma unroll
-            for (int h = 0; h < 64; ++h)
-              if (h < p.H) dst[(int64_t)h * D] = o[h];
+          for (int h = 0; h < 64; ++h) stg[h * 128 + e] = __float2bfloat16_rn(o[h]);
+          named_bar_sync(1, 128);
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + obase * D + 128 * tt;
+#pragma unroll 4
+          for (int q = e; q < 64 * 16; q += 128) {
+            const int h = q >> 4, c = q & 15;
+            if (h < p.H)
+              *reinterpret_cast<uint4*>(dst + (int64_t)h * D + 8 * c) = *reinterpret_cast<const uint4*>(stg + h * 128 + 8 * c);
           }
+          named_bar_sync(1, 128);             // staging read out before the next tile's exchange reuses it
         } else {
-          float* dst = p.O_part + obase * D + d;
+          float* stg = reinterpret_cast<float*>(sP);                          // [64][64]
+          float* dst = (EPI == EPI_COMBINE ? reinterpret_cast<float*>(p.out) : p.O_part) + obase * D + 128 * tt;
+#pragma unroll 1
+          for (int hf = 0; hf < 2; ++hf) {
+            named_bar_sync(1, 128);
+            if ((e >> 6) == hf) {
 #pragma unroll
-          for (int h = 0; h < 64; ++h)
-            if (h < p.H) dst[(int64_t)h * D] = o[h];
+              for (int h = 0; h < 64; ++h) stg[h * 64 + (e & 63)] = o[h];
+            }
+            named_bar_sync(1, 128);
+#pragma unroll 4
+            for (int q = e; q < 64 * 16; q += 128) {
+              const int h = q >> 4, c = q & 15;
+              if (h < p.H)
+                *reinterpret_cast<float4*>(dst + (int64_t)h * D + 64 * hf + 4 * c) =
+                    *reinterpret_cast<const float4*>(stg + h * 64 + 4 * c);
+            }
+          }
+          named_bar_sync(1, 128);             // staging read out before the next tile's exchange reuses it
         }
       }
       ++icount;
