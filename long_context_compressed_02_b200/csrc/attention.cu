@@ -968,44 +968,23 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
             o[h] = first ? o[h] * csj.x + w * csj.y : o[h] * csj.x - w * csj.y;
           }
         }
-        // Out through shared memory: thread e puts its 64 heads' values of dim d
-        // into a [head][dim] staging tile in the P buffers (free: the item's last
-        // PV has retired), then the 128 threads store whole 16-byte pieces of the
-        // head rows (fp32 tiles in two 64-dim halves).
-        if (EPI == EPI_COMBINE && p.out_bf16) {
-          __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(sP);          // [64][128]
-          named_bar_sync(1, 128);             // exchange reads / previous tile's stores done
+        if (EPI == EPI_COMBINE) {
+          if (p.out_bf16) {
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + obase * D + d;
 #pragma unroll
-          for (int h = 0; h < 64; ++h) stg[h * 128 + e] = __float2bfloat16_rn(o[h]);
-          named_bar_sync(1, 128);
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + obase * D + 128 * tt;
-#pragma unroll 4
-          for (int q = e; q < 64 * 16; q += 128) {
-            const int h = q >> 4, c = q & 15;
-            if (h < p.H)
-              *reinterpret_cast<uint4*>(dst + (int64_t)h * D + 8 * c) = *reinterpret_cast<const uint4*>(stg + h * 128 + 8 * c);
+            for (int h = 0; h < 64; ++h)
+              if (h < p.H) dst[(int64_t)h * D] = __float2bfloat16_rn(o[h]);
+          } else {
+            float* dst = reinterpret_cast<float*>(p.out) + obase * D + d;
+#pragma unroll
+            for (int h = 0; h < 64; ++h)
+              if (h < p.H) dst[(int64_t)h * D] = o[h];
           }
-          named_bar_sync(1, 128);             // staging read out before the next tile's exchange reuses it
         } else {
-          float* stg = reinterpret_cast<float*>(sP);                          // [64][64]
-          float* dst = (EPI == EPI_COMBINE ? reinterpret_cast<float*>(p.out) : p.O_part) + obase * D + 128 * tt;
-#pragma unroll 1
-          for (int hf = 0; hf < 2; ++hf) {
-            named_bar_sync(1, 128);
-            if ((e >> 6) == hf) {
+          float* dst = p.O_part + obase * D + d;
 #pragma unroll
-              for (int h = 0; h < 64; ++h) stg[h * 64 + (e & 63)] = o[h];
-            }
-            named_bar_sync(1, 128);
-#pragma unroll 4
-            for (int q = e; q < 64 * 16; q += 128) {
-              const int h = q >> 4, c = q & 15;
-              if (h < p.H)
-                *reinterpret_cast<float4*>(dst + (int64_t)h * D + 64 * hf + 4 * c) =
-                    *reinterpret_cast<const float4*>(stg + h * 64 + 4 * c);
-            }
-          }
-          named_bar_sync(1, 128);             // staging read out before the next tile's exchange reuses it
+          for (int h = 0; h < 64; ++h)
+            if (h < p.H) dst[(int64_t)h * D] = o[h];
         }
       }
       ++icount;
