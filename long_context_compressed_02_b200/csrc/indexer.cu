@@ -218,7 +218,7 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
 // the e4m3 operand ring, and the key row scales reach the epilogue through
 // shared memory.  FP8: tmap_ks is unused.
 template <bool FP4, int NST>
-__global__ void __launch_bounds__(FP4 ? kIdxThreadsFp4 : kIdxThreads, FP4 ? 1 : 2)
+__global__ void __launch_bounds__(FP4 ? kIdxThreadsFp4 : kIdxThreads, (FP4 || NST != kStagesPair) ? 1 : 2)
 indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_ks, IdxParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -468,7 +468,41 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
         }
         const uint32_t tb = tmem + ((uint32_t)(sp * 32) << 16) + acc * p.N;
         float run = 0.f;
-        for (int cc = 0; cc < p.N; cc += 32) {
+        // One CTA per SM (wide query blocks, prefill): registers for 64 columns,
+        // so a tile's 256 columns take four TMEM round trips instead of eight.
+        constexpr bool kWide = !FP4 && NST != kStagesPair;
+        if (kWide && p.HI >= 32) {
+          for (int cc0 = 0; cc0 < p.N; cc0 += 64) {
+            float v[64];
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+              if (cc0 + 32 * q < p.N) tmem_ld32(tb + cc0 + 32 * q, v + 32 * q);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int cc = cc0 + 32 * q;
+              if (cc < p.N) {
+                // w * ReLU(x) summed by fused multiply-adds into four partial sums
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 w4 = ld_shared_f4(w_addr + (cc + 4 * i) * 4);
+                  a0 = fmaf(w4.x, fmaxf(v[32 * q + 4 * i + 0], 0.f), a0);
+                  a1 = fmaf(w4.y, fmaxf(v[32 * q + 4 * i + 1], 0.f), a1);
+                  a2 = fmaf(w4.z, fmaxf(v[32 * q + 4 * i + 2], 0.f), a2);
+                  a3 = fmaf(w4.w, fmaxf(v[32 * q + 4 * i + 3], 0.f), a3);
+                }
+                run += (a0 + a1) + (a2 + a3);
+                if (((cc + 32) & (p.HI - 1)) == 0) {
+                  const int tq = (cc + 31) >> log2hi;
+                  if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = run * ksc_use;
+                  run = 0.f;
+                }
+              }
+            }
+          }
+        }
+        for (int cc = 0; cc < (kWide && p.HI >= 32 ? 0 : p.N); cc += 32) {
           float v[32];
           tmem_ld32(tb + cc, v);
           tmem_wait_ld();
