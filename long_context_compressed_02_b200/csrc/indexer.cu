@@ -792,10 +792,21 @@ topk_hist_kernel(TopkParams p) {
   const int64_t lo = (int64_t)chunk * kChunk;
   const int n = (int)max((int64_t)0, min((int64_t)kChunk, nv - lo));
   if (n == 0) return;
+  // every key of this thread is loaded first (one memory latency for the
+  // chunk), the histogram cleared meanwhile
+  constexpr int kPer = kChunk / kTopkThreads;   // 32
+  const float* src = p.scores + row * p.cap + lo;
+  uint32_t bin[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int e = threadIdx.x + kTopkThreads * j;
+    bin[j] = e < n ? order_key(__ldcg(src + e)) >> 20 : 0xffffffffu;
+  }
   for (int i = threadIdx.x; i < kHistBins; i += kTopkThreads) h[i] = 0;
   __syncthreads();
-  const float* src = p.scores + row * p.cap + lo;
-  for (int e = threadIdx.x; e < n; e += kTopkThreads) atomicAdd(&h[order_key(src[e]) >> 20], 1u);
+#pragma unroll
+  for (int j = 0; j < kPer; ++j)
+    if (bin[j] != 0xffffffffu) atomicAdd(&h[bin[j]], 1u);
   __syncthreads();
   uint32_t* g = p.hist + row * kHistBins;
   for (int i = threadIdx.x; i < kHistBins; i += kTopkThreads)
