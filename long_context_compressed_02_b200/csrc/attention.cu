@@ -1003,11 +1003,11 @@ attn_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtens
 // Split-KV merge: each token's n_split partials (O normalised by its own sum,
 // lse) and the sink in one softmax, then the inverse RoPE of the output.
 // One CTA per token; 16-byte vector loads and stores along d.
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 attn_merge_kernel(const float* __restrict__ Os, const float* __restrict__ Ls, const float* __restrict__ sink,
                   const int64_t* __restrict__ q_pos, int T, int n_split, int H, int D, int inv_rope, int rope_dim,
                   float rope_base, void* __restrict__ out, int out_bf16) {
-  constexpr int kHeads = 8;                       // heads per CTA (blockIdx.y selects the group)
+  constexpr int kHeads = 4;                       // heads per CTA (blockIdx.y selects the group): one warp each
   __shared__ float s_coef[kHeads][kMaxSplit];
   __shared__ int s_act[kMaxSplit];                // splits with a nonzero weight for some head of the group
   __shared__ int s_nact;
@@ -1520,7 +1520,7 @@ extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q
   const int64_t toks = (int64_t)n_seq * T;
   if (toks == 0) return CSA_OK;
   CSA_REQUIRE(toks <= 0x7fffffff, "csa_fused_attention_splitkv: too many tokens");
-  cudaError_t le = launch_pdl(attn_merge_kernel, dim3((unsigned)toks, (unsigned)((H + 7) / 8)), dim3(256), 0, stream,
+  cudaError_t le = launch_pdl(attn_merge_kernel, dim3((unsigned)toks, (unsigned)((H + 3) / 4)), dim3(128), 0, stream,
                               (const float*)Os, (const float*)Ls, sink, q_pos, T, n_split, H, D, inv_rope, rope_dim,
                               rope_base, out, (int)(out_dtype == CSA_BF16));
   if (le != cudaSuccess)
