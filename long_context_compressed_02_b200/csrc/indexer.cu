@@ -80,6 +80,8 @@ struct IdxParams {
   int T, HI, DI, m, TQ, N, tiles_per_chunk;
   int n_seq, n_qblocks;
   int64_t n_items;        // n_seq x n_qblocks x key chunks
+  int chunk_small;        // > 0: rows of unequal length take chunks of this many tiles (decided on the
+                          // device from the visible lengths), so the last items are short
   uint32_t* item_counter; // zeroed before the launch: items are claimed dynamically
   uint32_t* hist_zero;    // non-null: [hist_words] histogram words this grid zeroes
   int64_t hist_words;
@@ -93,7 +95,7 @@ struct IdxItem {
   int b, t0, tile0, n_tiles;
   int64_t pos0;
 };
-__device__ __forceinline__ IdxItem idx_item(const IdxParams& p, int64_t item) {
+__device__ __forceinline__ IdxItem idx_item(const IdxParams& p, int64_t item, int tiles_per_chunk) {
   IdxItem r;
   r.b = (int)(item % p.n_seq);
   const int64_t rest = item / p.n_seq;
@@ -104,8 +106,8 @@ __device__ __forceinline__ IdxItem idx_item(const IdxParams& p, int64_t item) {
   r.pos0 = p.q_pos[r.b];
   const int64_t nv_max = min(p.cap, (r.pos0 + t_last + 1) / p.m);
   const int n_tiles_all = (int)((nv_max + 127) / 128);
-  r.tile0 = chunk * p.tiles_per_chunk;
-  r.n_tiles = max(0, min(n_tiles_all - r.tile0, p.tiles_per_chunk));
+  r.tile0 = chunk * tiles_per_chunk;
+  r.n_tiles = max(0, min(n_tiles_all - r.tile0, tiles_per_chunk));
   return r;
 }
 
@@ -279,12 +281,45 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     *s_abort = 0;
     fence_mbar_init();
   }
+  // Rows of unequal visible length (decode over sequences of different
+  // contexts): the producer warp sums the rows' key tiles; unless the rows are
+  // nearly equal, items take the small chunk, so that the grid's last items are
+  // short and the CTAs finish together.
+  __shared__ int s_chunk;
+  __shared__ long long s_nitems;
+  if (warp == 0 && p.chunk_small > 0) {
+    const int64_t rb = (int64_t)p.n_seq * p.n_qblocks;
+    long long tot = 0;
+    int mx = 0;
+    for (int64_t r = lane; r < rb; r += 32) {
+      const int b = (int)(r % p.n_seq);
+      const int qb = p.n_qblocks - 1 - (int)((r / p.n_seq) % p.n_qblocks);
+      const int t_last = min(p.T, qb * p.TQ + p.TQ) - 1;
+      const int64_t nv = min(p.cap, (p.q_pos[b] + t_last + 1) / p.m);
+      const int tl = (int)((nv + 127) / 128);
+      tot += tl;
+      mx = max(mx, tl);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      tot += __shfl_xor_sync(0xffffffffu, tot, o);
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+      const bool uniform = tot * 10 >= 9 * rb * (long long)mx;
+      const int c = uniform ? p.tiles_per_chunk : p.chunk_small;
+      s_chunk = c;
+      s_nitems = rb * (long long)((mx + c - 1) / c);
+    }
+  }
   if (warp == 1) tmem_alloc(s_tmem, tmem_cols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   volatile int* abort_flag = s_abort;
+  const int chunk_t = p.chunk_small > 0 ? s_chunk : p.tiles_per_chunk;
+  const int64_t n_items = p.chunk_small > 0 ? (int64_t)s_nitems : p.n_items;
 
   // Non-empty items are claimed from a global counter by the producer warp (so
   // CTAs that drew short rows take more items), which also fills the slot's
@@ -294,16 +329,16 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   // it has finished the item's tiles.  Whole-warp call for the producer.
   auto claim_item = [&](uint32_t k) {
     const uint32_t slot = k & 3, par = (k >> 2) & 1;
-    int64_t item = p.n_items;
+    int64_t item = n_items;
     if (lane == 0 && wait_bar(&iempty[slot], par ^ 1, abort_flag)) {
       for (;;) {
         item = (int64_t)atomicAdd(p.item_counter, 1u);
-        if (item >= p.n_items || idx_item(p, item).n_tiles > 0) break;
+        if (item >= n_items || idx_item(p, item, chunk_t).n_tiles > 0) break;
       }
     }
     item = __shfl_sync(0xffffffffu, item, 0);
-    if (item < p.n_items) {
-      const IdxItem it = idx_item(p, item);
+    if (item < n_items) {
+      const IdxItem it = idx_item(p, item, chunk_t);
       float* gw = s_w + slot * p.N;
       int* gnv = s_nv + slot * p.TQ;
       for (int c = lane; c < p.N; c += 32) {
@@ -327,7 +362,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   };
   auto read_item = [&](uint32_t k) -> int64_t {
     const uint32_t slot = k & 3, par = (k >> 2) & 1;
-    return wait_bar(&ifull[slot], par, abort_flag) ? s_items[slot] : p.n_items;
+    return wait_bar(&ifull[slot], par, abort_flag) ? s_items[slot] : n_items;
   };
   auto release_item = [&](uint32_t k) { mbar_arrive(&iempty[k & 3]); };
 
@@ -349,9 +384,9 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       bool ok = true;
       for (uint32_t kk = 0; ok; ++kk) {
         const int64_t item = claim_item(kk);
-        if (item >= p.n_items) break;
+        if (item >= n_items) break;
         if (lane == 0) {
-          const IdxItem it = idx_item(p, item);
+          const IdxItem it = idx_item(p, item, chunk_t);
           const uint32_t qs = ic & 1;
           if (!wait_bar(&qempty[qs], ((ic >> 1) & 1) ^ 1, abort_flag)) ok = false;
           if (ok) {
@@ -390,8 +425,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       for (uint32_t kk = 0; ok; ++kk) {
         const int64_t item = read_item(kk);
         release_item(kk);
-        if (item >= p.n_items) break;
-        const IdxItem it = idx_item(p, item);
+        if (item >= n_items) break;
+        const IdxItem it = idx_item(p, item, chunk_t);
         const uint32_t qs = ic & 1;
         if (!wait_bar(&qfull[qs], (ic >> 1) & 1, abort_flag)) { ok = false; break; }
         const uint64_t dB = dB0 + ((qs * b_stride) >> 4);
@@ -434,12 +469,12 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     bool ok = true;
     for (uint32_t kk = 0; ok; ++kk) {
       const int64_t item = read_item(kk);
-      if (item >= p.n_items) {
+      if (item >= n_items) {
         __syncwarp();
         if (lane == 0) release_item(kk);
         break;
       }
-      const IdxItem it = idx_item(p, item);
+      const IdxItem it = idx_item(p, item, chunk_t);
       // the slot's column weights and visible-entry counts (filled by the producer)
       const float* gw = s_w + (kk & 3) * p.N;
       const int* gnv = s_nv + (kk & 3) * p.TQ;
@@ -578,12 +613,12 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     bool ok = true;
     for (uint32_t kk = 0; ok; ++kk) {
       const int64_t item = read_item(kk);
-      if (item >= p.n_items) {
+      if (item >= n_items) {
         __syncwarp();
         if (lane == 0) release_item(kk);
         break;
       }
-      const IdxItem it = idx_item(p, item);
+      const IdxItem it = idx_item(p, item, chunk_t);
       for (int j = 0; j < it.n_tiles; ++j, ++gt) {
         const int s = gt % NST, o = gt % kOpStages, r = gt % kRsSlots;
         if (!wait_bar(&full[s], (gt / NST) & 1, abort_flag)) { ok = false; break; }
@@ -1078,6 +1113,9 @@ csa_status_t index_topk_run(const uint8_t* qI, const float* qI_scale, const floa
   if (rows_blocks < 2 * (int64_t)sms)
     chunk_tiles = std::max<int64_t>(8, std::min<int64_t>(tiles, (rows_blocks * tiles + 4 * sms - 1) / (4 * sms)));
   ip.tiles_per_chunk = (int)chunk_tiles;
+  // decode: chunks of about 16 per SM for rows of unequal length (decided on the device)
+  if (rows_blocks < 2 * (int64_t)sms)
+    ip.chunk_small = (int)std::max<int64_t>(8, std::min<int64_t>(tiles, (rows_blocks * tiles + 16 * sms - 1) / (16 * sms)));
   const int64_t n_kchunks = (tiles + chunk_tiles - 1) / chunk_tiles;
   ip.n_seq = n_seq; ip.n_qblocks = n_qblocks;
   ip.n_items = rows_blocks * n_kchunks;
