@@ -188,8 +188,8 @@ csa_status_t csa_cache_append(const void* c_tok, const void* z_tok, csa_dtype_t 
  *   workspace / ws_bytes: at least csa_index_topk_workspace(n_seq, T, cap, k)
  *            bytes, 16-byte aligned, owned by the caller: the fp32 score matrix,
  *            for rows longer than 16384 entries the per-chunk candidates and a
- *            key histogram per row (zeroed by the call's first kernel), and the
- *            work-item counter (reset by the call with a stream-ordered memset).
+ *            key histogram per row, and the work-item counter (the histograms
+ *            and the counter are reset by the call with one stream-ordered memset).
  *            Contents are undefined afterwards; calls sharing one workspace must
  *            be ordered on one stream.  The selection kernels are launched as
  *            dependents of the scoring kernel (programmatic dependent launch):
@@ -224,9 +224,9 @@ csa_status_t csa_index_topk(const uint8_t* qI, const float* qI_scale, const floa
  * cudaDeviceReset gets a fresh lookup); make that first call before any stream
  * capture.  Every call on a device shares the same array, which keeps the
  * previous call's contents: the call resets the work-item counter it uses
- * (a stream-ordered memset inside the array) and, for rows longer than 16384
- * entries, its key histograms (zeroed by its first kernel before they are
- * filled), and it reads only score entries it has written itself, so earlier
+ * and, for rows longer than 16384 entries, its key histograms (one
+ * stream-ordered memset inside the array before they are filled), and it
+ * reads only score entries it has written itself, so earlier
  * contents never reach the result.  Calls that may overlap
  * on the GPU (different streams, or host threads racing) race on the array and
  * must be serialised by the caller.  No memory is allocated or freed.

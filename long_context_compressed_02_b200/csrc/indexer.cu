@@ -22,7 +22,9 @@
 // shared memory by an 8-bit radix select (starting below the bits every key
 // shares) followed by an order-preserving compaction, so the result is
 // ascending, deterministic, and ties go to the lower entry index.  Longer
-// rows first build a histogram of the top 12 key bits; the threshold bin it
+// rows first build a histogram of the top 12 key bits (in the scores
+// kernel's epilogue when each work item holds one token, as in decode;
+// otherwise in a separate pass over the scores); the threshold bin it
 // gives bounds the row's k-th largest key from below, so each 16384-entry
 // chunk keeps only keys at or above it (exact: the global top-k restricted to
 // a chunk is among them), selects locally only if more than k survive, and
@@ -69,6 +71,16 @@ constexpr uint32_t kFp4Codes = 128 * 64;  // packed E2M1 codes of a 128-key tile
 constexpr uint32_t kFp4Stage = kFp4Codes + 128 * 4;   // + one E8M0 byte per 32-element block
 constexpr int kStages = 8;           // key-tile ring depth, one CTA per SM (deeper rings measured no faster)
 constexpr int kStagesPair = 5;       // ring depth when two CTAs share an SM (small query tiles: decode)
+constexpr int kHistBins = 4096;      // rows split into top-k chunks: histogram of the top 12 key bits
+constexpr int kHistItemTiles = 511;  // key tiles per item when the scores kernel builds the histograms:
+                                     // an item's count per bin then fits the 16 bits it has in shared memory
+
+// Total order of fp32 scores as unsigned keys (larger score, larger key).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f + 0.0f);   // -0 -> +0 so that equal values tie
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 
 struct IdxParams {
   const float* qs;        // [n_seq, T, HI] or null
@@ -83,8 +95,9 @@ struct IdxParams {
   int chunk_small;        // > 0: rows of unequal length take chunks of this many tiles (decided on the
                           // device from the visible lengths), so the last items are short
   uint32_t* item_counter; // zeroed before the launch: items are claimed dynamically
-  uint32_t* hist_zero;    // non-null: [hist_words] histogram words this grid zeroes
-  int64_t hist_words;
+  uint32_t* hist;         // non-null (one token per item, rows split into top-k chunks): the epilogue
+                          // adds every visible key to its row's [kHistBins] histogram of the top 12
+                          // order-key bits (zeroed before the launch)
 };
 
 // One work item of the persistent scores kernel: a key chunk of one token
@@ -227,14 +240,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   // aligned by offsetting the shared array itself, so accesses stay in the shared window
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // the selection kernels may start launching; they wait for this grid's end.
-  // Rows split into chunks: this grid zeroes their key histograms (filled by
-  // the next kernel), in place of a separate memset.
+  // the selection kernels may start launching; they wait for this grid's end
   pdl_trigger();
-  if (p.hist_zero) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + tid; i < p.hist_words; i += (int64_t)gridDim.x * blockDim.x)
-      p.hist_zero[i] = 0u;
-  }
 
   const uint32_t a_bytes = 128u * p.DI;
   const uint32_t b_bytes = (uint32_t)p.N * p.DI;
@@ -254,7 +261,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   uint64_t* opfull = iempty + 4;         // [kOpStages] FP4 only
   uint64_t* opempty = opfull + kOpStages;
   uint64_t* rsfull = opempty + kOpStages;   // [kRsSlots]
-  int64_t* s_items = reinterpret_cast<int64_t*>(rsfull + kRsSlots);   // [4]
+  uint64_t* hbar = rsfull + kRsSlots;    // [2] item's keys counted / its histogram flushed
+  int64_t* s_items = reinterpret_cast<int64_t*>(hbar + 2);   // [4]
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_items + 4);
   int* s_abort = reinterpret_cast<int*>(s_tmem + 1);
   // per item-ring slot: visible entries per token, column weights w * qs
@@ -262,6 +270,11 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
   float* s_w = reinterpret_cast<float*>(
       (reinterpret_cast<uintptr_t>(s_nv + 4 * p.TQ) + 15) & ~uintptr_t(15));   // [4][N]
   float* s_rs = s_w + 4 * p.N;                                // FP4: [kRsSlots][128] key row scales
+  // p.hist: the current item's key histogram, two 16-bit bins per word (not
+  // compiled into the one-CTA-per-SM FP8 instance, which serves wide token blocks)
+  constexpr bool kHist = FP4 || NST == kStagesPair;
+  const bool hist_on = kHist && p.hist != nullptr;
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(s_rs + (FP4 ? kRsSlots * 128 : 0));
 
   const uint32_t tmem_cols = p.N <= 16 ? 32u : (p.N <= 32 ? 64u : (p.N <= 64 ? 128u : (p.N <= 128 ? 256u : 512u)));
   if (tid == 0) {
@@ -278,6 +291,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       mbar_init(&ifull[i], 32);
       mbar_init(&iempty[i], 1 + kEpiThreads / 32 + (FP4 ? kConvThreads / 32 : 0));
     }
+    mbar_init(&hbar[0], kEpiThreads);
+    mbar_init(&hbar[1], kEpiThreads);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -312,6 +327,8 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       s_nitems = rb * (long long)((mx + c - 1) / c);
     }
   }
+  if (hist_on)
+    for (int i = tid; i < kHistBins / 2; i += blockDim.x) s_hist[i] = 0u;
   if (warp == 1) tmem_alloc(s_tmem, tmem_cols);
   tc_fence_before();
   __syncthreads();
@@ -465,7 +482,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
     const int grp = ew >> 2;
     const int log2hi = __ffs(p.HI) - 1;
     const int key_in_tile = sp * 32 + lane;
-    uint32_t gt = 0;
+    uint32_t gt = 0, hn = 0;
     bool ok = true;
     for (uint32_t kk = 0; ok; ++kk) {
       const int64_t item = read_item(kk);
@@ -479,6 +496,16 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
       const float* gw = s_w + (kk & 3) * p.N;
       const int* gnv = s_nv + (kk & 3) * p.TQ;
       const uint32_t w_addr = smem_u32(gw);
+      // a visible key's score; with p.hist it is also counted in the item's histogram
+      auto put = [&](int tq, int64_t key, float sv) {
+        if (key < gnv[tq]) {
+          p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = sv;
+          if (hist_on) {
+            const uint32_t bin = order_key(sv) >> 20;
+            atomicAdd(&s_hist[bin >> 1], 1u << ((bin & 1u) << 4));
+          }
+        }
+      };
       // this group's tiles of the item: global tile numbers gt with gt % 2 == grp
       const int j0 = ((int)(gt & 1) == grp) ? 0 : 1;
       auto key_scale = [&](int j) -> float {
@@ -530,7 +557,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
                 run += (a0 + a1) + (a2 + a3);
                 if (((cc + 32) & (p.HI - 1)) == 0) {
                   const int tq = (cc + 31) >> log2hi;
-                  if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = run * ksc_use;
+                  put(tq, key, run * ksc_use);
                   run = 0.f;
                 }
               }
@@ -557,7 +584,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             run += (a0 + a1) + (a2 + a3);
             if (((cc + 32) & (p.HI - 1)) == 0) {
               const int tq = (cc + 31) >> log2hi;
-              if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = run * ksc_use;
+              put(tq, key, run * ksc_use);
               run = 0.f;
             }
             continue;
@@ -584,7 +611,7 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             run += pr[0];
             if (((cc + 32) & (p.HI - 1)) == 0) {
               const int tq = (cc + 31) >> log2hi;
-              if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = run * ksc_use;
+              put(tq, key, run * ksc_use);
               run = 0.f;
             }
           } else {
@@ -592,13 +619,35 @@ indexer_scores_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_c
             for (int jj = 0; jj < 32; ++jj) {
               if ((jj & (p.HI - 1)) == 0) {
                 const int tq = (cc + jj) >> log2hi;
-                if (key < gnv[tq]) p.scores[((int64_t)it.b * p.T + it.t0 + tq) * p.cap + key] = pr[jj] * ksc_use;
+                put(tq, key, pr[jj] * ksc_use);
               }
             }
           }
         }
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
+      }
+      if (hist_on && ok) {
+        // Once all 256 epilogue threads have counted the item's keys, its
+        // nonzero bins go to the row's histogram in global memory and are
+        // cleared; the next item's counting starts after every flush.
+        const uint32_t hp = hn & 1u;
+        mbar_arrive(&hbar[0]);
+        if (!wait_bar(&hbar[0], hp, abort_flag)) ok = false;
+        if (ok) {
+          uint32_t* g = p.hist + ((int64_t)it.b * p.T + it.t0) * kHistBins;
+          for (int i = ew * 32 + lane; i < kHistBins / 2; i += kEpiThreads) {
+            const uint32_t v = s_hist[i];
+            if (v) {
+              s_hist[i] = 0u;
+              if (v & 0xffffu) atomicAdd(g + 2 * i, v & 0xffffu);
+              if (v >> 16) atomicAdd(g + 2 * i + 1, v >> 16);
+            }
+          }
+          mbar_arrive(&hbar[1]);
+          if (!wait_bar(&hbar[1], hp, abort_flag)) ok = false;
+        }
+        ++hn;
       }
       __syncwarp();
       if (lane == 0) release_item(kk);       // this warp is done with the slot's weights
@@ -661,12 +710,6 @@ constexpr int kTopkThreads = 512;      // histogram, filtered-chunk and merge ke
 constexpr int kTopkThreadsSmall = 256; // rows of one chunk: smaller CTAs, twice as many in flight
 constexpr int kChunk = 16384;          // keys per shared-memory chunk (64 KB)
 constexpr int kMergeCap = 16384;       // candidates per row in the merge stage
-constexpr int kHistBins = 4096;        // rows split into chunks: histogram of the top 12 key bits
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f + 0.0f);   // -0 -> +0 so that equal values tie
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 template <int NTH>
 struct SelectSmem {
@@ -813,12 +856,14 @@ struct TopkParams {
   uint32_t* hist;          // [rows, kHistBins] (rows split into chunks)
 };
 
-// Rows split into chunks, pass 1: histogram of the top 12 bits of every
-// visible key of the row, one CTA per (row, chunk), merged in global memory.
+// Rows split into chunks whose histograms the scores kernel did not build
+// (several tokens per work item), pass 1: histogram of the top 12 bits of
+// every visible key of the row, one CTA per (row, chunk), merged in global
+// memory.
 __global__ void __launch_bounds__(kTopkThreads)
 topk_hist_kernel(TopkParams p) {
   __shared__ uint32_t h[kHistBins];
-  pdl_wait();                              // the scores (and the zeroed histograms) are complete
+  pdl_wait();                              // the scores are complete (histograms zeroed before them)
   pdl_trigger();
   const int64_t row = blockIdx.x;
   const int chunk = blockIdx.y;
@@ -1112,10 +1157,16 @@ csa_status_t index_topk_run(const uint8_t* qI, const float* qI_scale, const floa
   int64_t chunk_tiles = tiles;
   if (rows_blocks < 2 * (int64_t)sms)
     chunk_tiles = std::max<int64_t>(8, std::min<int64_t>(tiles, (rows_blocks * tiles + 4 * sms - 1) / (4 * sms)));
+  // one token per item and rows split into top-k chunks: the scores kernel
+  // builds the rows' key histograms (items of at most kHistItemTiles tiles)
+  bool hist_fused = L.n_chunks > 1 && TQ == 1;
+  if (hist_fused) chunk_tiles = std::min<int64_t>(chunk_tiles, kHistItemTiles);
   ip.tiles_per_chunk = (int)chunk_tiles;
   // decode: chunks of about 16 per SM for rows of unequal length (decided on the device)
-  if (rows_blocks < 2 * (int64_t)sms)
+  if (rows_blocks < 2 * (int64_t)sms) {
     ip.chunk_small = (int)std::max<int64_t>(8, std::min<int64_t>(tiles, (rows_blocks * tiles + 16 * sms - 1) / (16 * sms)));
+    if (hist_fused) ip.chunk_small = std::min(ip.chunk_small, kHistItemTiles);
+  }
   const int64_t n_kchunks = (tiles + chunk_tiles - 1) / chunk_tiles;
   ip.n_seq = n_seq; ip.n_qblocks = n_qblocks;
   ip.n_items = rows_blocks * n_kchunks;
@@ -1137,17 +1188,17 @@ csa_status_t index_topk_run(const uint8_t* qI, const float* qI_scale, const floa
     const size_t tiles_bytes = fp4 ? (size_t)kOpStages * 128 * DI + (size_t)stages * kFp4Stage
                                    : (size_t)stages * 128 * DI;
     return 1024 + 2 * (((size_t)N * DI + 1023) / 1024) * 1024 + tiles_bytes +
-           (2 * kStages + 16 + 2 * kOpStages + kRsSlots) * 8 + 4 * 8 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4 +
-           (fp4 ? (size_t)kRsSlots * 128 * 4 : 0);
+           (2 * kStages + 18 + 2 * kOpStages + kRsSlots) * 8 + 4 * 8 + 8 + 4 * TQ * 4 + 16 + 4 * N * 4 +
+           (fp4 ? (size_t)kRsSlots * 128 * 4 : 0) + (hist_fused ? (size_t)kHistBins * 2 : 0);
   };
   ip.item_counter = reinterpret_cast<uint32_t*>(ws + L.counter);
+  if (hist_fused) ip.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
   {
-    cudaError_t e = cudaMemsetAsync(ip.item_counter, 0, sizeof(uint32_t), stream);
+    // the item counter, and with rows split into chunks the key histograms just
+    // before it in the layout, start at zero
+    const size_t first = L.n_chunks > 1 ? L.hist : L.counter;
+    cudaError_t e = cudaMemsetAsync(ws + first, 0, L.counter + sizeof(uint32_t) - first, stream);
     if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_index_topk: counter reset failed: %s", cudaGetErrorString(e));
-  }
-  if (L.n_chunks > 1) {
-    ip.hist_zero = reinterpret_cast<uint32_t*>(ws + L.hist);
-    ip.hist_words = (int64_t)n_seq * T * kHistBins;
   }
   if (fp4) {
     const size_t smem = smem_for(kStages);
@@ -1166,6 +1217,10 @@ csa_status_t index_topk_run(const uint8_t* qI, const float* qI_scale, const floa
     cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
     cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev);
     const bool pair = 2 * tmem_cols <= 512 && 2 * (smem_pair + (size_t)smem_rsv) <= (size_t)smem_sm;
+    if (!pair && hist_fused) {            // that instance has no histogram epilogue
+      hist_fused = false;
+      ip.hist = nullptr;
+    }
     if (pair) {
       cudaFuncSetAttribute(indexer_scores_kernel<false, kStagesPair>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem_pair);
@@ -1205,7 +1260,7 @@ csa_status_t index_topk_run(const uint8_t* qI, const float* qI_scale, const floa
     if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
     return check_launch(what);
   };
-  if (L.n_chunks > 1) {
+  if (L.n_chunks > 1 && !hist_fused) {
     st = launched(launch_pdl(topk_hist_kernel, g1, dim3(kTopkThreads), 0, stream, tp), "csa_index_topk(histogram)");
     if (st != CSA_OK) return st;
   }

@@ -277,3 +277,45 @@ def test_f32_path_fused_with_window_sink_and_inverse_rope(H, D, n_split, dense):
                                   rope_dim=64, out_dtype=torch.float32, n_split=n_split)
     csa.check_device_error()
     assert_close(host(out)[0], ref, max_abs=MAX_ABS_F32, rel_l2=REL_L2_F32, what="fp32 fused attention")
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_growing_logits_lazy_rescale(fused):
+    """Unit-RMS entries (and window rows) lean more and more on one direction u
+    along the visit order, the heads lean on u by different amounts, and one
+    head per token points at a late entry: the running maxima of later half
+    chunks jump by more than the lazy-rescale threshold (a factor 2^8) for some
+    columns and rise by less for others (these keep the old maximum, so their
+    probabilities exceed 1).  Both branches run against the oracle."""
+    import long_context_compressed_02_b200 as csa
+    rng = np.random.default_rng(31)
+    T, ne, H, D, k, W = 200, 1000, 64, 512, 512, 128
+    u = rng.standard_normal(D)
+
+    def leaning(n):
+        a = 6.0 * (np.arange(n) / n) ** 2
+        return O.rmsnorm(a[:, None] * u[None] + rng.standard_normal((n, D)))
+
+    kv = synth.to_bf16_values(leaning(ne))
+    kt = synth.to_bf16_values(leaning(T))
+    idx = _rand_idx(rng, T, k, ne, [512, 300, 129, 64])
+    beta = np.linspace(0, 3, H)
+    q = O.rmsnorm(beta[None, :, None] * u[None, None] + rng.standard_normal((T, H, D)))
+    for t in range(T):
+        n = int((idx[t] >= 0).sum())
+        q[t, t % H] = O.rmsnorm(kv[idx[t, n - 3]])       # one head locks onto a late entry
+    q = synth.to_bf16_values(q)
+    tq, tkv, ti = cuda(q, torch.bfloat16)[None], cuda(kv, torch.bfloat16)[None], cuda(idx)[None]
+    Or, Lr = O.sparse_attention_partial(q, kv, idx)
+    if not fused:
+        Og, Lg = csa.csa_sparse_mqa(tq, tkv, ti)
+        csa.check_device_error()
+        assert_close(host(Og)[0], Or, what="growing-logit O_part")
+        assert_close(host(Lg)[0], Lr, max_abs=1e-2, rel_l2=1e-3, what="growing-logit lse")
+        return
+    sink = rng.standard_normal(H).astype(np.float32)
+    out = csa.csa_fused_attention(tq, tkv, cuda(kt, torch.bfloat16)[None], cuda(np.array([0], np.int64)), W,
+                                  cuda(sink), idx=ti, inv_rope=True, rope_dim=64, out_dtype=torch.float32)
+    csa.check_device_error()
+    ref = O.window_sink_combine(q, kt, np.arange(T), W, sink, Or, Lr, inv_rope=True)
+    assert_close(host(out)[0], ref, what="growing-logit fused")

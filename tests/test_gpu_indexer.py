@@ -92,14 +92,17 @@ def test_ties_go_to_lower_index():
     assert np.array_equal(got[0], np.repeat(np.arange(50, dtype=np.int32)[None], T, 0))
 
 
+@pytest.mark.parametrize("HI", [8, 64])
 @pytest.mark.parametrize("mode", ["all_equal", "coarse_ties"])
-def test_long_rows_with_crowded_threshold_bin(mode):
+def test_long_rows_with_crowded_threshold_bin(mode, HI):
     """Rows of more than 16384 entries (histogram-filtered selection) where the
     threshold bin holds most of a chunk: every score equal (the filter keeps
     whole chunks and the local selection runs on all of them), or only a few
-    distinct score values (ties broken by the lower index across chunks)."""
+    distinct score values (ties broken by the lower index across chunks).
+    8 index heads put four tokens in a work item (separate histogram pass);
+    64 put one (the scores kernel counts the histogram bins itself)."""
     rng = np.random.default_rng(8)
-    n_seq, cap, HI, DI, m, k = 2, 40000, 8, 32, 4, 512
+    n_seq, cap, DI, m, k = 2, 40000, 32, 4, 512
     if mode == "all_equal":
         kI = np.repeat(synth.grid_codes(rng, (1, 1, DI)), cap, axis=1).repeat(n_seq, axis=0)
     else:
