@@ -34,10 +34,9 @@ WORKLOAD = "csa_prefill"
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
 # dominant kernels, from ncu captures of smaller cases of the same kernels scaled
 # by the units processed: the fused attention at S 4096 (507.5 MB) x 4 for
-# S 16384; the indexer scores kernel at decode batch 4 x 4 for batch 16 (not
-# yet taken for the current kernel).  Reset to None whenever one of these
-# kernels changes.
-PROFILED_TRAFFIC = {"fused_attention": 4 * 507.55e6, "index_topk": None}
+# S 16384; the indexer scores kernel at decode batch 4 (142.9 MB) x 4 for
+# batch 16.  Reset to None whenever one of these kernels changes.
+PROFILED_TRAFFIC = {"fused_attention": 4 * 507.55e6, "index_topk": 4 * 142.95e6}
 
 
 def _peaks():
