@@ -342,14 +342,15 @@ csa_status_t csa_fused_attention(const void* q, csa_dtype_t q_dtype, const void*
  * Every token's rows are cut into ranges of one common length: the longest
  * possible row set (k gathered or cap dense entries, plus the window) divided
  * by n_split, so a short token takes fewer, fuller ranges and its remaining
- * ranges are empty (lse -inf, output not written, skipped by the merge).  CTAs
- * claim (token, range) items from a counter in the workspace, so ranges of
- * sequences of unequal context balance across the GPU.
+ * ranges are empty (lse -inf, output not written, skipped by the merge).  When
+ * the (token, range) items outnumber the SMs, CTAs claim them from a counter in
+ * the workspace, so ranges of sequences of unequal context balance across the
+ * GPU; otherwise each CTA takes one item and the counter is not used.
  *   n_split in [1, 32]; workspace of csa_fused_attention_workspace(n_seq, T, H, D,
  *   n_split) bytes, 16-byte aligned, owned by the caller (partials: fp32
  *   [n_seq*T*n_split, H, D] + lse, then the item counter, reset by the call with a
- *   stream-ordered memset); calls sharing one workspace must be ordered on one
- *   stream.
+ *   stream-ordered memset when it is used); calls sharing one workspace must be
+ *   ordered on one stream.
  * ------------------------------------------------------------------------- */
 size_t csa_fused_attention_workspace(int n_seq, int T, int H, int D, int n_split);
 

@@ -40,8 +40,8 @@
 // pipe on products this small).  Each slot is refilled slab
 // pair by slab pair as the PV tile pair that read it retires, and S MMAs start
 // on a slab pair as soon as it lands.  Work items (query token, range of half
-// chunks) are taken grid-stride, or, for split-KV calls, claimed from a
-// counter so that ranges of unequal length balance.
+// chunks) are taken grid-stride, or, for split-KV calls with more items than
+// SMs, claimed from a counter so that ranges of unequal length balance.
 #include <algorithm>
 #include <cstring>
 #include <cuda_bf16.h>
@@ -1512,9 +1512,15 @@ extern "C" csa_status_t csa_fused_attention_splitkv(const void* q, csa_dtype_t q
     const int64_t nh_max = (rows1 + kRows - 1) / kRows + (rows2 + kRows - 1) / kRows;
     p.per_item = (int)std::max<int64_t>(1, (nh_max + n_split - 1) / n_split);
   }
-  p.item_counter = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(Ls) + ((parts * 4 + 255) / 256) * 256);
-  cudaError_t ce = cudaMemsetAsync(p.item_counter, 0, sizeof(uint32_t), stream);
-  if (ce != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_fused_attention_splitkv: counter reset failed: %s", cudaGetErrorString(ce));
+  // Items are claimed from a counter only when they outnumber the grid's CTAs
+  // (one per SM); otherwise CTA i takes item i, no counter reset is needed, and
+  // the attention follows the previous kernel by dependent launch directly.
+  if ((int64_t)n_seq * T * n_split > num_sms()) {
+    p.item_counter = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(Ls) + ((parts * 4 + 255) / 256) * 256);
+    cudaError_t ce = cudaMemsetAsync(p.item_counter, 0, sizeof(uint32_t), stream);
+    if (ce != cudaSuccess)
+      return fail(CSA_ERR_CUDA, "csa_fused_attention_splitkv: counter reset failed: %s", cudaGetErrorString(ce));
+  }
   s = dispatch<EPI_PARTIAL>(p, D, q_dtype, kv_dtype, tok_dtype, stream);
   if (s != CSA_OK) return s;
   const int64_t toks = (int64_t)n_seq * T;
