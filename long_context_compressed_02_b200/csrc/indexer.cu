@@ -81,7 +81,6 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-
 struct IdxParams {
   const float* qs;        // [n_seq, T, HI] or null
   const float* w;         // [n_seq, T, HI]
